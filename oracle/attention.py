@@ -1,0 +1,151 @@
+"""FP64 CPU oracle for the fused attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module: it
+is used by ``tests/``, by ``__graft_entry__.smoke()`` and by the CPU-baseline
+leg of ``bench.py``.  It shares no code with the CUDA library.
+
+What it computes is the plain definition of scaled-dot-product attention, the
+computation all the source pages turn on:
+
+    O = softmax(scale * Q K^T + mask) V
+
+* "Performance evidence" of the page "perf(metal): widen four-row flash KV
+  tiles - #89" fixes the problem statement: query rows, ``n_head`` query heads
+  sharing ``n_kv`` key/value heads, ``head_dim``, ``kv_len``, a start position
+  ``pos`` of query row 0 and a causal mask.
+* "Summary" of the same page adds a sliding-window lower bound on the keys.
+* Table "1 · Только ядро" of the page "Ядра attention на домашней RTX 5080"
+  gives the SDPA workload (1 x 40 heads x 32760 tokens x 128, bf16) against
+  which reduced-precision kernels are judged by their relative difference to
+  the full-precision result.
+
+The flash method (online softmax over key tiles) reaches exactly this result up
+to rounding order, so the oracle is the definition written out, with a library
+matmul as the only primitive and no tiling.
+
+Readings taken where the pages are silent (each is listed in the design doc):
+
+* layout ``[B, H, S, D]`` contiguous;
+* query head ``hq`` reads key/value head ``hq // (Hq // Hkv)`` (contiguous
+  groups);
+* query row ``i`` sits at absolute position ``start_pos + i``; with ``causal``
+  it sees keys ``j <= start_pos + i``;
+* ``window_lo`` is an inclusive absolute lower bound on the key index, applied
+  with or without ``causal``;
+* a row that sees no key returns O = 0 and lse = -inf;
+* ``scale`` defaults to ``1/sqrt(D)``.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def visible_range(i, *, kv_len, start_pos=0, causal=False, window_lo=0):
+    """Inclusive key range ``[lo, hi]`` seen by query row ``i`` (empty if lo > hi).
+
+    Row ``i`` is at absolute position ``start_pos + i`` (the ``pos`` of
+    "Performance evidence", page "perf(metal): widen four-row flash KV tiles").
+    """
+    lo = max(int(window_lo), 0)
+    hi = kv_len - 1
+    if causal:
+        hi = min(hi, int(start_pos) + int(i))
+    return lo, hi
+
+
+def _as_f64(x):
+    """Widen a torch tensor (bf16/fp16/fp32, any device) or array to float64."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch  # local: the oracle itself only needs numpy
+
+        x = x.to(torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def attention_f64(q, k, v, *, scale=None, causal=False, start_pos=0, window_lo=0,
+                  rows=None, return_probs=False):
+    """Attention forward in float64.
+
+    Arguments
+      q : [B, Hq, Sq, D];  k, v : [B, Hkv, Skv, D]  (any float dtype; widened exactly)
+      scale : multiplier of Q K^T (default 1/sqrt(D))
+      causal, start_pos, window_lo : mask parameters, see ``visible_range``
+      rows : optional 1-D index array of query rows to evaluate (same rows for
+             every (b, hq)); default all rows
+      return_probs : also return the softmax matrix P [B, Hq, len(rows), Skv]
+
+    Returns (O [B, Hq, R, D] float64, lse [B, Hq, R] float64[, P]) where
+    lse = natural-log of sum_j exp(scale * q.k_j) over the visible keys.
+    """
+    q = _as_f64(q)
+    k = _as_f64(k)
+    v = _as_f64(v)
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    assert Bk == B and Dk == D and v.shape == k.shape
+    assert Hq % Hkv == 0, "GQA needs n_q_heads to be a multiple of n_kv_heads"
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if rows is None:
+        rows = np.arange(Sq)
+    rows = np.asarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+
+    # Visibility of key j for row i: lo_i <= j <= hi_i.
+    lo = np.empty(R, dtype=np.int64)
+    hi = np.empty(R, dtype=np.int64)
+    for n, i in enumerate(rows):
+        lo[n], hi[n] = visible_range(int(i), kv_len=Skv, start_pos=start_pos,
+                                     causal=causal, window_lo=window_lo)
+    j = np.arange(Skv)
+    vis = (j[None, :] >= lo[:, None]) & (j[None, :] <= hi[:, None])  # [R, Skv]
+    any_vis = vis.any(axis=1)
+
+    out = np.zeros((B, Hq, R, D), dtype=np.float64)
+    lse = np.full((B, Hq, R), -np.inf, dtype=np.float64)
+    probs = np.zeros((B, Hq, R, Skv), dtype=np.float64) if return_probs else None
+
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // group
+            s = scale * (q[b, hq, rows, :] @ k[b, hk].T)  # [R, Skv] scores
+            s = np.where(vis, s, -np.inf)                  # masked keys
+            m = np.max(s, axis=1)                           # row max (-inf if none)
+            m_safe = np.where(any_vis, m, 0.0)
+            p = np.where(vis, np.exp(s - m_safe[:, None]), 0.0)
+            l = p.sum(axis=1)
+            l_safe = np.where(any_vis, l, 1.0)
+            p = p / l_safe[:, None]                         # softmax rows
+            out[b, hq] = p @ v[b, hk]
+            lse[b, hq] = np.where(any_vis, m_safe + np.log(l_safe), -np.inf)
+            if return_probs:
+                probs[b, hq] = p
+    if return_probs:
+        return out, lse, probs
+    return out, lse
+
+
+def attention_flops(B, Hq, Sq, Skv, D, *, causal=False):
+    """Work count of the headline metric: 4*B*Hq*Sq*Skv*D, halved for causal.
+
+    The 4 = 2 (multiply-add) x 2 (Q K^T and P V).  The same count reproduces the
+    "≈ 520 TOPS" the page "Ядра attention на домашней RTX 5080" quotes for a
+    42 ms kernel at 1 x 40 x 32760 x 128 (section "1 · Только ядро").
+    """
+    f = 4.0 * B * Hq * Sq * Skv * D
+    return f / 2.0 if causal else f
+
+
+def visible_pairs(Sq, Skv, *, start_pos=0, causal=False, window_lo=0):
+    """Exact number of visible (query, key) pairs of one head."""
+    n = 0
+    for i in range(Sq):
+        lo, hi = visible_range(i, kv_len=Skv, start_pos=start_pos, causal=causal,
+                               window_lo=window_lo)
+        n += max(0, hi - lo + 1)
+    return n
