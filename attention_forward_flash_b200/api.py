@@ -1,0 +1,118 @@
+"""Torch-facing convenience wrapper over the C ABI.
+
+Torch provides device memory and streams only; every computation runs in the
+library's kernels.  Shapes: q [B, Hq, Sq, D], k/v [B, Hkv, Skv, D], contiguous
+CUDA tensors of the context's dtype.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import _abi
+from ._abi import (ATTN_BF16, ATTN_EXACT, ATTN_FP16, ATTN_INT8QK_FP8PV, AttnParams, AttnQBufs)
+
+_PRECISIONS = {"exact": ATTN_EXACT, "quant": ATTN_INT8QK_FP8PV}
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class QuantBuffers:
+    """Device buffers of the quantised mode (see ``attn_qbufs`` in include/attn.h)."""
+
+    def __init__(self, params: AttnParams, device):
+        B, Hq, Hk = params.batch, params.n_q_heads, params.n_kv_heads
+        Sq, Sk, D = params.q_len, params.kv_len, params.head_dim
+        nbq, nbk = (Sq + 127) // 128, (Sk + 127) // 128
+        self.q = torch.empty((B, Hq, Sq, D), dtype=torch.int8, device=device)
+        self.k = torch.empty((B, Hk, Sk, D), dtype=torch.int8, device=device)
+        self.q_scale = torch.empty((B, Hq, nbq), dtype=torch.float32, device=device)
+        self.k_scale = torch.empty((B, Hk, nbk), dtype=torch.float32, device=device)
+        self.v_t = torch.empty((B, Hk, D, nbk * 128), dtype=torch.uint8, device=device)
+        self.v_scale = torch.empty((B, Hk, D), dtype=torch.float32, device=device)
+
+    def struct(self):
+        return AttnQBufs(self.q.data_ptr(), self.k.data_ptr(), self.q_scale.data_ptr(),
+                         self.k_scale.data_ptr(), self.v_t.data_ptr(), self.v_scale.data_ptr())
+
+
+class Attention:
+    """One attention problem shape bound to a library context."""
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, q_len, kv_len, head_dim, *,
+                 dtype=torch.bfloat16, causal=False, start_pos=0, window_lo=0, scale=0.0,
+                 precision="exact", num_splits=0):
+        if dtype not in (torch.bfloat16, torch.float16):
+            raise ValueError("dtype must be torch.bfloat16 or torch.float16")
+        self.dtype = dtype
+        self.precision = precision
+        self.params = AttnParams(batch, n_q_heads, n_kv_heads, q_len, kv_len, head_dim, start_pos,
+                                 int(bool(causal)), window_lo, float(scale),
+                                 ATTN_FP16 if dtype == torch.float16 else ATTN_BF16,
+                                 _PRECISIONS[precision], num_splits)
+        self.ctx = _abi.attn_create(self.params)
+
+    @property
+    def num_splits(self):
+        return _abi.attn_num_splits(self.ctx)
+
+    def _check_inputs(self, q, k, v):
+        p = self.params
+        want_q = (p.batch, p.n_q_heads, p.q_len, p.head_dim)
+        want_kv = (p.batch, p.n_kv_heads, p.kv_len, p.head_dim)
+        for name, t, shape in (("q", q, want_q), ("k", k, want_kv), ("v", v, want_kv)):
+            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or not t.is_cuda:
+                raise ValueError(f"{name}: expected contiguous CUDA {self.dtype} of shape {shape}, "
+                                 f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+    def quantize(self, q, k, v, qbufs=None, stream=None):
+        if self.precision != "quant":
+            raise ValueError("quantize() needs precision='quant'")
+        self._check_inputs(q, k, v)
+        qbufs = qbufs if qbufs is not None else QuantBuffers(self.params, q.device)
+        _abi.attn_quantize_qk(self.ctx, q.data_ptr(), k.data_ptr(), v.data_ptr(), qbufs.struct(),
+                              _stream_handle(stream))
+        return qbufs
+
+    def forward(self, q=None, k=None, v=None, *, qbufs=None, out=None, lse=None, return_lse=False,
+                stream=None):
+        p = self.params
+        device = (q if q is not None else qbufs.q).device
+        if out is None:
+            out = torch.empty((p.batch, p.n_q_heads, p.q_len, p.head_dim), dtype=self.dtype,
+                              device=device)
+        if lse is None and return_lse:
+            lse = torch.empty((p.batch, p.n_q_heads, p.q_len), dtype=torch.float32, device=device)
+        st = _stream_handle(stream)
+        lse_ptr = lse.data_ptr() if lse is not None else None
+        if self.precision == "quant":
+            if qbufs is None:
+                qbufs = self.quantize(q, k, v, stream=stream)
+            _abi.attn_forward(self.ctx, None, None, None, qbufs.struct(), out.data_ptr(), lse_ptr, st)
+        else:
+            self._check_inputs(q, k, v)
+            _abi.attn_forward(self.ctx, q.data_ptr(), k.data_ptr(), v.data_ptr(), None,
+                              out.data_ptr(), lse_ptr, st)
+        return (out, lse) if return_lse else out
+
+    __call__ = forward
+
+    def check_error(self, stream=None):
+        """Synchronise and raise AttnError if a kernel recorded a failed wait."""
+        status = _abi.attn_get_error(self.ctx, _stream_handle(stream))
+        if status != _abi.ATTN_OK:
+            raise _abi.AttnError(status, "device")
+
+    def close(self):
+        if getattr(self, "ctx", None) is not None and self.ctx.value:
+            _abi.attn_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

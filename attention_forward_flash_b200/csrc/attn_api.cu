@@ -1,0 +1,414 @@
+// Host side of the C ABI declared in include/attn.h: argument validation, the
+// choice of kernel variant and key/value split, workspace ownership, TMA
+// tensor-map encoding and the launches.  No computation happens here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "flash_fwd.cuh"
+#include "merge.cuh"
+#include "quant.cuh"
+
+using namespace attn;
+
+struct attn_ctx {
+  attn_params p;
+  int device;
+  int num_sms;
+  int G;           // query heads per kv head
+  int R;           // stacked rows per unit
+  int units;       // batch * n_kv_heads
+  int split_path;  // 1: single-query-tile kernel + merge; 0: two-query-tile kernel
+  int splits;
+  int tiles_per_split;
+  int row_tiles;
+  float scale;
+  void* ws;         // workspace (one allocation)
+  size_t ws_bytes;
+  float* o_part;
+  float* lse_part;
+  unsigned* v_amax;
+  unsigned* err;
+  unsigned debug;
+};
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D tiled map: dims (d0 fastest, d1, d2), byte strides of d1 and d2, box (b0, b1, 1).
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+              uint64_t d2, uint64_t st1, uint64_t st2, uint32_t b0, uint32_t b1,
+              CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {st1, st2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT>
+attn_status launch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+                       cudaStream_t st) {
+  using Cfg = FwdCfg<D, NQT, QUANT, SPLIT>;
+  auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT>;
+  static bool attr_ok = set_smem(kern, Cfg::kSmemBytes);
+  if (!attr_ok) return ATTN_ERR_CUDA;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool QUANT, bool F16>
+attn_status dispatch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
+                         const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+                         cudaStream_t st) {
+  if (c->split_path) return launch_fwd<D, 1, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
+  return launch_fwd<D, 2, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
+}
+
+template <int D, bool F16>
+attn_status launch_merge(const attn_ctx* c, void* o, float* lse, cudaStream_t st) {
+  const int rows = c->units * c->R;
+  splitkv_merge_kernel<D, F16><<<ceil_div(rows, 8), 256, 0, st>>>(
+      c->o_part, c->lse_part, static_cast<uint16_t*>(o), lse, rows, c->splits);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status validate(const attn_params* p) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1) return ATTN_ERR_INVALID_ARG;
+  if (p->n_q_heads % p->n_kv_heads != 0) return ATTN_ERR_INVALID_ARG;
+  if (p->q_len < 0 || p->kv_len < 0 || p->start_pos < 0 || p->window_lo < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_INVALID_ARG;
+  if (p->precision != ATTN_EXACT && p->precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
+  if (p->num_splits < 0 || p->num_splits > kMergeMaxSplits) return ATTN_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(p->n_q_heads / p->n_kv_heads) * p->q_len;
+  if (rows > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->start_pos) + p->q_len > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_OOM: return "out of device memory";
+    case ATTN_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+attn_status attn_qbufs_sizes(const attn_params* p, size_t sizes[6]) {
+  if (!sizes) return ATTN_ERR_INVALID_ARG;
+  attn_status v = validate(p);
+  if (v != ATTN_OK) return v;
+  const size_t B = p->batch, Hq = p->n_q_heads, Hk = p->n_kv_heads, D = p->head_dim;
+  const size_t Sq = p->q_len, Sk = p->kv_len;
+  const size_t nbq = (Sq + 127) / 128, nbk = (Sk + 127) / 128;
+  sizes[0] = B * Hq * Sq * D;
+  sizes[1] = B * Hk * Sk * D;
+  sizes[2] = B * Hq * nbq * 4;
+  sizes[3] = B * Hk * nbk * 4;
+  sizes[4] = B * Hk * D * nbk * 128;
+  sizes[5] = B * Hk * D * 4;
+  return ATTN_OK;
+}
+
+attn_status attn_create(const attn_params* p, attn_ctx** out) {
+  if (!out) return ATTN_ERR_INVALID_ARG;
+  *out = nullptr;
+  attn_status v = validate(p);
+  if (v != ATTN_OK) return v;
+
+  int dev = 0, sms = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (major != 10) return ATTN_ERR_UNSUPPORTED;  // built for sm_100a only
+
+  attn_ctx* c = new attn_ctx();
+  c->p = *p;
+  c->device = dev;
+  c->num_sms = sms;
+  c->G = p->n_q_heads / p->n_kv_heads;
+  c->R = c->G * p->q_len;
+  c->units = p->batch * p->n_kv_heads;
+  c->scale = p->scale > 0.0f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
+  const int kv_tiles = ceil_div(p->kv_len, 128);
+
+  // Few rows per kv head (decode-shaped) or too few CTAs to fill the GPU:
+  // one 128-row query tile per CTA, keys split across CTAs, then a merge.
+  const int big_ctas = c->units * ceil_div(c->R, 256);
+  bool split = false;
+  int splits = 1;
+  if (p->num_splits > 1) {
+    split = true;
+    splits = p->num_splits;
+  } else if (p->num_splits == 0) {
+    if (c->R <= 128 || (big_ctas * 2 < sms && kv_tiles >= 4)) {
+      split = true;
+      const int base = c->units * ceil_div(c->R, 128);
+      splits = std::max(1, std::min(kv_tiles, ceil_div(sms, base)));
+    }
+  }
+  splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
+  splits = std::min(splits, kMergeMaxSplits);
+  c->split_path = split ? 1 : 0;
+  c->tiles_per_split = std::max(1, ceil_div(kv_tiles, splits));
+  c->splits = split ? std::max(1, ceil_div(kv_tiles, c->tiles_per_split)) : 1;
+  c->row_tiles = ceil_div(c->R, split ? 128 : 256);
+
+  // workspace: error word | V channel maxima | split partials
+  size_t off = 256;
+  size_t vamax_off = 0, opart_off = 0, lpart_off = 0;
+  if (p->precision == ATTN_INT8QK_FP8PV) {
+    vamax_off = off;
+    off += (static_cast<size_t>(c->units) * p->head_dim * 4 + 255) / 256 * 256;
+  }
+  if (split) {
+    const size_t rows = static_cast<size_t>(c->units) * c->R;
+    opart_off = off;
+    off += (static_cast<size_t>(c->splits) * rows * p->head_dim * 4 + 255) / 256 * 256;
+    lpart_off = off;
+    off += (static_cast<size_t>(c->splits) * rows * 4 + 255) / 256 * 256;
+  }
+  if (cudaMalloc(&c->ws, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete c;
+    return ATTN_ERR_OOM;
+  }
+  c->ws_bytes = off;
+  uint8_t* base = static_cast<uint8_t*>(c->ws);
+  c->err = reinterpret_cast<unsigned*>(base);
+  c->v_amax = vamax_off ? reinterpret_cast<unsigned*>(base + vamax_off) : nullptr;
+  c->o_part = split ? reinterpret_cast<float*>(base + opart_off) : nullptr;
+  c->lse_part = split ? reinterpret_cast<float*>(base + lpart_off) : nullptr;
+  if (cudaMemset(c->err, 0, 256) != cudaSuccess) {
+    cudaFree(c->ws);
+    delete c;
+    return ATTN_ERR_CUDA;
+  }
+  *out = c;
+  return ATTN_OK;
+}
+
+void attn_destroy(attn_ctx* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  cudaFree(c->ws);
+  delete c;
+}
+
+int attn_num_splits(const attn_ctx* c) { return c ? (c->split_path ? c->splits : 1) : 0; }
+
+attn_status attn_debug_set(attn_ctx* c, unsigned flags) {
+  if (!c) return ATTN_ERR_INVALID_ARG;
+  c->debug = flags;
+  return ATTN_OK;
+}
+
+attn_status attn_get_error(attn_ctx* c, void* stream) {
+  if (!c) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned h = 0;
+  if (cudaMemcpy(&h, c->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (h != 0) {
+    if (cudaMemset(c->err, 0, 4) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_ERR_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const void* v,
+                             const attn_qbufs* qb, void* stream) {
+  if (!c || !qb || !q || !k || !v) return ATTN_ERR_INVALID_ARG;
+  if (c->p.precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
+  if (!qb->q || !qb->k || !qb->q_scale || !qb->k_scale || !qb->v_t || !qb->v_scale)
+    return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, qb->q, qb->k, qb->q_scale, qb->k_scale, qb->v_t, qb->v_scale};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+  const attn_params& p = c->p;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D = p.head_dim;
+  const bool f16 = p.dtype == ATTN_FP16;
+  const int nbq = ceil_div(p.q_len, 128), nbk = ceil_div(p.kv_len, 128);
+  const int S_pad = nbk * 128;
+  const unsigned BHq = p.batch * p.n_q_heads;
+  const unsigned BHk = c->units;
+  auto X = [](const void* ptr) { return static_cast<const uint16_t*>(ptr); };
+
+#define ATTN_QUANT_LAUNCH(DD, FF)                                                              \
+  do {                                                                                         \
+    if (nbq > 0)                                                                               \
+      quant_qk_kernel<DD, FF><<<dim3(nbq, BHq), 256, 0, st>>>(X(q), qb->q, qb->q_scale,        \
+                                                               p.q_len, nbq);                  \
+    if (nbk > 0) {                                                                             \
+      quant_qk_kernel<DD, FF><<<dim3(nbk, BHk), 256, 0, st>>>(X(k), qb->k, qb->k_scale,        \
+                                                               p.kv_len, nbk);                 \
+      v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(           \
+          X(v), c->v_amax, p.kv_len);                                                          \
+      v_quant_kernel<DD, FF><<<dim3(nbk, BHk), 256, 0, st>>>(X(v), c->v_amax, qb->v_t,         \
+                                                              qb->v_scale, p.kv_len, S_pad);   \
+    }                                                                                          \
+  } while (0)
+
+  if (nbk > 0 &&
+      cudaMemsetAsync(c->v_amax, 0, static_cast<size_t>(c->units) * D * 4, st) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (D == 128) {
+    if (f16) ATTN_QUANT_LAUNCH(128, true);
+    else ATTN_QUANT_LAUNCH(128, false);
+  } else {
+    if (f16) ATTN_QUANT_LAUNCH(64, true);
+    else ATTN_QUANT_LAUNCH(64, false);
+  }
+#undef ATTN_QUANT_LAUNCH
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* v,
+                         const attn_qbufs* qb, void* o, float* lse, void* stream) {
+  if (!c || !o) return ATTN_ERR_INVALID_ARG;
+  const attn_params& p = c->p;
+  const bool quant = p.precision == ATTN_INT8QK_FP8PV;
+  if (quant) {
+    if (!qb || !qb->q || !qb->k || !qb->q_scale || !qb->k_scale || !qb->v_t || !qb->v_scale)
+      return ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {qb->q, qb->k, qb->q_scale, qb->k_scale, qb->v_t, qb->v_scale};
+    for (const void* ptr : ptrs)
+      if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+  } else {
+    if (qb || !q || !k || !v) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_INVALID_ARG;
+  }
+  if (!aligned16(o) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D = p.head_dim;
+  const bool f16 = p.dtype == ATTN_FP16;
+  const size_t rows = static_cast<size_t>(c->units) * c->R;
+  if (rows == 0) return ATTN_OK;
+  if (p.kv_len == 0) {  // every row sees no key
+    if (cudaMemsetAsync(o, 0, rows * D * 2, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (lse) fill_lse_kernel<<<ceil_div(rows, 256), 256, 0, st>>>(lse, rows);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+
+  // Tensor maps.  Q, O: [units][R][D]; K, V: [units][Skv][D]; V^T: [units][D][S_pad].
+  const CUtensorMapDataType t16 =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t R = c->R, Sk = p.kv_len, U = c->units;
+  CUtensorMap tq, tk, tv, to;
+  bool ok = true;
+  if (quant) {
+    const CUtensorMapSwizzle sw8 =
+        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const uint64_t S_pad = static_cast<uint64_t>(ceil_div(p.kv_len, 128)) * 128;
+    ok &= make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, D, R, U, D, R * D, D, 128, sw8);
+    ok &= make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, D, Sk, U, D, Sk * D, D, 128, sw8);
+    ok &= make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->v_t, S_pad, D, U, S_pad, S_pad * D, 128,
+                   D, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok &= make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return ATTN_ERR_CUDA;
+
+  FwdArgs a{};
+  a.R = c->R;
+  a.Sq = p.q_len;
+  a.Skv = p.kv_len;
+  a.G = c->G;
+  a.units = c->units;
+  a.row_tiles = c->row_tiles;
+  a.splits = c->splits;
+  a.tiles_per_split = c->tiles_per_split;
+  a.start_pos = p.start_pos;
+  a.causal = p.causal;
+  a.window_lo = p.window_lo;
+  a.scale_log2 = c->scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.o_part = c->o_part;
+  a.lse_part = c->lse_part;
+  if (quant) {
+    a.q_scale = qb->q_scale;
+    a.k_scale = qb->k_scale;
+    a.v_scale = qb->v_scale;
+  }
+  a.nblk_q = ceil_div(p.q_len, 128);
+  a.nblk_k = ceil_div(p.kv_len, 128);
+  a.err = c->err;
+  a.debug = c->debug;
+  const int grid = c->units * c->row_tiles * (c->split_path ? c->splits : 1);
+
+  attn_status s;
+  if (D == 128) {
+    if (quant) s = f16 ? dispatch_fwd<128, true, true>(c, tq, tk, tv, to, a, grid, st)
+                       : dispatch_fwd<128, true, false>(c, tq, tk, tv, to, a, grid, st);
+    else s = f16 ? dispatch_fwd<128, false, true>(c, tq, tk, tv, to, a, grid, st)
+                 : dispatch_fwd<128, false, false>(c, tq, tk, tv, to, a, grid, st);
+  } else {
+    if (quant) s = f16 ? dispatch_fwd<64, true, true>(c, tq, tk, tv, to, a, grid, st)
+                       : dispatch_fwd<64, true, false>(c, tq, tk, tv, to, a, grid, st);
+    else s = f16 ? dispatch_fwd<64, false, true>(c, tq, tk, tv, to, a, grid, st)
+                 : dispatch_fwd<64, false, false>(c, tq, tk, tv, to, a, grid, st);
+  }
+  if (s != ATTN_OK) return s;
+  if (c->split_path) {
+    if (D == 128) s = f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
+    else s = f16 ? launch_merge<64, true>(c, o, lse, st) : launch_merge<64, false>(c, o, lse, st);
+  }
+  return s;
+}
+
+}  // extern "C"

@@ -1,0 +1,592 @@
+// Fused attention forward for sm_100a: O = softmax(scale * Q K^T + mask) V.
+//
+// The method is the one all the source pages turn on (flash attention over
+// key/value tiles with an online softmax; "perf(metal): widen four-row flash
+// KV tiles - #89", "Summary"), laid out for Blackwell:
+//
+//  * one CTA owns NQT query tiles of 128 rows of one (batch, kv-head) "unit";
+//    the rows of the query heads that share a kv head (GQA) are stacked, so a
+//    unit has R = (Hq/Hkv) * Sq rows and row r is query head g = r / Sq,
+//    position start_pos + r % Sq;
+//  * warp 0 streams Q once and K/V tiles of 128 keys through a ring of
+//    shared-memory slots with TMA (128-byte swizzle, no multicast);
+//  * one thread of warp 1 issues the tcgen05 MMAs: S = Q K^T into tensor
+//    memory (TMEM), then O += P V with P read from TMEM, O accumulated in TMEM;
+//  * one warpgroup per query tile runs the softmax: each thread owns one row
+//    (tcgen05.ld 32x32b), applies the causal / window / length masks on
+//    boundary tiles only, keeps the running max and sum in base 2, writes P
+//    back over S in TMEM, and rescales O in TMEM only when the row max grew by
+//    more than a threshold (the final division uses the same stale max, so the
+//    result is unchanged);
+//  * the epilogue divides O by the row sum and stores it with TMA (or, in the
+//    split-KV variant, writes float32 partials and base-2 log-sum-exp for the
+//    merge kernel; qsa2 audit, "implementation and review").
+//
+// Quantised variant (QUANT): Q/K are INT8 codes with one float32 scale per
+// 128-token block (kind::i8 MMA, s32 accumulators), P is E4M3 scaled by 2^8,
+// V^T is E4M3 with per-channel scales (kind::f8f6f4 MMA); this is the
+// "INT8 QK · FP8 PV" form of the table in section "1 · Только ядро" of the page
+// "Ядра attention на домашней RTX 5080".
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace attn {
+
+struct FwdArgs {
+  int R;           // stacked query rows per unit: (Hq/Hkv) * Sq
+  int Sq;          // query rows per head
+  int Skv;         // keys
+  int G;           // query heads per kv head
+  int units;       // batch * Hkv
+  int row_tiles;   // ceil(R / (NQT*128))
+  int splits;      // key splits per row tile (split variant)
+  int tiles_per_split;
+  int start_pos;
+  int causal;
+  int window_lo;
+  float scale_log2;  // scale * log2(e)
+  float* lse;        // [units * R] natural-log lse or nullptr (non-split variant)
+  float* o_part;     // [splits, units, R, D] float32 (split variant)
+  float* lse_part;   // [splits, units, R] base-2 lse (split variant)
+  const float* q_scale;  // quantised variant
+  const float* k_scale;
+  const float* v_scale;
+  int nblk_q;
+  int nblk_k;
+  unsigned* err;     // device error word
+  unsigned debug;    // bit 0: skip the second key tile (timeout test)
+};
+
+constexpr int kErrTimeout = 1;
+
+template <int D, int NQT, bool QUANT, bool SPLIT>
+struct FwdCfg {
+  static constexpr int kThreads = 128 * (1 + NQT);
+  static constexpr int kElem = QUANT ? 1 : 2;                 // bytes per Q/K element
+  static constexpr int kQTile = 128 * D * kElem;              // one 128-row Q tile
+  static constexpr int kKTile = 128 * D * kElem;
+  static constexpr int kVTile = 128 * D * (QUANT ? 1 : 2);
+  static constexpr int kSlot = kKTile > kVTile ? kKTile : kVTile;
+  static constexpr int kOStage = 128 * D * 2;                 // 16-bit output tile
+  static constexpr bool kStageInQ = (kQTile >= kOStage);
+  static constexpr int kStageBytes = (SPLIT || kStageInQ) ? 0 : NQT * kOStage;
+  static constexpr int kFixed = NQT * kQTile + kStageBytes;
+  static constexpr int kBudget = 200 * 1024;
+  static constexpr int kNSraw = (kBudget - kFixed) / kSlot;
+  static constexpr int kNS = kNSraw > 8 ? 8 : kNSraw;
+  static_assert(kNS >= 2, "ring too small");
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = NQT * kQTile;
+  static constexpr int kRingOff = kFixed;
+  static constexpr int kBarOff = kRingOff + kNS * kSlot;
+  // barriers: q_full, full[NS], empty[NS], s_ready[NQT], p_ready[NQT], o_final
+  static constexpr int kNumBars = 1 + 2 * kNS + 2 * NQT + 1;
+  static constexpr int kMiscOff = kBarOff + 8 * kNumBars;      // tmem base, abort flag
+  static constexpr int kSvOff = kMiscOff + 16;                  // v scales (quant)
+  static constexpr int kSmemBytes = kSvOff + (QUANT ? D * 4 : 0) + 1024;  // + alignment slack
+  static constexpr int kTmemNeed = NQT * (128 + D);
+  static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
+  // transaction bytes
+  static constexpr uint32_t kQBytes = NQT * kQTile;
+  static constexpr uint32_t kKBytes = kKTile;
+  static constexpr uint32_t kVBytes = kVTile;
+  // softmax rescale threshold (base-2 units).  Quantised: P*2^8 must stay
+  // within the E4M3 range (448), so the max is tracked exactly.
+  static constexpr float kRescaleThresh = QUANT ? 0.0f : 8.0f;
+};
+
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_16x2(float lo, float hi) {
+  if constexpr (F16) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// Exact conversion of |s| < 2^22 integers to float with integer + float adds.
+__device__ __forceinline__ float s32_to_f32(uint32_t s) {
+  return __uint_as_float(s + 0x4B400000u) - 12582912.0f;
+}
+
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT>
+__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
+    flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
+  using C = FwdCfg<D, NQT, QUANT, SPLIT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---------------------------------------------------------- work decode
+  int u, t, split = 0;
+  {
+    int lin = blockIdx.x;
+    if constexpr (SPLIT) {
+      split = lin % a.splits;
+      lin /= a.splits;
+    }
+    u = lin / a.row_tiles;
+    t = lin % a.row_tiles;
+    if (!SPLIT && a.causal) t = a.row_tiles - 1 - t;  // heaviest tiles of a unit first
+  }
+  const int BM = NQT * 128;
+  const int r0 = t * BM;
+  const int r_last = min(r0 + BM, a.R) - 1;
+  int pos_min, pos_max;
+  if (r0 / a.Sq != r_last / a.Sq) {
+    pos_min = a.start_pos;
+    pos_max = a.start_pos + a.Sq - 1;
+  } else {
+    pos_min = a.start_pos + r0 % a.Sq;
+    pos_max = a.start_pos + r_last % a.Sq;
+  }
+  const int kv_lo = a.window_lo;
+  const int kv_hi = a.causal ? min(a.Skv - 1, pos_max) : a.Skv - 1;
+  int jt0 = 0, jt1 = 0;  // absolute key-tile range [jt0, jt1)
+  if (kv_hi >= kv_lo) {
+    jt0 = kv_lo / 128;
+    jt1 = kv_hi / 128 + 1;
+    if constexpr (SPLIT) {
+      const int b0 = jt0 + split * a.tiles_per_split;
+      jt1 = min(jt1, b0 + a.tiles_per_split);
+      jt0 = b0;
+      if (jt0 > jt1) jt0 = jt1;
+    }
+  }
+  const int n = jt1 - jt0;
+
+  // ------------------------------------------------------------ set-up
+  auto bar = [&](int i) { return sbase + C::kBarOff + 8 * i; };
+  const uint32_t q_full = bar(0);
+  auto full_bar = [&](int s) { return bar(1 + s); };
+  auto empty_bar = [&](int s) { return bar(1 + C::kNS + s); };
+  auto s_ready = [&](int q) { return bar(1 + 2 * C::kNS + q); };
+  auto p_ready = [&](int q) { return bar(1 + 2 * C::kNS + NQT + q); };
+  const uint32_t o_final = bar(1 + 2 * C::kNS + 2 * NQT);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  float* sv_smem = reinterpret_cast<float*>(smem + C::kSvOff);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::kNS; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int q = 0; q < NQT; ++q) {
+      mbar_init(s_ready(q), 1);
+      mbar_init(p_ready(q), 128);
+    }
+    mbar_init(o_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if constexpr (QUANT) {
+    if (warp == 2)
+      for (int c = lane; c < D; c += 32) sv_smem[c] = a.v_scale[(size_t)u * D + c];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  auto raise = [&]() {
+    *abort_flag = 1;
+    atomicOr(a.err, (unsigned)kErrTimeout);
+  };
+
+  if (warp == 0) {
+    // ======================================================== TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      constexpr int kBoxCols = QUANT ? D : 64;         // elements per box row
+      constexpr int kQBoxes = QUANT ? 1 : D / 64;
+      constexpr int kQBox = 128 * kBoxCols * C::kElem;
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      for (int q = 0; q < NQT; ++q)
+        for (int bx = 0; bx < kQBoxes; ++bx)
+          tma_load_3d(&tm_q, sbase + C::kQOff + q * C::kQTile + bx * kQBox, q_full,
+                      bx * kBoxCols, r0 + q * 128, u);
+      int last_issue[C::kNS];
+      for (int s = 0; s < C::kNS; ++s) last_issue[s] = -1;
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int kv0 = (jt0 + j) * 128;
+        for (int part = 0; part < 2 && ok; ++part, ++it) {  // 0: K tile, 1: V tile
+          const int s = it % C::kNS;
+          const uint32_t ph = (it / C::kNS) & 1;
+          if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag)) { raise(); ok = false; break; }
+          if ((a.debug & 1u) && j == 1 && part == 0) continue;  // timeout test: never load
+          const uint32_t dst = sbase + C::kRingOff + s * C::kSlot;
+          if (part == 0) {
+            mbar_arrive_expect_tx(full_bar(s), C::kKBytes);
+            if constexpr (QUANT) {
+              tma_load_3d(&tm_k, dst, full_bar(s), 0, kv0, u);
+            } else {
+              for (int bx = 0; bx < D / 64; ++bx)
+                tma_load_3d(&tm_k, dst + bx * 128 * 64 * 2, full_bar(s), bx * 64, kv0, u);
+            }
+          } else {
+            mbar_arrive_expect_tx(full_bar(s), C::kVBytes);
+            if constexpr (QUANT) {
+              tma_load_3d(&tm_v, dst, full_bar(s), kv0, 0, u);   // V^T: [D rows, 128 keys]
+            } else {
+              for (int bx = 0; bx < D / 64; ++bx)
+                tma_load_3d(&tm_v, dst + bx * 128 * 64 * 2, full_bar(s), bx * 64, kv0, u);
+            }
+          }
+          last_issue[s] = it;
+        }
+      }
+      // Never leave with copies in flight into this CTA's shared memory.
+      {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(q_full, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+        }
+      }
+      for (int s = 0; s < C::kNS; ++s)
+        if (last_issue[s] >= 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(full_bar(s), (last_issue[s] / C::kNS) & 1) &&
+                 globaltimer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+    }
+  } else if (warp == 1) {
+    // ========================================================= MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t fmt = F16 ? 0u : 1u;
+      constexpr uint32_t idesc_qk =
+          QUANT ? instr_desc(2, 1, 1, 0, 0, 128, 128) : instr_desc(1, fmt, fmt, 0, 0, 128, 128);
+      constexpr uint32_t idesc_pv =
+          QUANT ? instr_desc(1, 0, 0, 0, 0, 128, D) : instr_desc(1, fmt, fmt, 0, 1, 128, D);
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      if (!ok) raise();
+      int it = 0;
+
+      auto issue_qk = [&](int q, uint32_t kslot) {
+        const uint32_t qs = sbase + C::kQOff + q * C::kQTile;
+        const uint32_t d = tmem + q * 128;
+        if constexpr (QUANT) {
+          // int8, K = D bytes per row: one swizzle atom column (128 B, or 64 B at D = 64)
+          constexpr uint32_t layout = (D == 128) ? 2u : 4u;
+          constexpr uint32_t sbo = (D == 128) ? 1024u : 512u;
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_i8_ss(d, smem_desc(qs + kk * 32, 16, sbo, layout),
+                      smem_desc(kslot + kk * 32, 16, sbo, layout), idesc_qk, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_f16_ss(d, smem_desc(qs + off, 16, 1024, 2), smem_desc(kslot + off, 16, 1024, 2),
+                       idesc_qk, kk > 0);
+          }
+        }
+      };
+      auto issue_pv = [&](int q, uint32_t vslot, uint32_t accum) {
+        const uint32_t d = tmem + NQT * 128 + q * D;
+        const uint32_t p = tmem + q * 128;
+        if constexpr (QUANT) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // 32 keys (8 columns of 4 e4m3) per step
+            mma_f8_ts(d, p + kk * 8, smem_desc(vslot + kk * 32, 16, 1024, 2), idesc_pv,
+                      (accum | kk) != 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)   // 16 keys (8 columns of 2 x 16-bit) per step
+            mma_f16_ts(d, p + kk * 8, smem_desc(vslot + kk * 2048, 128 * 128, 1024, 2), idesc_pv,
+                       (accum | kk) != 0);
+        }
+      };
+
+      // S_0 for every query tile
+      if (ok) {
+        const int s = it % C::kNS;
+        ok = mbar_wait(full_bar(s), (it / C::kNS) & 1, abort_flag);
+        if (!ok) raise();
+        else {
+          tc_fence_after();
+          const uint32_t kslot = sbase + C::kRingOff + s * C::kSlot;
+          for (int q = 0; q < NQT; ++q) {
+            issue_qk(q, kslot);
+            tc_commit(s_ready(q));
+          }
+          tc_commit(empty_bar(s));
+          ++it;
+        }
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int sv = it % C::kNS;
+        if (!mbar_wait(full_bar(sv), (it / C::kNS) & 1, abort_flag)) { raise(); ok = false; break; }
+        ++it;
+        const bool has_next = (j + 1 < n);
+        int sk = 0;
+        if (has_next) {
+          sk = it % C::kNS;
+          if (!mbar_wait(full_bar(sk), (it / C::kNS) & 1, abort_flag)) { raise(); ok = false; break; }
+          ++it;
+        }
+        tc_fence_after();
+        const uint32_t vslot = sbase + C::kRingOff + sv * C::kSlot;
+        const uint32_t kslot = sbase + C::kRingOff + sk * C::kSlot;
+        for (int q = 0; q < NQT && ok; ++q) {
+          if (!mbar_wait(p_ready(q), j & 1, abort_flag)) { raise(); ok = false; break; }
+          tc_fence_after();
+          issue_pv(q, vslot, j > 0);
+          if (q == NQT - 1) tc_commit(empty_bar(sv));
+          if (has_next) {
+            issue_qk(q, kslot);
+            tc_commit(s_ready(q));
+          }
+        }
+        if (ok && has_next) tc_commit(empty_bar(sk));
+      }
+      tc_commit(o_final);
+      // Leave only once every issued MMA has finished (TMEM is freed at exit).
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(o_final, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+  } else if (warp >= 4) {
+    // ============================================================ softmax
+    const int q = (warp - 4) >> 2;            // query tile of this warpgroup
+    const int wq = warp & 3;                  // TMEM lane quarter
+    const int row = wq * 32 + lane;
+    const int r = r0 + q * 128 + row;
+    const bool rvalid = r < a.R;
+    const int ri = rvalid ? r : a.R - 1;
+    const int i = ri % a.Sq;
+    const int pos = a.start_pos + i;
+    const int lo_r = a.window_lo;
+    const int hi_r = a.causal ? min(pos, a.Skv - 1) : a.Skv - 1;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + q * 128;
+    const uint32_t tO = tmem + lane_off + NQT * 128 + q * D;
+    float qsc = 1.0f;
+    if constexpr (QUANT) {
+      const int g = ri / a.Sq;
+      qsc = a.q_scale[((size_t)u * a.G + g) * a.nblk_q + i / 128];
+    }
+
+    float m_used = -INFINITY;  // running max of the base-2 scaled scores
+    float l = 0.0f;            // running row sum (relative to m_used)
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_ready(q), j & 1, abort_flag));
+      if (!ok) { if (lane == 0) raise(); break; }
+      tc_fence_after();
+      const int kv0 = (jt0 + j) * 128;
+      const bool need_mask =
+          (kv0 < a.window_lo) || (kv0 + 128 > a.Skv) || (a.causal && kv0 + 127 > pos_min);
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(tS + 0, s0);
+      tmem_ld32(tS + 32, s1);
+      tmem_ld32(tS + 64, s2);
+      tmem_ld32(tS + 96, s3);
+      tmem_ld_wait(s0);
+      tmem_ld_wait(s1);
+      tmem_ld_wait(s2);
+      tmem_ld_wait(s3);
+      float x[128];
+      float cj = a.scale_log2;  // raw-score -> base-2 scaled score factor
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        if constexpr (QUANT) {
+          x[c] = s32_to_f32(s0[c]);
+          x[32 + c] = s32_to_f32(s1[c]);
+          x[64 + c] = s32_to_f32(s2[c]);
+          x[96 + c] = s32_to_f32(s3[c]);
+        } else {
+          x[c] = __uint_as_float(s0[c]);
+          x[32 + c] = __uint_as_float(s1[c]);
+          x[64 + c] = __uint_as_float(s2[c]);
+          x[96 + c] = __uint_as_float(s3[c]);
+        }
+      }
+      // (kept positive so that masked -inf scores stay -inf for an all-zero block)
+      if constexpr (QUANT)
+        cj = fmaxf(qsc * a.k_scale[(size_t)u * a.nblk_k + jt0 + j] * a.scale_log2, 1e-30f);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int kj = kv0 + c;
+          if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_tile = mx * cj;  // cj > 0; -inf stays -inf
+      const float m_prev = m_used;
+      const float m_new = fmaxf(m_prev, m_tile);
+      const bool need = (m_prev != -INFINITY) && (m_new > m_prev + C::kRescaleThresh);
+      if (m_prev == -INFINITY || need) m_used = m_new;
+      if (__any_sync(0xffffffffu, need)) {
+        const float f = need ? ex2(m_prev - m_new) : 1.0f;
+        l *= f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+          tmem_st32(tO + c0, o);
+        }
+      }
+      // P = 2^(x * cj - m)  (quantised: times 2^8 before the E4M3 cast)
+      const float mb = (m_used == -INFINITY ? 0.0f : m_used) - (QUANT ? 8.0f : 0.0f);
+      float rs = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        x[c] = ex2(fmaf(x[c], cj, -mb));
+        rs += x[c];
+      }
+      l += rs;
+      if constexpr (QUANT) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const uint32_t lo = f32x2_to_e4m3x2(x[4 * c], x[4 * c + 1]);
+          const uint32_t hi = f32x2_to_e4m3x2(x[4 * c + 2], x[4 * c + 3]);
+          pk[c] = lo | (hi << 16);
+        }
+        tmem_st32(tS, pk);
+      } else {
+        uint32_t pk0[32], pk1[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          pk0[c] = pack_16x2<F16>(x[2 * c], x[2 * c + 1]);
+          pk1[c] = pack_16x2<F16>(x[64 + 2 * c], x[64 + 2 * c + 1]);
+        }
+        tmem_st32(tS, pk0);
+        tmem_st32(tS + 32, pk1);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_ready(q));
+    }
+
+    // ----------------------------------------------------------- epilogue
+    if (ok && n > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, abort_flag));
+      if (!ok && lane == 0) raise();
+      tc_fence_after();
+    } else if (n == 0) {
+      // No key tile: the Q copy (whose buffer stages the output) must have landed.
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
+      if (!ok && lane == 0) raise();
+    }
+    const bool have_o = ok && n > 0;
+    const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+    const float lse2 = (l > 0.0f) ? m_used + lg2(l) - (QUANT ? 8.0f : 0.0f) : -INFINITY;
+    if constexpr (SPLIT) {
+      const size_t prow = ((size_t)split * a.units + u) * a.R + r;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(tO + c0, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        if (rvalid) {
+          float4* dst = reinterpret_cast<float4*>(a.o_part + prow * D + c0);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            float4 v;
+            float sv0 = 1.f, sv1 = 1.f, sv2 = 1.f, sv3 = 1.f;
+            if constexpr (QUANT) {
+              sv0 = sv_smem[c0 + c];
+              sv1 = sv_smem[c0 + c + 1];
+              sv2 = sv_smem[c0 + c + 2];
+              sv3 = sv_smem[c0 + c + 3];
+            }
+            v.x = __uint_as_float(o[c]) * inv * sv0;
+            v.y = __uint_as_float(o[c + 1]) * inv * sv1;
+            v.z = __uint_as_float(o[c + 2]) * inv * sv2;
+            v.w = __uint_as_float(o[c + 3]) * inv * sv3;
+            dst[c / 4] = v;
+          }
+        }
+      }
+      if (rvalid) a.lse_part[prow] = lse2;
+    } else {
+      const uint32_t stage = C::kStageInQ ? sbase + C::kQOff + q * C::kQTile
+                                          : sbase + C::kStageOff + q * C::kOStage;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(tO + c0, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float v0 = __uint_as_float(o[2 * c]) * inv;
+          float v1 = __uint_as_float(o[2 * c + 1]) * inv;
+          if constexpr (QUANT) {
+            v0 *= sv_smem[c0 + 2 * c];
+            v1 *= sv_smem[c0 + 2 * c + 1];
+          }
+          pk[c] = pack_16x2<F16>(v0, v1);
+        }
+        // 128-byte swizzled box of 64 columns: 16-byte chunk k of row r sits at k ^ (r & 7)
+        const uint32_t box = stage + (c0 / 64) * (128 * 128);
+        const int cb = (c0 % 64) / 8;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t addr = box + row * 128 + (((cb + k) ^ (row & 7)) * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]),
+                       "r"(pk[4 * k + 1]), "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + q, 128);
+      if (row == 0 && !*abort_flag && r0 + q * 128 < a.R) {
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_store_3d(&tm_o, stage + bx * (128 * 128), bx * 64, r0 + q * 128, u);
+        bulk_commit();
+        bulk_wait_all();
+      }
+      if (rvalid && a.lse != nullptr) a.lse[(size_t)u * a.R + r] = lse2 * 0.69314718055994531f;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,96 @@
+// Merge of split-KV partial results (the qsa2 audit page, "implementation and
+// review": the merge caches each chunk's maximum and weight and computes the
+// denominator once).
+//
+// Each split s of a row left O_s (already divided by its own row sum) and
+// L_s = base-2 log-sum-exp of its scaled scores (-inf for an empty split).
+// With M = max_s L_s and w_s = 2^(L_s - M):
+//     O = sum_s w_s O_s / sum_s w_s,     lse = ln 2 * (M + log2 sum_s w_s).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace attn {
+
+constexpr int kMergeMaxSplits = 128;
+
+// grid: ceil(rows / 8), 256 threads; one warp per output row.
+template <int D, bool F16>
+__global__ void __launch_bounds__(256) splitkv_merge_kernel(const float* __restrict__ o_part,
+                                                            const float* __restrict__ lse_part,
+                                                            uint16_t* __restrict__ out,
+                                                            float* __restrict__ lse, int rows,
+                                                            int splits) {
+  constexpr int kPer = D / 32;  // channels per lane
+  __shared__ float wts[8][kMergeMaxSplits];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  // maxima and weights, computed once per split and cached
+  float M = -INFINITY;
+  for (int s = lane; s < splits; s += 32) M = fmaxf(M, lse_part[(size_t)s * rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float wsum = 0.0f;
+  for (int s = lane; s < splits; s += 32) {
+    const float L = lse_part[(size_t)s * rows + row];
+    const float w = (M == -INFINITY) ? 0.0f : ex2(L - M);
+    wts[warp][s] = w;
+    wsum += w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  __syncwarp();
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.0f;
+  for (int s = 0; s < splits; ++s) {
+    const float w = wts[warp][s];
+    if (w == 0.0f) continue;  // empty or negligible split: its partials are never read
+    const float* src = o_part + ((size_t)s * rows + row) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+      acc[2] += w * v.z;
+      acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+    }
+  }
+  const float inv = (wsum > 0.0f) ? 1.0f / wsum : 0.0f;
+  uint16_t h[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const float val = acc[e] * inv;
+    if constexpr (F16) {
+      const __half b = __float2half_rn(val);
+      h[e] = *reinterpret_cast<const uint16_t*>(&b);
+    } else {
+      const __nv_bfloat16 b = __float2bfloat16_rn(val);
+      h[e] = *reinterpret_cast<const uint16_t*>(&b);
+    }
+  }
+  uint16_t* dst = out + (size_t)row * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = h[0] | (uint32_t(h[1]) << 16);
+  }
+  if (lse != nullptr && lane == 0)
+    lse[row] = (wsum > 0.0f) ? (M + lg2(wsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+// O = 0 and lse = -inf for every row (a problem whose rows see no key at all).
+__global__ void fill_lse_kernel(float* lse, size_t rows) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i < rows) lse[i] = -INFINITY;
+}
+
+}  // namespace attn

@@ -1,0 +1,183 @@
+// Per-block quantisers of the opt-in reduced-precision mode ("SageAttention 2
+// INT8 QK · FP8 PV" row of the table in section "1 · Только ядро" of the page
+// "Ядра attention на домашней RTX 5080"; its ~14 ms of data preparation next to
+// a 42 ms kernel is why these kernels must run at HBM speed).
+//
+//  * Q and K: one float32 scale per (b, h, 128-token block):
+//      s = amax / 127,  code = clamp(rint_half_even(x / s), -127, 127).
+//  * V: one float32 scale per (b, hkv, channel) over all tokens:
+//      s = amax / 448,  code = E4M3(v / s), nearest-even, saturating,
+//    written transposed [b, hkv, channel, token] (zero padded to 128 tokens)
+//    so that it is the K-major operand of the P.V MMA.
+// Every arithmetic step is one correctly rounded float32 operation, so the
+// codes are reproducible bit for bit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace attn {
+
+template <bool F16>
+__device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if constexpr (F16) {
+      const __half2 h = *reinterpret_cast<const __half2*>(&u[k]);
+      f[2 * k] = __low2float(h);
+      f[2 * k + 1] = __high2float(h);
+    } else {
+      const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&u[k]);
+      f[2 * k] = __low2float(h);
+      f[2 * k + 1] = __high2float(h);
+    }
+  }
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// grid: (ceil(S/128), B*H), 256 threads.  One CTA quantises one 128-token block.
+template <int D, bool F16>
+__global__ void __launch_bounds__(256) quant_qk_kernel(const uint16_t* __restrict__ x,
+                                                       int8_t* __restrict__ codes,
+                                                       float* __restrict__ scales, int S,
+                                                       int nblk) {
+  constexpr int kChunks = 128 * D / 8;  // 16-byte chunks of a full block
+  constexpr int kPer = kChunks / 256;
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int tok0 = t * 128;
+  const int nelem = min(128, S - tok0) * D;
+  const size_t base = (bh * S + tok0) * D;
+
+  uint4 w[kPer];
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int c = threadIdx.x + k * 256;
+    if (c * 8 < nelem) {
+      w[k] = ld_nc_v4(x + base + (size_t)c * 8);
+      float f[8];
+      unpack8<F16>(w[k], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    } else {
+      w[k] = make_uint4(0, 0, 0, 0);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int k = 1; k < 8; ++k) amax = fmaxf(amax, red[k]);
+
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (threadIdx.x == 0) scales[bh * nblk + t] = s;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int c = threadIdx.x + k * 256;
+    if (c * 8 < nelem) {
+      float f[8];
+      unpack8<F16>(w[k], f);
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        int qv = 0;
+        if (s > 0.0f) qv = max(-127, min(127, __float2int_rn(__fdiv_rn(f[e], s))));
+        packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+      }
+      *reinterpret_cast<uint2*>(codes + base + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
+    }
+  }
+}
+
+// grid: (ceil(S/kVTok), B*Hkv), 256 threads.  Channel maxima of |V| as float
+// bit patterns (non-negative floats order like unsigned integers).
+constexpr int kVTok = 256;
+
+template <int D, bool F16>
+__global__ void __launch_bounds__(256) v_amax_kernel(const uint16_t* __restrict__ v,
+                                                     unsigned* __restrict__ amax_bits, int S) {
+  constexpr int kCC = D / 8;            // 16-byte chunks per token
+  constexpr int kRows = 256 / kCC;      // tokens covered per pass
+  __shared__ unsigned smax[D];
+  for (int c = threadIdx.x; c < D; c += 256) smax[c] = 0u;
+  __syncthreads();
+  const size_t u = blockIdx.y;
+  const int tok0 = blockIdx.x * kVTok;
+  const int cc = threadIdx.x % kCC;
+  float m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int tk = threadIdx.x / kCC; tk < kVTok; tk += kRows) {
+    const int tok = tok0 + tk;
+    if (tok < S) {
+      float f[8];
+      unpack8<F16>(ld_nc_v4(v + ((u * S + tok) * D + cc * 8)), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) atomicMax(&smax[cc * 8 + e], __float_as_uint(m[e]));
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 256) atomicMax(&amax_bits[u * D + c], smax[c]);
+}
+
+// grid: (S_pad/128, B*Hkv), 256 threads.  Quantise a 128-token tile of V and
+// write it transposed.
+template <int D, bool F16>
+__global__ void __launch_bounds__(256) v_quant_kernel(const uint16_t* __restrict__ v,
+                                                      const unsigned* __restrict__ amax_bits,
+                                                      uint8_t* __restrict__ vt,
+                                                      float* __restrict__ v_scale, int S,
+                                                      int S_pad) {
+  constexpr int kCC = D / 8;
+  constexpr int kPitch = 128 + 16;  // bytes per transposed row in shared memory
+  __shared__ float sc[D];
+  __shared__ __align__(16) uint8_t tile[D * kPitch];
+  const size_t u = blockIdx.y;
+  const int tok0 = blockIdx.x * 128;
+  for (int c = threadIdx.x; c < D; c += 256) {
+    const float s = __fdiv_rn(__uint_as_float(amax_bits[u * D + c]), 448.0f);
+    sc[c] = s;
+    if (blockIdx.x == 0) v_scale[u * D + c] = s;
+  }
+  __syncthreads();
+  for (int ch = threadIdx.x; ch < 128 * kCC; ch += 256) {
+    const int tk = ch / kCC;
+    const int cc = ch % kCC;
+    const int tok = tok0 + tk;
+    float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (tok < S) unpack8<F16>(ld_nc_v4(v + ((u * S + tok) * D + cc * 8)), f);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const int c0 = cc * 8 + e;
+      const float s0 = sc[c0], s1 = sc[c0 + 1];
+      const float a0 = (tok < S && s0 > 0.0f) ? __fdiv_rn(f[e], s0) : 0.0f;
+      const float a1 = (tok < S && s1 > 0.0f) ? __fdiv_rn(f[e + 1], s1) : 0.0f;
+      const uint16_t p = f32x2_to_e4m3x2(a0, a1);
+      tile[c0 * kPitch + tk] = static_cast<uint8_t>(p & 0xFF);
+      tile[(c0 + 1) * kPitch + tk] = static_cast<uint8_t>(p >> 8);
+    }
+  }
+  __syncthreads();
+  for (int ch = threadIdx.x; ch < D * 8; ch += 256) {
+    const int c = ch / 8;
+    const int part = ch % 8;
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + c * kPitch + part * 16);
+    *reinterpret_cast<uint4*>(vt + (u * D + c) * (size_t)S_pad + tok0 + part * 16) = w;
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,154 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) fused attention forward library.
+ *
+ * The operation is scaled-dot-product attention, O = softmax(scale*Q K^T + mask) V,
+ * computed flash-style (key/value tiles streamed through shared memory, an
+ * online softmax, no score matrix in global memory).  Sources for the problem
+ * statement:
+ *   - "perf(metal): widen four-row flash KV tiles - #89", section "Performance
+ *     evidence": query rows, n_head query heads over n_kv key/value heads,
+ *     head_dim, kv_len, the start position `pos` of query row 0, f16 K/V and a
+ *     causal mask; section "Summary": a sliding-window lower bound on the keys.
+ *   - "Shmoosh update", sections "The measured changes" and "An explicit
+ *     fast-mode policy": an exact default precision and an opt-in fast mode
+ *     that is never switched on silently.
+ *   - "Ядра attention на домашней RTX 5080", table of section "1 · Только
+ *     ядро": the opt-in mode's form, INT8 Q K^T with FP8 P V.
+ *   - "round 21 track b -- qsa2" (the qsa2 audit), section "implementation and
+ *     review": chunked (split-KV) attention whose partial results are merged
+ *     with cached per-chunk maxima and weights and one denominator.
+ *
+ * Conventions
+ *   - Layout: Q and O are [batch, n_q_heads, q_len, head_dim]; K and V are
+ *     [batch, n_kv_heads, kv_len, head_dim]; all contiguous, head_dim fastest.
+ *     lse is [batch, n_q_heads, q_len] float32.
+ *   - GQA: query head h reads key/value head h / (n_q_heads / n_kv_heads).
+ *   - Query row i sits at absolute position start_pos + i.  With causal != 0
+ *     it sees keys j <= start_pos + i.  Keys j < window_lo are never seen.
+ *     A row that sees no key gets O = 0 and lse = -inf.
+ *   - All tensor pointers are DEVICE pointers owned by the caller and must be
+ *     16-byte aligned; the library never frees them.  `stream` is a
+ *     cudaStream_t passed as void*.  Every call is asynchronous on that stream;
+ *     argument errors are reported synchronously, before anything is launched.
+ *   - A context is not safe for concurrent use from several host threads.
+ *   - Device-side waits are bounded (about 1.5 s).  A wait that runs out
+ *     records an error word in the context; attn_get_error() reports it.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* a parameter or pointer is invalid */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid but not supported (e.g. head_dim, alignment) */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  ATTN_ERR_OOM = 4,         /* workspace allocation failed */
+  ATTN_ERR_TIMEOUT = 5      /* a device-side wait ran out (see attn_get_error) */
+} attn_status;
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype;
+
+/* ATTN_EXACT is the default: 16-bit inputs, f32 accumulation.
+ * ATTN_INT8QK_FP8PV is opt-in: Q/K quantised to INT8 per 128-token block with
+ * FP32 scales, P and V in FP8 E4M3 (V with one FP32 scale per head and channel). */
+typedef enum { ATTN_EXACT = 0, ATTN_INT8QK_FP8PV = 1 } attn_precision;
+
+typedef struct {
+  int batch;       /* B >= 1 */
+  int n_q_heads;   /* Hq >= 1, a multiple of n_kv_heads */
+  int n_kv_heads;  /* Hkv >= 1 */
+  int q_len;       /* Sq >= 0 (0: nothing to do) */
+  int kv_len;      /* Skv >= 0 (0: every row sees no key) */
+  int head_dim;    /* 64 or 128 */
+  int start_pos;   /* absolute position of query row 0, >= 0 */
+  int causal;      /* 0 or 1 */
+  int window_lo;   /* first visible key index, >= 0 (0: no window) */
+  float scale;     /* multiplier of Q K^T; <= 0 selects 1/sqrt(head_dim) */
+  int dtype;       /* attn_dtype of Q, K, V and O */
+  int precision;   /* attn_precision */
+  int num_splits;  /* key/value splits: 0 = chosen by the library, 1 = none, >1 = forced */
+} attn_params;
+
+/* Caller-owned device buffers of the quantised mode (all 16-byte aligned):
+ *   q       int8   [B, Hq,  Sq,  D]          q_scale float [B, Hq,  ceil(Sq/128)]
+ *   k       int8   [B, Hkv, Skv, D]          k_scale float [B, Hkv, ceil(Skv/128)]
+ *   v_t     uint8  [B, Hkv, D, ceil(Skv/128)*128]  E4M3 codes of V, transposed,
+ *                                            zero padded;  v_scale float [B, Hkv, D] */
+typedef struct {
+  int8_t *q;
+  int8_t *k;
+  float *q_scale;
+  float *k_scale;
+  uint8_t *v_t;
+  float *v_scale;
+} attn_qbufs;
+
+typedef struct attn_ctx attn_ctx;
+
+/* Validates `p`, picks the kernel variant and the key/value split for the
+ * current CUDA device, and allocates the context's workspace (split partial
+ * results, the V channel maxima, the device error word).  On success *out
+ * owns that workspace until attn_destroy().  Launches nothing.
+ * Errors: ATTN_ERR_INVALID_ARG (bad field or NULL), ATTN_ERR_UNSUPPORTED
+ * (head_dim not 64/128), ATTN_ERR_CUDA (no device), ATTN_ERR_OOM. */
+attn_status attn_create(const attn_params *p, attn_ctx **out);
+
+/* Quantised mode, step 1 (the per-block quantiser): reads q, k, v (dtype of
+ * the context) and writes every buffer of *qb.  Q and K: per (b, h, 128-token
+ * block) s = max|x| / 127 and code = clamp(round_half_even(x / s), +-127), s = 0
+ * for an all-zero block.  V: per (b, hkv, channel) s = max|v| / 448 and code =
+ * E4M3(v / s) rounded to nearest-even and saturated.  Each step is one
+ * correctly rounded float32 operation, so the bytes are reproducible.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, context not in the
+ * quantised mode), ATTN_ERR_CUDA (launch failure). */
+attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const void *v,
+                             const attn_qbufs *qb, void *stream);
+
+/* The attention forward.  Exact mode: q, k, v are read and qb must be NULL.
+ * Quantised mode: q, k, v are ignored (may be NULL) and qb holds the output of
+ * attn_quantize_qk.  Writes o ([B, Hq, Sq, D], the context's dtype) and, if
+ * lse is not NULL, the natural-log sum of exp(scale * q.k) over each row's
+ * visible keys.  Few-row (decode-shaped) problems are split along the keys and
+ * merged by a second kernel into the same outputs.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, qb presence not
+ * matching the mode), ATTN_ERR_CUDA (tensor-map encode or launch failure). */
+attn_status attn_forward(attn_ctx *c, const void *q, const void *k, const void *v,
+                         const attn_qbufs *qb, void *o, float *lse, void *stream);
+
+/* Synchronises `stream`, reads and clears the context's device error word.
+ * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last call,
+ * ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK. */
+attn_status attn_get_error(attn_ctx *c, void *stream);
+
+/* Frees the context's workspace (after synchronising the device). NULL is ignored. */
+void attn_destroy(attn_ctx *c);
+
+/* Static string naming a status code. */
+const char *attn_status_string(attn_status s);
+
+/* Sizes, in bytes, of the caller-owned buffers of the quantised mode for `p`,
+ * in the order of attn_qbufs (q, k, q_scale, k_scale, v_t, v_scale).  Pure
+ * host arithmetic.  Errors: ATTN_ERR_INVALID_ARG. */
+attn_status attn_qbufs_sizes(const attn_params *p, size_t sizes[6]);
+
+/* Number of key/value splits the context uses (1 = the single-pass kernel). */
+int attn_num_splits(const attn_ctx *c);
+
+/* TEST HOOK.  Bit 0 of `flags` makes the next attn_forward's loader skip the
+ * second key tile of every CTA, so that the waits on it run out: the kernel then
+ * records ATTN_ERR_TIMEOUT in the context and returns without hanging.  The
+ * hook exists only to test that error path; 0 restores normal operation. */
+attn_status attn_debug_set(attn_ctx *c, unsigned flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,89 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every
+function ``include/attn.h`` declares, and rejects bad arguments before touching
+the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_forward_flash_b200 as afb
+from attention_forward_flash_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    L = afb.lib()
+    names = _declared_functions()
+    assert "attn_forward" in names and "attn_create" in names and "attn_quantize_qk" in names
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(names) <= set(_abi.EXPORTED)
+
+
+def _params(**kw):
+    base = dict(batch=1, n_q_heads=2, n_kv_heads=2, q_len=256, kv_len=256, head_dim=64,
+                start_pos=0, causal=0, window_lo=0, scale=0.0, dtype=0, precision=0, num_splits=0)
+    base.update(kw)
+    return _abi.AttnParams(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_q_heads=3, n_kv_heads=2), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(batch=0), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(q_len=-1), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(kv_len=-5), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(start_pos=-1), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(window_lo=-1), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(dtype=7), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(precision=3), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(num_splits=-1), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(num_splits=100000), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(head_dim=96), _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(head_dim=256), _abi.ATTN_ERR_UNSUPPORTED),
+])
+def test_create_rejects_bad_params_before_any_device_call(kw, status):
+    L = afb.lib()
+    ctx = ctypes.c_void_p(1234)
+    p = _params(**kw)
+    assert L.attn_create(ctypes.byref(p), ctypes.byref(ctx)) == status
+    assert ctx.value is None  # *out is cleared on failure
+
+
+def test_null_arguments():
+    L = afb.lib()
+    assert L.attn_create(None, None) == _abi.ATTN_ERR_INVALID_ARG
+    p = _params()
+    assert L.attn_create(ctypes.byref(p), None) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_forward(None, None, None, None, None, None, None, None) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_quantize_qk(None, None, None, None, None, None) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_get_error(None, None) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_debug_set(None, 0) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_num_splits(None) == 0
+    L.attn_destroy(None)
+
+
+def test_status_strings():
+    for s in range(6):
+        assert isinstance(afb.attn_status_string(s), str) and afb.attn_status_string(s)
+    assert afb.attn_status_string(99) == "unknown status"
+
+
+def test_qbufs_sizes():
+    p = _params(batch=2, n_q_heads=8, n_kv_heads=2, q_len=300, kv_len=4133, head_dim=128)
+    q, k, qs, ks, vt, vs = afb.attn_qbufs_sizes(p)
+    assert q == 2 * 8 * 300 * 128 and k == 2 * 2 * 4133 * 128
+    assert qs == 2 * 8 * 3 * 4 and ks == 2 * 2 * 33 * 4
+    assert vt == 2 * 2 * 128 * 33 * 128 and vs == 2 * 2 * 128 * 4
+    with pytest.raises(afb.AttnError):
+        afb.attn_qbufs_sizes(_params(head_dim=80))

@@ -1,0 +1,186 @@
+"""CUDA path (through the C ABI) against the float64 oracle on the same seeded inputs.
+
+Covers every workload at its full size (all rows where the oracle is quick,
+a seeded subset of 256 query rows per head on the two largest), in both
+precision modes where the workload uses them, plus the boundary matrix of key
+lengths, start positions, windows and query-row counts, empty rows, the
+single-pass and split-KV variants, determinism and masked-key independence.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from attention_forward_flash_b200 import Attention
+from attention_forward_flash_b200.inputs import WORKLOADS, Workload, make_qkv, sample_rows
+from parity_util import (EXACT_MAXABS, EXACT_RMSE, QUANT_RMSE, check_exact, check_lse, max_abs,
+                         oracle_for, rel_rmse, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "decode_window", "image"])
+def test_exact_full(name):
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w)
+    o, lse, att = run_gpu(w, q, k, v)
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro, name)
+    check_lse(lse, rl, name)
+    if name.startswith("decode"):
+        assert att.num_splits > 1  # few-row problems take the split-KV path
+
+
+@pytest.mark.parametrize("name", ["video", "llm"])
+def test_exact_full_size_sampled_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w)
+    o, lse, _ = run_gpu(w, q, k, v)
+    rows = sample_rows(w).numpy()
+    ro, rl = oracle_for(w, q, k, v, rows=rows)
+    check_exact(o[:, :, rows], ro, name)
+    check_lse(lse[:, :, rows], rl, name)
+
+
+@pytest.mark.parametrize("name", ["image", "video", "llm"])
+def test_quant_mode(name):
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w)
+    o, lse, _ = run_gpu(w, q, k, v, precision="quant")
+    rows = sample_rows(w).numpy()
+    ro, rl = oracle_for(w, q, k, v, rows=rows)
+    e = rel_rmse(o[:, :, rows], ro)
+    assert e <= QUANT_RMSE, f"{name} quant rel_rmse={e:.4f}"
+    check_lse(lse[:, :, rows], rl, name, tol=0.25)
+
+
+def _small(**kw):
+    base = dict(name="small", batch=1, n_q_heads=4, n_kv_heads=2, q_len=4, kv_len=4096,
+                head_dim=128, dtype="fp16", causal=True, start_pos=4092, seed=41)
+    base.update(kw)
+    return Workload(**base)
+
+
+# query-row counts x start positions x key lengths x window bounds, in the spirit of
+# the qsa2 audit's 40 position/window cases (partial chunks included)
+BOUNDARY = []
+for ntok in (1, 2, 4, 8):
+    for pos0 in (0, 1, 63, 64, 127, 128, 129, 512, 2047, 2048, 2050, 4095):
+        for kv_extra, win in ((1, 0), (0, 40), (37, 127)):
+            kv_len = pos0 + ntok + kv_extra - 1
+            win = min(win, max(pos0, 0))
+            BOUNDARY.append((ntok, pos0, kv_len, win))
+
+
+@pytest.mark.parametrize("ntok,pos0,kv_len,win", BOUNDARY)
+def test_decode_boundary_matrix(ntok, pos0, kv_len, win):
+    w = _small(q_len=ntok, start_pos=pos0, kv_len=kv_len, window_lo=win, seed=41 + pos0)
+    q, k, v = make_qkv(w)
+    o, lse, _ = run_gpu(w, q, k, v)
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro, str((ntok, pos0, kv_len, win)))
+    check_lse(lse, rl)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal,start_pos,window_lo,Sq,Skv", [
+    (False, 0, 0, 1000, 1000),
+    (True, 0, 0, 1000, 1000),
+    (True, 0, 0, 777, 1291),
+    (True, 300, 0, 700, 1000),
+    (False, 0, 200, 513, 1111),
+    (True, 0, 130, 1000, 1000),
+    (True, 0, 0, 129, 129),
+])
+def test_single_pass_ragged(D, causal, start_pos, window_lo, Sq, Skv):
+    w = Workload("ragged", 2, 4, 2, Sq, Skv, D, "bf16", causal=causal, start_pos=start_pos,
+                 window_lo=window_lo, seed=7 + Sq)
+    q, k, v = make_qkv(w)
+    o, lse, att = run_gpu(w, q, k, v, num_splits=1)
+    assert att.num_splits == 1
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro)
+    check_lse(lse, rl)
+
+
+@pytest.mark.parametrize("splits", [2, 3, 7])
+def test_forced_splits(splits):
+    w = Workload("split", 1, 4, 1, 300, 2000, 128, "bf16", causal=True, start_pos=1700, seed=9)
+    q, k, v = make_qkv(w)
+    o, lse, att = run_gpu(w, q, k, v, num_splits=splits)
+    assert att.num_splits > 1
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro)
+    check_lse(lse, rl)
+
+
+@pytest.mark.parametrize("num_splits", [0, 1])
+def test_rows_that_see_no_key(num_splits):
+    # causal from position 0 with a window starting at key 5: rows 0..4 see nothing
+    w = Workload("empty", 1, 2, 2, 300, 300, 64, "bf16", causal=True, window_lo=5, seed=3)
+    q, k, v = make_qkv(w)
+    o, lse, _ = run_gpu(w, q, k, v, num_splits=num_splits)
+    assert np.all(o[:, :, :5] == 0) and np.all(lse[:, :, :5] == -math.inf)
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro)
+    check_lse(lse, rl)
+
+
+def test_zero_kv_len_and_window_past_end():
+    w = Workload("nokv", 1, 2, 1, 5, 0, 128, "fp16")
+    att = Attention(1, 2, 1, 5, 0, 128, dtype=torch.float16)
+    q = torch.randn(1, 2, 5, 128, device="cuda").half()
+    kv = torch.empty(1, 1, 0, 128, device="cuda").half()
+    out = torch.full((1, 2, 5, 128), 7.0, device="cuda").half()
+    out, lse = att.forward(q, kv, kv, out=out, return_lse=True)
+    att.check_error()
+    assert torch.all(out == 0) and torch.all(lse == -math.inf)
+    w = Workload("pastend", 1, 2, 1, 5, 100, 128, "fp16", window_lo=100, seed=2)
+    q, k, v = make_qkv(w)
+    o, lse, _ = run_gpu(w, q, k, v)
+    assert np.all(o == 0) and np.all(lse == -math.inf)
+
+
+def test_deterministic():
+    w = WORKLOADS["image"].scaled(batch=1)
+    q, k, v = (t.cuda() for t in make_qkv(w))
+    for precision in ("exact", "quant"):
+        att = Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
+                        precision=precision)
+        a = att.forward(q, k, v)
+        b = att.forward(q, k, v)
+        att.check_error()
+        assert torch.equal(a, b)
+
+
+def test_masked_keys_do_not_matter():
+    w = Workload("mask", 1, 4, 2, 200, 700, 128, "bf16", causal=True, start_pos=300,
+                 window_lo=77, seed=4)
+    q, k, v = make_qkv(w)
+    o1, l1, _ = run_gpu(w, q, k, v)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, :77] = 1e4
+    v2[:, :, :77] = -3e4
+    k2[:, :, 500:] = float("nan")   # beyond every row's causal limit (300 + 199)
+    v2[:, :, 500:] = 3e4
+    o2, l2, _ = run_gpu(w, q, k2, v2)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    from attention_forward_flash_b200 import _abi
+    w = Workload("timeout", 1, 2, 2, 256, 1024, 64, "bf16", seed=8)
+    q, k, v = (t.cuda() for t in make_qkv(w))
+    att = Attention(1, 2, 2, 256, 1024, 64, num_splits=1)
+    _abi.attn_debug_set(att.ctx, 1)
+    att.forward(q, k, v)
+    with pytest.raises(_abi.AttnError) as e:
+        att.check_error()
+    assert e.value.status == _abi.ATTN_ERR_TIMEOUT
+    _abi.attn_debug_set(att.ctx, 0)
+    o = att.forward(q, k, v)
+    att.check_error()
+    ro, _ = oracle_for(w, *(t.cpu() for t in (q, k, v)))
+    check_exact(o.double().cpu().numpy(), ro)
