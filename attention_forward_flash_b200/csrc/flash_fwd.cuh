@@ -97,6 +97,8 @@ struct FwdCfg {
   // softmax rescale threshold (base-2 units).  Quantised: P*2^8 must stay
   // within the E4M3 range (448), so the max is tracked exactly.
   static constexpr float kRescaleThresh = QUANT ? 0.0f : 8.0f;
+  static constexpr int kRegsLow = 64;    // loader / MMA warpgroup (two-tile variant)
+  static constexpr int kRegsHigh = 216;  // softmax warpgroups (two-tile variant)
 };
 
 template <bool F16>
@@ -107,6 +109,18 @@ __device__ __forceinline__ uint32_t pack_16x2(float lo, float hi) {
   } else {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+template <bool F16>
+__device__ __forceinline__ void unpack_16x2(uint32_t v, float& lo, float& hi) {
+  if constexpr (F16) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+    lo = f.x;
+    hi = f.y;
+  } else {
+    lo = __uint_as_float(v << 16);
+    hi = __uint_as_float(v & 0xFFFF0000u);
   }
 }
 
@@ -206,11 +220,19 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // Two-tile variant: 384 threads launched at 168 registers each (64512).  The
+  // loader/MMA warpgroup needs few, the softmax warpgroups many:
+  // 128 x 56 + 256 x 224 = 64512, exactly the launch budget.
+  static_assert(NQT != 2 || 128 * C::kRegsLow + 256 * C::kRegsHigh <= C::kThreads * 168,
+                "register split");
+
   auto raise = [&]() {
     *abort_flag = 1;
     atomicOr(a.err, (unsigned)kErrTimeout);
   };
 
+  if (warp < 4) {
+  if constexpr (NQT == 2) regs_dec<C::kRegsLow>();
   if (warp == 0) {
     // ======================================================== TMA producer
     if (lane == 0) {
@@ -367,7 +389,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
       while (!mbar_try_wait(o_final, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    if constexpr (NQT == 2) regs_inc<C::kRegsHigh>();
     // ============================================================ softmax
     const int q = (warp - 4) >> 2;            // query tile of this warpgroup
     const int wq = warp & 3;                  // TMEM lane quarter
@@ -433,9 +457,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
           if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
         }
       }
-      float mx = x[0];
+      // row max: eight independent chains, then a tree
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      for (int e = 0; e < 8; ++e) mx8[e] = x[e];
+#pragma unroll
+      for (int c = 8; c < 128; c += 8)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[c + e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * cj;  // cj > 0; -inf stays -inf
       const float m_prev = m_used;
       const float m_new = fmaxf(m_prev, m_tile);
@@ -454,34 +485,43 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
           tmem_st32(tO + c0, o);
         }
       }
-      // P = 2^(x * cj - m)  (quantised: times 2^8 before the E4M3 cast)
+      // P = 2^(x * cj - m)  (quantised: times 2^8 before the E4M3 cast), written
+      // over S in 32-key chunks.  Exact mode: the row sum adds the 16-bit values
+      // that the P.V product actually uses, so O is a convex combination of V rows.
       const float mb = (m_used == -INFINITY ? 0.0f : m_used) - (QUANT ? 8.0f : 0.0f);
-      float rs = 0.0f;
+      float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2(fmaf(x[c], cj, -mb));
-        rs += x[c];
-      }
-      l += rs;
-      if constexpr (QUANT) {
-        uint32_t pk[32];
+      for (int ch = 0; ch < 4; ++ch) {
+        if constexpr (QUANT) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const uint32_t lo = f32x2_to_e4m3x2(x[4 * c], x[4 * c + 1]);
-          const uint32_t hi = f32x2_to_e4m3x2(x[4 * c + 2], x[4 * c + 3]);
-          pk[c] = lo | (hi << 16);
+          for (int c = 0; c < 8; ++c) {
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              p[e] = ex2(fmaf(x[32 * ch + 4 * c + e], cj, -mb));
+              rs4[e] += p[e];
+            }
+            pk[c] = uint32_t(f32x2_to_e4m3x2(p[0], p[1])) |
+                    (uint32_t(f32x2_to_e4m3x2(p[2], p[3])) << 16);
+          }
+          tmem_st8(tS + 8 * ch, pk);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ex2(fmaf(x[32 * ch + 2 * c], cj, -mb));
+            const float p1 = ex2(fmaf(x[32 * ch + 2 * c + 1], cj, -mb));
+            pk[c] = pack_16x2<F16>(p0, p1);
+            float r0, r1;
+            unpack_16x2<F16>(pk[c], r0, r1);
+            rs4[(2 * c) & 3] += r0;
+            rs4[(2 * c + 1) & 3] += r1;
+          }
+          tmem_st16(tS + 16 * ch, pk);
         }
-        tmem_st32(tS, pk);
-      } else {
-        uint32_t pk0[32], pk1[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          pk0[c] = pack_16x2<F16>(x[2 * c], x[2 * c + 1]);
-          pk1[c] = pack_16x2<F16>(x[64 + 2 * c], x[64 + 2 * c + 1]);
-        }
-        tmem_st32(tS, pk0);
-        tmem_st32(tS + 32, pk1);
       }
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready(q));

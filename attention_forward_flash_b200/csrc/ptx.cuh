@@ -242,8 +242,39 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 #undef ATTN_RI
 
+#define ATTN_RI(i) "r"(r[i])
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      ATTN_RI(0), ATTN_RI(1), ATTN_RI(2), ATTN_RI(3), ATTN_RI(4), ATTN_RI(5), ATTN_RI(6),
+      ATTN_RI(7), ATTN_RI(8), ATTN_RI(9), ATTN_RI(10), ATTN_RI(11), ATTN_RI(12), ATTN_RI(13),
+      ATTN_RI(14), ATTN_RI(15)
+      : "memory");
+}
+#undef ATTN_RI
+
+#define ATTN_RI(i) "r"(r[i])
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               ATTN_RI(0), ATTN_RI(1), ATTN_RI(2), ATTN_RI(3), ATTN_RI(4), ATTN_RI(5), ATTN_RI(6),
+               ATTN_RI(7)
+               : "memory");
+}
+#undef ATTN_RI
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Per-warpgroup register budget changes (all warps of a warpgroup execute them).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------- arithmetic

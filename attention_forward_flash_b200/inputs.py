@@ -106,6 +106,27 @@ def make_qkv(w: Workload, device="cpu"):
     return out
 
 
+def make_qkv_device(w: Workload, device):
+    """Same recipe as ``make_qkv`` but drawn by a generator on ``device``.
+
+    Used where only the distribution matters (timing); the random stream differs
+    from the CPU one, so parity tests use ``make_qkv``.
+    """
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    qs, ks = w.shapes()
+    dt = w.torch_dtype
+    q = torch.randn(qs, generator=g, device=device, dtype=torch.float32).to(dt)
+    k = torch.randn(ks, generator=g, device=device, dtype=torch.float32)
+    v = torch.randn(ks, generator=g, device=device, dtype=torch.float32).to(dt)
+    if w.k_channel_offset_var > 0:
+        k += torch.randn((w.batch, w.n_kv_heads, 1, w.head_dim), generator=g, device=device,
+                         dtype=torch.float32) * math.sqrt(w.k_channel_offset_var)
+    if w.k_outlier_frac > 0:
+        sel = torch.rand(ks, generator=g, device=device, dtype=torch.float32) < w.k_outlier_frac
+        k = torch.where(sel, k * w.k_outlier_mult, k)
+    return q, k.to(dt), v
+
+
 def sample_rows(w: Workload, n=None, seed=None):
     """Seeded subset of query rows (sorted) evaluated by the oracle on large workloads."""
     n = w.oracle_rows if n is None else n

@@ -1,0 +1,506 @@
+"""Benchmark of the fused attention forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload video]
+                    [--precision exact|quant] [--impl native|reference] [--no-extra]
+
+A step is one call of the hot path on one batch of synthetic input already
+resident in HBM: ``attn_forward`` (plus ``attn_quantize_qk`` in the quantised
+mode).  The headline workload is the 1 x 40 x 32760 x 128 bf16 self-attention
+of section "1 · Только ядро" of the page "Ядра attention на домашней RTX 5080".
+The metric is attention TFLOP/s = 4*B*Hq*Sq*Skv*D (halved for causal) / time.
+
+With N > 1 (torchrun) every rank runs its own copy of the workload (the
+problems are independent; no collective is on the data path): the value is the
+work of all ranks over the slowest rank's device time ("scaling": "weak").
+
+``--impl reference`` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_forward_flash_b200.inputs import WORKLOADS, Workload, make_qkv_device  # noqa: E402
+
+METRIC = "attention TFLOP/s (4·B·Hq·Sq·Skv·d, causal halved) and % of B200 tensor peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="video", choices=sorted(WORKLOADS))
+    ap.add_argument("--precision", default="exact", choices=["exact", "quant"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="run the workload with this many kv heads (same group size); for "
+                         "profiling captures on a smaller case")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def max_over_ranks(x, world):
+    """Largest value of ``x`` across ranks (host plumbing, not the data path)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "attention_forward_flash_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, precision):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for line in open(path):
+        m = re.match(r"\s*(\w+)\s+(\w+)\s+([0-9a-f]{16})\s+([0-9.eE+]+)", line)
+        if m and m.group(1) == workload and m.group(2) == precision and m.group(3) == src:
+            return float(m.group(4))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], cap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        load = [r for r in rows if r["power"] > 300] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("cap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(load), "power_w_median": statistics.median(r["power"] for r in load)}
+
+
+def make_attention(w: Workload, precision):
+    from attention_forward_flash_b200 import Attention
+    return Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
+                     dtype=w.torch_dtype, causal=w.causal, start_pos=w.start_pos,
+                     window_lo=w.window_lo, precision=precision)
+
+
+def launches_per_step(att, precision):
+    n = 1 + (1 if att.num_splits > 1 else 0)
+    if precision == "quant":
+        n += 4  # Q and K block quantisers, V channel maxima, V quantiser
+    return n
+
+
+def time_steps(fn, steps, warmup, flush=None):
+    """Device time per step (ms) of ``fn``: CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+    total = 0.0
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    return total / steps
+
+
+# ------------------------------------------------------- CPU oracle timing
+def oracle_sample_time(w: Workload, target_s=12.0, max_rows=None, seed=0):
+    """Times the float64 oracle on a bounded sample: the first ``r`` query rows of
+    every (batch, q-head), r grown until one run takes about ``target_s``.
+    Returns (flops, seconds, description, threads)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import attention_f64
+    from attention_forward_flash_b200.inputs import make_qkv
+
+    small = w.scaled(q_len=min(w.q_len, 4096)) if w.q_len > 4096 else w
+    q, k, v = make_qkv(small)
+    rows_cap = max_rows or w.q_len
+    r = 8
+    while True:
+        rows = np.linspace(0, small.q_len - 1, min(r, small.q_len)).astype(np.int64)
+        t0 = time.perf_counter()
+        attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
+                      rows=rows)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or r >= min(rows_cap, small.q_len):
+            break
+        r = min(r * 4, rows_cap, small.q_len)
+    # scale the sample so that it takes about target_s
+    if dt < target_s and r < min(rows_cap, small.q_len):
+        r = int(min(rows_cap, small.q_len, max(r, r * target_s / max(dt, 1e-3))))
+        rows = np.linspace(0, small.q_len - 1, r).astype(np.int64)
+        t0 = time.perf_counter()
+        attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
+                      rows=rows)
+        dt = time.perf_counter() - t0
+    from oracle import visible_range
+    pairs = 0
+    for i in rows:
+        lo, hi = visible_range(int(i), kv_len=w.kv_len, start_pos=w.start_pos, causal=w.causal,
+                               window_lo=w.window_lo)
+        pairs += max(0, hi - lo + 1)
+    flops = 4.0 * w.batch * w.n_q_heads * pairs * w.head_dim
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    desc = (f"{len(rows)} evenly spaced query rows x {w.batch * w.n_q_heads} heads of the "
+            f"{w.name} workload (all {w.kv_len} keys each), float64 numpy")
+    return flops, dt, desc, threads
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    # size one step so that the whole run stays within a few minutes
+    per_step_s = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    flops, dt, desc, threads = oracle_sample_time(w, target_s=per_step_s)
+    import numpy as np
+
+    from oracle import attention_f64
+    from attention_forward_flash_b200.inputs import make_qkv
+    small = w.scaled(q_len=min(w.q_len, 4096)) if w.q_len > 4096 else w
+    q, k, v = make_qkv(small)
+    nrows = int(re.match(r"(\d+)", desc).group(1))
+    rows = np.linspace(0, small.q_len - 1, nrows).astype(np.int64)
+
+    def step():
+        attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
+                      rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    ms = (time.perf_counter() - t0) * 1e3 / args.steps
+    value = flops / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, args.precision),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: Workload, precision):
+    in_bytes = (w.batch * w.n_q_heads * w.q_len + 2 * w.batch * w.n_kv_heads * w.kv_len) * \
+        w.head_dim * 2
+    return {"workload": w.name, "batch": w.batch, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": w.n_kv_heads, "q_len": w.q_len, "kv_len": w.kv_len,
+            "head_dim": w.head_dim, "causal": w.causal, "start_pos": w.start_pos,
+            "window_lo": w.window_lo, "precision": precision, "input_dtype": w.dtype,
+            "l2": (f"inputs {in_bytes / 1e9:.2f} GB > 126 MB L2" if in_bytes > L2_BYTES
+                   else "L2 flushed (256 MB write) before every timed call"),
+            "parallelism": "replicas (independent problem per GPU)"}
+
+
+# ------------------------------------------------------------ native arm
+def measure(w: Workload, precision, steps, warmup, device):
+    """Device ms per step (resident inputs), ms of the dominant kernel, launches."""
+    att = make_attention(w, precision)
+    q, k, v = make_qkv_device(w, device)
+    out = torch.empty((w.batch, w.n_q_heads, w.q_len, w.head_dim), dtype=w.torch_dtype,
+                      device=device)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    flush = None
+    if in_bytes <= L2_BYTES:
+        scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+        flush = lambda: scratch.fill_(1)  # noqa: E731
+    qb = att.quantize(q, k, v) if precision == "quant" else None
+
+    def step():
+        if precision == "quant":
+            att.quantize(q, k, v, qbufs=qb)
+            att.forward(qbufs=qb, out=out)
+        else:
+            att.forward(q, k, v, out=out)
+
+    def kernel_only():
+        att.forward(q, k, v, qbufs=qb, out=out)
+
+    ms_step = time_steps(step, steps, warmup, flush)
+    ms_kernel = ms_step if precision == "exact" else time_steps(kernel_only, steps, 2, flush)
+    att.check_error()
+    return dict(ms_step=ms_step, ms_kernel=ms_kernel, att=att, q=q, k=k, v=v, out=out, qb=qb,
+                launches=launches_per_step(att, precision))
+
+
+def measure_e2e(w: Workload, precision, m, steps, warmup):
+    """Same metric through the public API with host buffers: every step copies
+    Q, K, V from pinned host memory, runs the call, and copies O back."""
+    att = m["att"]
+    hq, hk, hv = (t.cpu().pin_memory() for t in (m["q"], m["k"], m["v"]))
+    ho = torch.empty(m["out"].shape, dtype=m["out"].dtype).pin_memory()
+    dq, dk, dv, do = (torch.empty_like(t) for t in (m["q"], m["k"], m["v"], m["out"]))
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if precision == "quant":
+            qb = att.quantize(dq, dk, dv, qbufs=m["qb"])
+            att.forward(qbufs=qb, out=do)
+        else:
+            att.forward(dq, dk, dv, out=do)
+        ho.copy_(do, non_blocking=True)
+
+    ms = time_steps(step, steps, warmup)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
+    return ms, h2d, d2h
+
+
+def run_native(args):
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    peaks, peak_src = load_peaks()
+    w = WORKLOADS[args.workload]
+    if args.kv_heads:
+        g = w.n_q_heads // w.n_kv_heads
+        w = w.scaled(n_kv_heads=args.kv_heads, n_q_heads=args.kv_heads * g,
+                     name=f"{w.name}_kvh{args.kv_heads}")
+    precision = args.precision
+    if precision not in w.modes:
+        raise SystemExit(f"workload {w.name} is not run in {precision} mode")
+
+    # ---- headline: resident inputs, K timed steps between barriers
+    m = measure(w, precision, 1, max(args.warmup, 3), device)  # build + warm
+    att, step_args = m["att"], m
+    out, q, k, v, qb = m["out"], m["q"], m["k"], m["v"], m["qb"]
+
+    def step():
+        if precision == "quant":
+            att.quantize(q, k, v, qbufs=qb)
+            att.forward(qbufs=qb, out=out)
+        else:
+            att.forward(q, k, v, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local_rank) as clocks:
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    att.check_error()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    flops = w.flops()
+    value = flops * world / (ms * 1e-3) / 1e12
+
+    # ---- dominant kernel (the fused attention kernel) for the roofline
+    if precision == "quant":
+        ms_kernel = time_steps(lambda: att.forward(qbufs=qb, out=out), args.steps, 2)
+    else:
+        ms_kernel = ms_local
+    peak_key = "bf16_tflops"
+    peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
+    if precision == "quant":
+        peak = 2.0 * peak  # INT8 / FP8 dense rate = 2x the bf16 rate (nominal 4.5 vs 2.25 PF)
+    achieved = flops / (ms_kernel * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(w.name, precision),
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" +
+                (" x2 for INT8/FP8" if precision == "quant" else ""),
+                "kernel": "flash_fwd_kernel", "kernel_ms": ms_kernel}
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_ms, h2d, d2h = measure_e2e(w, precision, m, e2e_steps, 2)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if precision == "exact" else "int8/fp8e4m3",
+        "data": "synthetic (seeded N(0,1), workload recipe of attention_forward_flash_b200.inputs)",
+        "config": workload_config(w, precision),
+        "pct_of_peak": 100.0 * achieved / peak,
+        "roofline": roofline, "e2e": e2e,
+        "gpu_launches": m["launches"] * args.steps,
+        "clocks": clocks.summary(),
+    }
+
+    # ---- secondary measurements (other workloads and modes), rank 0 prints them
+    if not args.no_extra:
+        extra = {}
+        for name, prec in (("video", "quant" if precision == "exact" else "exact"),
+                           ("llm", "exact"), ("llm", "quant"), ("image", "exact"),
+                           ("image", "quant"), ("decode", "exact"), ("decode_window", "exact")):
+            if name == w.name and prec == precision:
+                continue
+            wx = WORKLOADS[name]
+            mx = measure(wx, prec, 10 if wx.flops() > 1e12 else 50, 3, device)
+            fl = wx.flops()
+            entry = {"ms_per_step": mx["ms_step"], "ms_kernel": mx["ms_kernel"],
+                     "tflops_step": fl / (mx["ms_step"] * 1e-3) / 1e12,
+                     "tflops_kernel": fl / (mx["ms_kernel"] * 1e-3) / 1e12,
+                     "splits": mx["att"].num_splits}
+            if name.startswith("decode"):
+                kv_bytes = 2 * wx.batch * wx.n_kv_heads * wx.kv_len * wx.head_dim * 2
+                entry["hbm_gbs_kernel"] = kv_bytes / (mx["ms_kernel"] * 1e-3) / 1e9
+                entry["us_per_call"] = mx["ms_kernel"] * 1e3
+            if prec == "quant":
+                entry["pct_of_int8_peak_kernel"] = 100 * entry["tflops_kernel"] / (2 * peaks.get(
+                    "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+            else:
+                entry["pct_of_bf16_peak_kernel"] = 100 * entry["tflops_kernel"] / peaks.get(
+                    "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            extra[f"{name}/{prec}"] = entry
+            del mx
+            torch.cuda.empty_cache()
+        line["extra"] = extra
+
+    # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops_s, dt, desc, threads = oracle_sample_time(w, target_s=12.0)
+        line["cpu_baseline"] = {"value": flops_s / dt / 1e12, "unit": "TFLOP/s",
+                                "cores": threads, "kind": "oracle", "sample": desc,
+                                "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
