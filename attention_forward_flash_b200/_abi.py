@@ -11,7 +11,8 @@ ATTN_BF16, ATTN_FP16 = 0, 1
 ATTN_EXACT, ATTN_INT8QK_FP8PV = 0, 1
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
-            "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set")
+            "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
+            "attn_debug_exp2")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -71,6 +72,8 @@ def lib():
         L.attn_num_splits.restype = c_int
         L.attn_debug_set.argtypes = [vp, ctypes.c_uint]
         L.attn_debug_set.restype = c_int
+        L.attn_debug_exp2.argtypes = [vp, vp, ctypes.c_size_t, vp]
+        L.attn_debug_exp2.restype = c_int
         _LIB = L
     return _LIB
 
@@ -119,3 +122,7 @@ def attn_num_splits(ctx):
 
 def attn_debug_set(ctx, flags):
     _check(lib().attn_debug_set(ctx, flags), "attn_debug_set")
+
+
+def attn_debug_exp2(x, y, n, stream):
+    _check(lib().attn_debug_exp2(x, y, n, stream), "attn_debug_exp2")

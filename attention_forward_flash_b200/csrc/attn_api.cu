@@ -216,7 +216,7 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
     opart_off = off;
     off += (static_cast<size_t>(c->splits) * rows * p->head_dim * 4 + 255) / 256 * 256;
     lpart_off = off;
-    off += (static_cast<size_t>(c->splits) * rows * 4 + 255) / 256 * 256;
+    off += (2 * static_cast<size_t>(c->splits) * rows * 4 + 255) / 256 * 256;
   }
   if (cudaMalloc(&c->ws, off) != cudaSuccess) {
     cudaGetLastError();
@@ -253,6 +253,14 @@ attn_status attn_debug_set(attn_ctx* c, unsigned flags) {
   return ATTN_OK;
 }
 
+attn_status attn_debug_exp2(const float* x, float* y, size_t n, void* stream) {
+  if ((!x || !y) && n > 0) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  poly_exp2_kernel<<<ceil_div(static_cast<long long>(n), 256), 256, 0,
+                     static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 attn_status attn_get_error(attn_ctx* c, void* stream) {
   if (!c) return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -268,13 +276,17 @@ attn_status attn_get_error(attn_ctx* c, void* stream) {
 
 attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const void* v,
                              const attn_qbufs* qb, void* stream) {
-  if (!c || !qb || !q || !k || !v) return ATTN_ERR_INVALID_ARG;
+  if (!c || !qb) return ATTN_ERR_INVALID_ARG;
   if (c->p.precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
-  if (!qb->q || !qb->k || !qb->q_scale || !qb->k_scale || !qb->v_t || !qb->v_scale)
+  // Buffers of zero length may be NULL (an empty tensor has no storage).
+  const bool need_q = c->p.q_len > 0, need_kv = c->p.kv_len > 0;
+  auto bad = [](const void* ptr, bool needed) {
+    return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));
+  };
+  if (bad(q, need_q) || bad(qb->q, need_q) || bad(qb->q_scale, need_q) || bad(k, need_kv) ||
+      bad(v, need_kv) || bad(qb->k, need_kv) || bad(qb->k_scale, need_kv) ||
+      bad(qb->v_t, need_kv) || bad(qb->v_scale, need_kv))
     return ATTN_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, qb->q, qb->k, qb->q_scale, qb->k_scale, qb->v_t, qb->v_scale};
-  for (const void* ptr : ptrs)
-    if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D = p.head_dim;
@@ -316,20 +328,24 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
 
 attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* v,
                          const attn_qbufs* qb, void* o, float* lse, void* stream) {
-  if (!c || !o) return ATTN_ERR_INVALID_ARG;
+  if (!c) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
   const bool quant = p.precision == ATTN_INT8QK_FP8PV;
+  // Buffers of zero length may be NULL (an empty tensor has no storage).
+  const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
+  auto bad = [](const void* ptr, bool needed) {
+    return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));
+  };
+  if (bad(o, need_q) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
   if (quant) {
-    if (!qb || !qb->q || !qb->k || !qb->q_scale || !qb->k_scale || !qb->v_t || !qb->v_scale)
+    if (!qb) return ATTN_ERR_INVALID_ARG;
+    if (bad(qb->q, need_q) || bad(qb->q_scale, need_q) || bad(qb->k, need_kv) ||
+        bad(qb->k_scale, need_kv) || bad(qb->v_t, need_kv) || bad(qb->v_scale, need_kv))
       return ATTN_ERR_INVALID_ARG;
-    const void* ptrs[] = {qb->q, qb->k, qb->q_scale, qb->k_scale, qb->v_t, qb->v_scale};
-    for (const void* ptr : ptrs)
-      if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
   } else {
-    if (qb || !q || !k || !v) return ATTN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_INVALID_ARG;
+    if (qb) return ATTN_ERR_INVALID_ARG;
+    if (bad(q, need_q) || bad(k, need_kv) || bad(v, need_kv)) return ATTN_ERR_INVALID_ARG;
   }
-  if (!aligned16(o) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D = p.head_dim;

@@ -23,7 +23,7 @@
 //    merge kernel; qsa2 audit, "implementation and review").
 //
 // Quantised variant (QUANT): Q/K are INT8 codes with one float32 scale per
-// 128-token block (kind::i8 MMA, s32 accumulators), P is E4M3 scaled by 2^8,
+// 128-token block (kind::i8 MMA, s32 accumulators), P is E4M3 scaled by 2^7,
 // V^T is E4M3 with per-channel scales (kind::f8f6f4 MMA); this is the
 // "INT8 QK · FP8 PV" form of the table in section "1 · Только ядро" of the page
 // "Ядра attention на домашней RTX 5080".
@@ -51,7 +51,8 @@ struct FwdArgs {
   float scale_log2;  // scale * log2(e)
   float* lse;        // [units * R] natural-log lse or nullptr (non-split variant)
   float* o_part;     // [splits, units, R, D] float32 (split variant)
-  float* lse_part;   // [splits, units, R] base-2 lse (split variant)
+  float* lse_part;   // [2, splits, units, R] base-2 lse of the P.V weights, then of the
+                     // float32 weights (split variant)
   const float* q_scale;  // quantised variant
   const float* k_scale;
   const float* v_scale;
@@ -94,9 +95,12 @@ struct FwdCfg {
   static constexpr uint32_t kQBytes = NQT * kQTile;
   static constexpr uint32_t kKBytes = kKTile;
   static constexpr uint32_t kVBytes = kVTile;
-  // softmax rescale threshold (base-2 units).  Quantised: P*2^8 must stay
-  // within the E4M3 range (448), so the max is tracked exactly.
-  static constexpr float kRescaleThresh = QUANT ? 0.0f : 8.0f;
+  // softmax rescale threshold (base-2 units): O and l are rescaled only when a
+  // row max grows by more than this, so P <= 2^thresh.  Quantised: P is scaled by
+  // 2^kPScale before the E4M3 cast and 2^(kPScale + thresh) = 2^8.8 ~ 445 stays
+  // within the largest finite E4M3 value (448).
+  static constexpr float kRescaleThresh = QUANT ? 1.8f : 8.0f;
+  static constexpr float kPScale = QUANT ? 7.0f : 0.0f;
   static constexpr int kRegsLow = 64;    // loader / MMA warpgroup (two-tile variant)
   static constexpr int kRegsHigh = 216;  // softmax warpgroups (two-tile variant)
 };
@@ -124,9 +128,73 @@ __device__ __forceinline__ void unpack_16x2(uint32_t v, float& lo, float& hi) {
   }
 }
 
-// Exact conversion of |s| < 2^22 integers to float with integer + float adds.
-__device__ __forceinline__ float s32_to_f32(uint32_t s) {
-  return __uint_as_float(s + 0x4B400000u) - 12582912.0f;
+// P = 2^(x * cj - mb) for one 128-key row chunk: written over S in tensor memory
+// (16-bit pairs, or E4M3 quads in the quantised mode) and added to the row sums.
+// POLY: every fourth exponential runs on the FMA pipe instead of the MUFU.
+template <bool F16, bool QUANT, bool POLY>
+__device__ __forceinline__ void softmax_emit(const float (&x)[128], float cj, float mb,
+                                             uint32_t tS, float& l, float& lf) {
+  const f32x2 cc{cj, cj}, mm{-mb, -mb};
+  f32x2 fs0{0.0f, 0.0f}, fs1{0.0f, 0.0f}, rs0{0.0f, 0.0f}, rs1{0.0f, 0.0f};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    if constexpr (QUANT) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int e = 32 * ch + 4 * c;
+        const f32x2 t0 = ffma2(f32x2{x[e], x[e + 1]}, cc, mm);
+        const f32x2 t1 = ffma2(f32x2{x[e + 2], x[e + 3]}, cc, mm);
+        float p0, p1;
+        if (POLY && (c % 2 == 0)) {
+          p0 = poly_ex2(t0.x);
+          p1 = poly_ex2(t0.y);
+        } else {
+          p0 = ex2(t0.x);
+          p1 = ex2(t0.y);
+        }
+        const float p2 = ex2(t1.x), p3 = ex2(t1.y);
+        pk[c] = uint32_t(f32x2_to_e4m3x2(p0, p1)) | (uint32_t(f32x2_to_e4m3x2(p2, p3)) << 16);
+        fs0 = fadd2(fs0, f32x2{p0, p1});
+        fs1 = fadd2(fs1, f32x2{p2, p3});
+      }
+      tmem_st8(tS + 8 * ch, pk);
+    } else {
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int e = 32 * ch + 2 * c;
+        const f32x2 t = ffma2(f32x2{x[e], x[e + 1]}, cc, mm);
+        float p0, p1;
+        if (POLY && (c % 4 == 0)) {
+          p0 = poly_ex2(t.x);
+          p1 = poly_ex2(t.y);
+        } else {
+          p0 = ex2(t.x);
+          p1 = ex2(t.y);
+        }
+        pk[c] = pack_16x2<F16>(p0, p1);
+        float r0, r1;
+        unpack_16x2<F16>(pk[c], r0, r1);
+        if (c & 1) {
+          rs1 = fadd2(rs1, f32x2{r0, r1});
+          fs1 = fadd2(fs1, f32x2{p0, p1});
+        } else {
+          rs0 = fadd2(rs0, f32x2{r0, r1});
+          fs0 = fadd2(fs0, f32x2{p0, p1});
+        }
+      }
+      tmem_st16(tS + 16 * ch, pk);
+    }
+  }
+  const float fsum = (fs0.x + fs0.y) + (fs1.x + fs1.y);
+  if constexpr (QUANT) {
+    l += fsum;
+    lf += fsum;
+  } else {
+    l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
+    lf += fsum;
+  }
 }
 
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT>
@@ -305,38 +373,44 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
       if (!ok) raise();
       int it = 0;
 
-      auto issue_qk = [&](int q, uint32_t kslot) {
-        const uint32_t qs = sbase + C::kQOff + q * C::kQTile;
+      // Descriptor words: the high word is fixed per operand kind; the low word
+      // is the start address (>> 4) plus a compile-time offset per K step.
+      constexpr uint32_t hi_qk =
+          QUANT ? desc_hi(D == 128 ? 1024u : 512u, D == 128 ? 2u : 4u) : desc_hi(1024u, 2u);
+      constexpr uint32_t hi_v = desc_hi(1024u, 2u);
+      constexpr uint32_t lbo_v = QUANT ? 16u : 128u * 128u;  // exact: 64-column halves of V
+      const uint32_t q_lo0 = desc_lo(sbase + C::kQOff, 16);
+      const uint32_t ring_lo = desc_lo(sbase + C::kRingOff, 16);
+      const uint32_t ring_lo_v = desc_lo(sbase + C::kRingOff, lbo_v);
+      auto issue_qk = [&](int q, uint32_t k_lo) {
+        const uint32_t q_lo = q_lo0 + q * (C::kQTile >> 4);
         const uint32_t d = tmem + q * 128;
         if constexpr (QUANT) {
           // int8, K = D bytes per row: one swizzle atom column (128 B, or 64 B at D = 64)
-          constexpr uint32_t layout = (D == 128) ? 2u : 4u;
-          constexpr uint32_t sbo = (D == 128) ? 1024u : 512u;
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(d, smem_desc(qs + kk * 32, 16, sbo, layout),
-                      smem_desc(kslot + kk * 32, 16, sbo, layout), idesc_qk, kk > 0);
+            mma_i8_ss(d, desc_pack(q_lo + kk * 2, hi_qk), desc_pack(k_lo + kk * 2, hi_qk),
+                      idesc_qk, kk > 0);
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_f16_ss(d, smem_desc(qs + off, 16, 1024, 2), smem_desc(kslot + off, 16, 1024, 2),
-                       idesc_qk, kk > 0);
+            const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 2;  // (64-col box, 32 B) >> 4
+            mma_f16_ss(d, desc_pack(q_lo + off, hi_qk), desc_pack(k_lo + off, hi_qk), idesc_qk,
+                       kk > 0);
           }
         }
       };
-      auto issue_pv = [&](int q, uint32_t vslot, uint32_t accum) {
+      auto issue_pv = [&](int q, uint32_t v_lo, uint32_t accum) {
         const uint32_t d = tmem + NQT * 128 + q * D;
         const uint32_t p = tmem + q * 128;
         if constexpr (QUANT) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)   // 32 keys (8 columns of 4 e4m3) per step
-            mma_f8_ts(d, p + kk * 8, smem_desc(vslot + kk * 32, 16, 1024, 2), idesc_pv,
-                      (accum | kk) != 0);
+            mma_f8_ts(d, p + kk * 8, desc_pack(v_lo + kk * 2, hi_v), idesc_pv, (accum | kk) != 0);
         } else {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)   // 16 keys (8 columns of 2 x 16-bit) per step
-            mma_f16_ts(d, p + kk * 8, smem_desc(vslot + kk * 2048, 128 * 128, 1024, 2), idesc_pv,
+            mma_f16_ts(d, p + kk * 8, desc_pack(v_lo + kk * 128, hi_v), idesc_pv,
                        (accum | kk) != 0);
         }
       };
@@ -348,9 +422,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
         if (!ok) raise();
         else {
           tc_fence_after();
-          const uint32_t kslot = sbase + C::kRingOff + s * C::kSlot;
+          const uint32_t k_lo = ring_lo + s * (C::kSlot >> 4);
           for (int q = 0; q < NQT; ++q) {
-            issue_qk(q, kslot);
+            issue_qk(q, k_lo);
             tc_commit(s_ready(q));
           }
           tc_commit(empty_bar(s));
@@ -369,15 +443,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
           ++it;
         }
         tc_fence_after();
-        const uint32_t vslot = sbase + C::kRingOff + sv * C::kSlot;
-        const uint32_t kslot = sbase + C::kRingOff + sk * C::kSlot;
+        const uint32_t v_lo = ring_lo_v + sv * (C::kSlot >> 4);
+        const uint32_t k_lo = ring_lo + sk * (C::kSlot >> 4);
         for (int q = 0; q < NQT && ok; ++q) {
           if (!mbar_wait(p_ready(q), j & 1, abort_flag)) { raise(); ok = false; break; }
           tc_fence_after();
-          issue_pv(q, vslot, j > 0);
+          issue_pv(q, v_lo, j > 0);
           if (q == NQT - 1) tc_commit(empty_bar(sv));
           if (has_next) {
-            issue_qk(q, kslot);
+            issue_qk(q, k_lo);
             tc_commit(s_ready(q));
           }
         }
@@ -413,9 +487,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
     }
 
     float m_used = -INFINITY;  // running max of the base-2 scaled scores
-    float l = 0.0f;            // running row sum (relative to m_used)
+    float l = 0.0f;            // row sum of the P values P.V uses (relative to m_used)
+    float lf = 0.0f;           // row sum of the float32 P values (for lse)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
+      float ksc = 1.0f;
+      if constexpr (QUANT) ksc = a.k_scale[(size_t)u * a.nblk_k + jt0 + j];
       ok = __all_sync(0xffffffffu, mbar_wait(s_ready(q), j & 1, abort_flag));
       if (!ok) { if (lane == 0) raise(); break; }
       tc_fence_after();
@@ -432,24 +509,41 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
       tmem_ld_wait(s2);
       tmem_ld_wait(s3);
       float x[128];
-      float cj = a.scale_log2;  // raw-score -> base-2 scaled score factor
+      if constexpr (QUANT) {
+        // s32 -> f32 exactly: the integer plus 1.5*2^23 is a float whose low
+        // mantissa bits hold it; subtract 1.5*2^23 again (packed, two per op).
+        const f32x2 magic{-12582912.0f, -12582912.0f};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        if constexpr (QUANT) {
-          x[c] = s32_to_f32(s0[c]);
-          x[32 + c] = s32_to_f32(s1[c]);
-          x[64 + c] = s32_to_f32(s2[c]);
-          x[96 + c] = s32_to_f32(s3[c]);
-        } else {
+        for (int c = 0; c < 32; c += 2) {
+          f32x2 v = fadd2(f32x2{__uint_as_float(s0[c] + 0x4B400000u),
+                                __uint_as_float(s0[c + 1] + 0x4B400000u)}, magic);
+          x[c] = v.x;
+          x[c + 1] = v.y;
+          v = fadd2(f32x2{__uint_as_float(s1[c] + 0x4B400000u),
+                          __uint_as_float(s1[c + 1] + 0x4B400000u)}, magic);
+          x[32 + c] = v.x;
+          x[33 + c] = v.y;
+          v = fadd2(f32x2{__uint_as_float(s2[c] + 0x4B400000u),
+                          __uint_as_float(s2[c + 1] + 0x4B400000u)}, magic);
+          x[64 + c] = v.x;
+          x[65 + c] = v.y;
+          v = fadd2(f32x2{__uint_as_float(s3[c] + 0x4B400000u),
+                          __uint_as_float(s3[c + 1] + 0x4B400000u)}, magic);
+          x[96 + c] = v.x;
+          x[97 + c] = v.y;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
           x[c] = __uint_as_float(s0[c]);
           x[32 + c] = __uint_as_float(s1[c]);
           x[64 + c] = __uint_as_float(s2[c]);
           x[96 + c] = __uint_as_float(s3[c]);
         }
       }
-      // (kept positive so that masked -inf scores stay -inf for an all-zero block)
-      if constexpr (QUANT)
-        cj = fmaxf(qsc * a.k_scale[(size_t)u * a.nblk_k + jt0 + j] * a.scale_log2, 1e-30f);
+      // raw score -> base-2 scaled score factor (quantised: kept positive so that
+      // masked -inf scores stay -inf for an all-zero block)
+      const float cj = QUANT ? fmaxf(qsc * ksc * a.scale_log2, 1e-30f) : a.scale_log2;
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
@@ -457,16 +551,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
           if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
         }
       }
-      // row max: eight independent chains, then a tree
-      float mx8[8];
+      // row max: four chains of three-input maxima
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = x[e];
+      for (int c = 0; c < 128; c += 8)
 #pragma unroll
-      for (int c = 8; c < 128; c += 8)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[c + e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
+      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
       const float m_tile = mx * cj;  // cj > 0; -inf stays -inf
       const float m_prev = m_used;
       const float m_new = fmaxf(m_prev, m_tile);
@@ -475,6 +566,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? ex2(m_prev - m_new) : 1.0f;
         l *= f;
+        lf *= f;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -485,43 +577,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
           tmem_st32(tO + c0, o);
         }
       }
-      // P = 2^(x * cj - m)  (quantised: times 2^8 before the E4M3 cast), written
-      // over S in 32-key chunks.  Exact mode: the row sum adds the 16-bit values
-      // that the P.V product actually uses, so O is a convex combination of V rows.
-      const float mb = (m_used == -INFINITY ? 0.0f : m_used) - (QUANT ? 8.0f : 0.0f);
-      float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if constexpr (QUANT) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              p[e] = ex2(fmaf(x[32 * ch + 4 * c + e], cj, -mb));
-              rs4[e] += p[e];
-            }
-            pk[c] = uint32_t(f32x2_to_e4m3x2(p[0], p[1])) |
-                    (uint32_t(f32x2_to_e4m3x2(p[2], p[3])) << 16);
-          }
-          tmem_st8(tS + 8 * ch, pk);
-        } else {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(x[32 * ch + 2 * c], cj, -mb));
-            const float p1 = ex2(fmaf(x[32 * ch + 2 * c + 1], cj, -mb));
-            pk[c] = pack_16x2<F16>(p0, p1);
-            float r0, r1;
-            unpack_16x2<F16>(pk[c], r0, r1);
-            rs4[(2 * c) & 3] += r0;
-            rs4[(2 * c + 1) & 3] += r1;
-          }
-          tmem_st16(tS + 16 * ch, pk);
-        }
-      }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      // P = 2^(x * cj - m)  (quantised: times 2^7 before the E4M3 cast), written
+      // over S in 32-key chunks.  Exact mode: the row sum l adds the 16-bit values
+      // that the P.V product actually uses, so O is a convex combination of V rows;
+      // lf adds the float32 values (for lse).  On tiles without masked keys a
+      // quarter of the exponentials run on the FMA pipe (poly_ex2).
+      const float mb = (m_used == -INFINITY ? 0.0f : m_used) - C::kPScale;
+      if (need_mask)
+        softmax_emit<F16, QUANT, false>(x, cj, mb, tS, l, lf);
+      else
+        softmax_emit<F16, QUANT, true>(x, cj, mb, tS, l, lf);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready(q));
@@ -539,7 +604,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
     }
     const bool have_o = ok && n > 0;
     const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
-    const float lse2 = (l > 0.0f) ? m_used + lg2(l) - (QUANT ? 8.0f : 0.0f) : -INFINITY;
+    // base-2 log-sum-exp: of the weights P.V used (merge weights) and of the
+    // float32 weights (the reported lse)
+    const float lse2_w = (l > 0.0f) ? m_used + lg2(l) - C::kPScale : -INFINITY;
+    const float lse2 = (lf > 0.0f) ? m_used + lg2(lf) - C::kPScale : -INFINITY;
     if constexpr (SPLIT) {
       const size_t prow = ((size_t)split * a.units + u) * a.R + r;
 #pragma unroll 1
@@ -572,7 +640,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
           }
         }
       }
-      if (rvalid) a.lse_part[prow] = lse2;
+      if (rvalid) {
+        a.lse_part[prow] = lse2_w;
+        a.lse_part[(size_t)a.splits * a.units * a.R + prow] = lse2;
+      }
     } else {
       const uint32_t stage = C::kStageInQ ? sbase + C::kQOff + q * C::kQTile
                                           : sbase + C::kStageOff + q * C::kOStage;

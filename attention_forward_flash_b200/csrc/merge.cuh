@@ -2,10 +2,12 @@
 // review": the merge caches each chunk's maximum and weight and computes the
 // denominator once).
 //
-// Each split s of a row left O_s (already divided by its own row sum) and
-// L_s = base-2 log-sum-exp of its scaled scores (-inf for an empty split).
-// With M = max_s L_s and w_s = 2^(L_s - M):
-//     O = sum_s w_s O_s / sum_s w_s,     lse = ln 2 * (M + log2 sum_s w_s).
+// Each split s of a row left O_s (already divided by its own row sum), W_s =
+// base-2 log of the sum of the weights its P.V product used, and L_s = base-2
+// log-sum-exp of its float32 weights (-inf for an empty split).  With
+// M = max_s W_s and w_s = 2^(W_s - M):
+//     O = sum_s w_s O_s / sum_s w_s,
+// and lse = ln 2 * (ML + log2 sum_s 2^(L_s - ML)) with ML = max_s L_s.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -83,14 +85,31 @@ __global__ void __launch_bounds__(256) splitkv_merge_kernel(const float* __restr
   } else {
     *reinterpret_cast<uint32_t*>(dst) = h[0] | (uint32_t(h[1]) << 16);
   }
-  if (lse != nullptr && lane == 0)
-    lse[row] = (wsum > 0.0f) ? (M + lg2(wsum)) * 0.69314718055994531f : -INFINITY;
+  if (lse != nullptr) {
+    const float* lf = lse_part + (size_t)splits * rows;
+    float ML = -INFINITY;
+    for (int s = lane; s < splits; s += 32) ML = fmaxf(ML, lf[(size_t)s * rows + row]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ML = fmaxf(ML, __shfl_xor_sync(0xffffffffu, ML, o));
+    float ls = 0.0f;
+    for (int s = lane; s < splits; s += 32)
+      ls += (ML == -INFINITY) ? 0.0f : ex2(lf[(size_t)s * rows + row] - ML);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) lse[row] = (ls > 0.0f) ? (ML + lg2(ls)) * 0.69314718055994531f : -INFINITY;
+  }
 }
 
 // O = 0 and lse = -inf for every row (a problem whose rows see no key at all).
 __global__ void fill_lse_kernel(float* lse, size_t rows) {
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   if (i < rows) lse[i] = -INFINITY;
+}
+
+// y = 2^x through poly_ex2 (test hook for the FMA-pipe exponential).
+__global__ void poly_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, size_t n) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i < n) y[i] = poly_ex2(x[i]);
 }
 
 }  // namespace attn

@@ -184,6 +184,20 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   return d;
 }
 
+// The same descriptor as two 32-bit words, so that per-MMA offsets are one add:
+// lo = start address >> 4 | (LBO >> 4) << 16,  hi = SBO >> 4 | version 1 | layout.
+__host__ __device__ constexpr uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo, uint32_t layout) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | ((layout & 7u) << 29);
+}
+__device__ __forceinline__ uint64_t desc_pack(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+
 // Instruction descriptor (dense).  c_fmt: 1 = f32, 2 = s32.  a/b_fmt: for
 // kind::f16 0 = f16, 1 = bf16; for kind::i8 1 = signed; for kind::f8f6f4
 // 0 = e4m3.  major: 0 = K-major, 1 = MN-major.
@@ -289,6 +303,54 @@ __device__ __forceinline__ float lg2(float x) {
   float y;
   asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe (keeps the MUFU free for the other exponentials).
+// Cody-Waite style range reduction x = n + f, n = round-to-nearest(x) through
+// the 1.5*2^23 addition, f in [-1/2, 1/2]; 2^f from a degree-3 polynomial
+// fitted to minimise the maximum relative error on that interval (fit in
+// float64, coefficients rounded to float32: max relative error 7.5e-5, about
+// 13.7 bits, enough for the 16-bit and 8-bit P it feeds); 2^n is added to the
+// exponent field.  Arguments are clamped to -125 (so the result stays a normal
+// float); callers only use this where no score is masked.
+__device__ __forceinline__ float poly_ex2(float x) {
+  x = fmaxf(x, -125.0f);
+  const float r = x + 12582912.0f;  // 1.5 * 2^23: rounds x to an integer in the low bits
+  const float f = x - (r - 12582912.0f);
+  float p = fmaf(0.05517113208770752f, f, 0.24261008203029633f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999281167984009f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed float32 pairs (Blackwell f32x2 FMA / add: two lanes per instruction).
+struct f32x2 {
+  float x, y;
+};
+__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+  uint64_t ra, rb, rc, rd;
+  f32x2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+__device__ __forceinline__ f32x2 fadd2(f32x2 a, f32x2 b) {
+  uint64_t ra, rb, rd;
+  f32x2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
 }
 
 // Two floats -> packed e4m3 pair, `lo` in the low byte (round to nearest even,

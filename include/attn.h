@@ -27,7 +27,8 @@
  *     it sees keys j <= start_pos + i.  Keys j < window_lo are never seen.
  *     A row that sees no key gets O = 0 and lse = -inf.
  *   - All tensor pointers are DEVICE pointers owned by the caller and must be
- *     16-byte aligned; the library never frees them.  `stream` is a
+ *     16-byte aligned; the library never frees them.  A buffer of zero length
+ *     (q_len or kv_len 0) may be NULL.  `stream` is a
  *     cudaStream_t passed as void*.  Every call is asynchronous on that stream;
  *     argument errors are reported synchronously, before anything is launched.
  *   - A context is not safe for concurrent use from several host threads.
@@ -146,6 +147,13 @@ int attn_num_splits(const attn_ctx *c);
  * records ATTN_ERR_TIMEOUT in the context and returns without hanging.  The
  * hook exists only to test that error path; 0 restores normal operation. */
 attn_status attn_debug_set(attn_ctx *c, unsigned flags);
+
+/* TEST HOOK.  y[i] = 2^x[i] (device pointers, n floats) computed by the
+ * polynomial exponential that the softmax runs on the FMA pipe for part of its
+ * exponentials (range reduction to [-1/2, 1/2] and a degree-3 fit of 2^f; max
+ * relative error 7.5e-5 for -125 <= x <= 126; inputs below -125 are treated as -125).
+ * Errors: ATTN_ERR_INVALID_ARG (NULL pointer with n > 0), ATTN_ERR_CUDA. */
+attn_status attn_debug_exp2(const float *x, float *y, size_t n, void *stream);
 
 #ifdef __cplusplus
 }

@@ -60,7 +60,7 @@ def check_exact(o, r, what=""):
     return e, m
 
 
-def check_lse(lse, ref, what="", tol=2e-3):
+def check_lse(lse, ref, what="", tol=1e-3):
     lse = np.asarray(lse, np.float64)
     ref = np.asarray(ref, np.float64)
     fin = np.isfinite(ref)
