@@ -113,6 +113,8 @@ def attention_f64(q, k, v, *, scale=None, causal=False, start_pos=0, window_lo=0
     for b in range(B):
         for hq in range(Hq):
             hk = hq // group
+            if Skv == 0:                                    # no key at all: every row is empty
+                continue
             s = scale * (q[b, hq, rows, :] @ k[b, hk].T)  # [R, Skv] scores
             s = np.where(vis, s, -np.inf)                  # masked keys
             m = np.max(s, axis=1)                           # row max (-inf if none)

@@ -236,3 +236,11 @@ def test_flop_count_reproduces_page_tops():
     assert attention_flops(4, 32, 8192, 8192, 128, causal=True) == f * 0 + 4 * 4 * 32 * 8192 * 8192 * 128 / 2
     assert visible_pairs(4, 4096, start_pos=4092, causal=True) == 4093 + 4094 + 4095 + 4096
     assert visible_pairs(3, 3, causal=True) == 6
+
+
+def test_no_keys_at_all():
+    # kv_len = 0: every row sees no key -> O = 0, lse = -inf (the empty-row reading)
+    q = np.ones((1, 2, 3, 4))
+    k = np.zeros((1, 1, 0, 4))
+    o, lse = attention_f64(q, k, k, causal=True)
+    assert o.shape == (1, 2, 3, 4) and np.all(o == 0) and np.all(lse == -math.inf)
