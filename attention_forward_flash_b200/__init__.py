@@ -19,6 +19,7 @@ from ._abi import (  # noqa: F401
     attn_debug_set,
     attn_destroy,
     attn_forward,
+    attn_forward_splitkv_noalloc,
     attn_get_error,
     attn_num_splits,
     attn_qbufs_sizes,

@@ -12,7 +12,7 @@ ATTN_EXACT, ATTN_INT8QK_FP8PV = 0, 1
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
-            "attn_debug_exp2")
+            "attn_debug_exp2", "attn_forward_splitkv_noalloc")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -74,6 +74,9 @@ def lib():
         L.attn_debug_set.restype = c_int
         L.attn_debug_exp2.argtypes = [vp, vp, ctypes.c_size_t, vp]
         L.attn_debug_exp2.restype = c_int
+        L.attn_forward_splitkv_noalloc.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp,
+                                                   vp, vp]
+        L.attn_forward_splitkv_noalloc.restype = c_int
         _LIB = L
     return _LIB
 
@@ -126,3 +129,8 @@ def attn_debug_set(ctx, flags):
 
 def attn_debug_exp2(x, y, n, stream):
     _check(lib().attn_debug_exp2(x, y, n, stream), "attn_debug_exp2")
+
+
+def attn_forward_splitkv_noalloc(params: AttnParams, q, k, v, o, lse, err, stream):
+    _check(lib().attn_forward_splitkv_noalloc(ctypes.byref(params), q, k, v, o, lse, err, stream),
+           "attn_forward_splitkv_noalloc")

@@ -428,3 +428,152 @@ attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of the split-KV forward (see attn_forward_splitkv_noalloc
+// in attn.h).  Its split partials live in this file-scope array instead of a
+// context workspace: every GPU that loads the library holds these bytes until
+// the process exits.  Layout: O partials | per-row statistics | error sink.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocPartFloats = size_t(1) << 20;  // 4 MiB of O partials
+constexpr size_t kNoAllocStatFloats = size_t(1) << 15;  // 128 KiB of row statistics
+constexpr size_t kNoAllocSinkFloats = 64;               // error word when the caller passes none
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartFloats +
+                                                         kNoAllocStatFloats +
+                                                         kNoAllocSinkFloats];
+
+namespace {
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  Host code must not
+// use the symbol itself (it is a host-side stand-in, not a device address).
+attn_status noalloc_scratch(int dev, float** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+}  // namespace
+
+extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const void* q,
+                                                    const void* k, const void* v, void* o,
+                                                    float* lse, unsigned* err, void* stream) {
+  attn_status st = validate(p);
+  if (st != ATTN_OK) return st;
+  if (p->precision != ATTN_EXACT) return ATTN_ERR_UNSUPPORTED;
+  const bool need_q = p->q_len > 0, need_kv = p->kv_len > 0;
+  auto bad = [](const void* ptr, bool needed) {
+    return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));
+  };
+  if (bad(q, need_q) || bad(o, need_q) || bad(k, need_kv) || bad(v, need_kv) ||
+      (lse && !aligned16(lse)) || (err && (reinterpret_cast<uintptr_t>(err) & 3u)))
+    return ATTN_ERR_INVALID_ARG;
+
+  int dev = 0, sms = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (major != 10) return ATTN_ERR_UNSUPPORTED;
+
+  // Same split choice as attn_create makes for the split-KV path.
+  attn_ctx c{};
+  c.p = *p;
+  c.device = dev;
+  c.num_sms = sms;
+  c.G = p->n_q_heads / p->n_kv_heads;
+  c.R = c.G * p->q_len;
+  c.units = p->batch * p->n_kv_heads;
+  c.scale = p->scale > 0.0f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
+  const int kv_tiles = ceil_div(p->kv_len, 128);
+  int splits = p->num_splits > 1
+                   ? p->num_splits
+                   : std::max(1, std::min(kv_tiles, ceil_div(sms, c.units * ceil_div(c.R, 128))));
+  splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
+  splits = std::min(splits, kMergeMaxSplits);
+  c.split_path = 1;
+  c.tiles_per_split = std::max(1, ceil_div(kv_tiles, splits));
+  c.splits = std::max(1, ceil_div(kv_tiles, c.tiles_per_split));
+  c.row_tiles = ceil_div(c.R, 128);
+
+  const size_t rows = static_cast<size_t>(c.units) * c.R;
+  if (rows == 0) return ATTN_OK;
+  const size_t part_floats = static_cast<size_t>(c.splits) * rows * p->head_dim;
+  const size_t stat_floats = 2 * static_cast<size_t>(c.splits) * rows;
+  if (part_floats > kNoAllocPartFloats || stat_floats > kNoAllocStatFloats)
+    return ATTN_ERR_UNSUPPORTED;  // larger than the static scratch: use attn_forward
+
+  float* scratch = nullptr;
+  st = noalloc_scratch(dev, &scratch);
+  if (st != ATTN_OK) return st;
+  c.o_part = scratch;
+  c.lse_part = scratch + kNoAllocPartFloats;
+  c.err = err ? err : reinterpret_cast<unsigned*>(scratch + kNoAllocPartFloats + kNoAllocStatFloats);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = p->head_dim;
+  const bool f16 = p->dtype == ATTN_FP16;
+  if (p->kv_len == 0) {  // every row sees no key
+    if (cudaMemsetAsync(o, 0, rows * D * 2, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (lse) fill_lse_kernel<<<ceil_div(rows, 256), 256, 0, s>>>(lse, rows);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+
+  const CUtensorMapDataType t16 =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t R = c.R, Sk = p->kv_len, U = c.units;
+  CUtensorMap tq, tk, tv, to;
+  bool ok = true;
+  ok &= make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return ATTN_ERR_CUDA;
+
+  FwdArgs a{};
+  a.R = c.R;
+  a.Sq = p->q_len;
+  a.Skv = p->kv_len;
+  a.G = c.G;
+  a.units = c.units;
+  a.row_tiles = c.row_tiles;
+  a.splits = c.splits;
+  a.tiles_per_split = c.tiles_per_split;
+  a.start_pos = p->start_pos;
+  a.causal = p->causal;
+  a.window_lo = p->window_lo;
+  a.scale_log2 = c.scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.o_part = c.o_part;
+  a.lse_part = c.lse_part;
+  a.nblk_q = ceil_div(p->q_len, 128);
+  a.nblk_k = kv_tiles;
+  a.err = c.err;
+  a.debug = 0;
+  const int grid = c.units * c.row_tiles * c.splits;
+  if (D == 128) {
+    st = f16 ? launch_fwd<128, 1, false, true, true>(&c, tq, tk, tv, to, a, grid, s)
+             : launch_fwd<128, 1, false, false, true>(&c, tq, tk, tv, to, a, grid, s);
+    if (st == ATTN_OK)
+      st = f16 ? launch_merge<128, true>(&c, o, lse, s) : launch_merge<128, false>(&c, o, lse, s);
+  } else {
+    st = f16 ? launch_fwd<64, 1, false, true, true>(&c, tq, tk, tv, to, a, grid, s)
+             : launch_fwd<64, 1, false, false, true>(&c, tq, tk, tv, to, a, grid, s);
+    if (st == ATTN_OK)
+      st = f16 ? launch_merge<64, true>(&c, o, lse, s) : launch_merge<64, false>(&c, o, lse, s);
+  }
+  return st;
+}

@@ -155,6 +155,38 @@ attn_status attn_debug_set(attn_ctx *c, unsigned flags);
  * Errors: ATTN_ERR_INVALID_ARG (NULL pointer with n > 0), ATTN_ERR_CUDA. */
 attn_status attn_debug_exp2(const float *x, float *y, size_t n, void *stream);
 
+/* Split-KV forward that allocates nothing (exact mode only).
+ * No counterpart on the source pages: it is a convenience for callers that
+ * cannot call cudaMalloc.  Examples are code whose device memory is owned by
+ * another allocator (a serving engine that reserves HBM up front and forbids
+ * stray allocations), and a latency-critical decode step that cannot afford
+ * cudaMalloc's implicit device synchronisation.  It takes the problem
+ * description directly (no context, so no attn_create) and computes the same
+ * result as attn_forward does on the split-KV path: key/value splits in one
+ * kernel, then the merge.  The split partials live in a fixed device array
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits: up to 2^20 floats (4 MiB) of partial outputs
+ * (splits x B x Hq x Sq x head_dim) and 2^15 floats (128 KiB) of per-row
+ * statistics (2 x splits x B x Hq x Sq).
+ *
+ * Arguments: as attn_forward, with `p` in place of a context; p->precision must
+ * be ATTN_EXACT; p->num_splits 0 (library's choice) or > 1 (forced).  `err` is
+ * an optional device word (4-byte aligned) into which a device-side wait that
+ * runs out ORs 1; pass NULL to ignore such errors.  The array is shared by
+ * every call: calls that overlap on the GPU (several streams, or several host
+ * threads) race on it and must be serialised by the caller.  Every value the
+ * kernels read from it is first written by the same call, so nothing needs
+ * clearing between calls.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture.
+ * Errors: ATTN_ERR_INVALID_ARG (bad field, NULL or misaligned pointer),
+ * ATTN_ERR_UNSUPPORTED (quantised mode, head_dim, or partials larger than the
+ * array; use attn_forward then), ATTN_ERR_CUDA (no sm_100 device, lookup,
+ * tensor-map encode or launch failure). */
+attn_status attn_forward_splitkv_noalloc(const attn_params *p, const void *q, const void *k,
+                                         const void *v, void *o, float *lse, unsigned *err,
+                                         void *stream);
+
 #ifdef __cplusplus
 }
 #endif
