@@ -100,11 +100,29 @@ attn_status dispatch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtenso
   return launch_fwd<D, 2, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
 }
 
+// The merge is a programmatic dependent launch of the split kernel: its launch
+// overlaps the split kernel's tail, and it waits on the grid dependency before
+// reading the partials.
 template <int D, bool F16>
 attn_status launch_merge(const attn_ctx* c, void* o, float* lse, cudaStream_t st) {
   const int rows = c->units * c->R;
-  splitkv_merge_kernel<D, F16><<<ceil_div(rows, 8), 256, 0, st>>>(
-      c->o_part, c->lse_part, static_cast<uint16_t*>(o), lse, rows, c->splits);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows);
+  cfg.blockDim = dim3(32 * kMergeWarps);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* op = c->o_part;
+  const float* lp = c->lse_part;
+  uint16_t* out = static_cast<uint16_t*>(o);
+  const int splits = c->splits;
+  if (cudaLaunchKernelEx(&cfg, splitkv_merge_kernel<D, F16>, op, lp, out, lse, rows, splits) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -194,7 +212,7 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
     if (c->R <= 128 || (big_ctas * 2 < sms && kv_tiles >= 4)) {
       split = true;
       const int base = c->units * ceil_div(c->R, 128);
-      splits = std::max(1, std::min(kv_tiles, ceil_div(sms, base)));
+      splits = std::max(1, std::min(kv_tiles, ceil_div(2 * sms, base)));  // two CTAs per SM
     }
   }
   splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
@@ -501,7 +519,8 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   const int kv_tiles = ceil_div(p->kv_len, 128);
   int splits = p->num_splits > 1
                    ? p->num_splits
-                   : std::max(1, std::min(kv_tiles, ceil_div(sms, c.units * ceil_div(c.R, 128))));
+                   : std::max(1, std::min(kv_tiles,
+                                          ceil_div(2 * sms, c.units * ceil_div(c.R, 128))));
   splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
   splits = std::min(splits, kMergeMaxSplits);
   c.split_path = 1;

@@ -78,7 +78,10 @@ struct FwdCfg {
   static constexpr int kFixed = NQT * kQTile + kStageBytes;
   static constexpr int kBudget = 200 * 1024;
   static constexpr int kNSraw = (kBudget - kFixed) / kSlot;
-  static constexpr int kNS = kNSraw > 8 ? 8 : kNSraw;
+  // The split-KV variant serves few-row (decode) problems whose CTAs each see a
+  // short key range: two K/V slots suffice, so that two CTAs share an SM.
+  static constexpr int kNS = SPLIT ? 2 : (kNSraw > 8 ? 8 : kNSraw);
+  static constexpr int kCtasPerSm = SPLIT ? 2 : 1;
   static_assert(kNS >= 2, "ring too small");
   static constexpr int kQOff = 0;
   static constexpr int kStageOff = NQT * kQTile;
@@ -101,8 +104,12 @@ struct FwdCfg {
   // within the largest finite E4M3 value (448).
   static constexpr float kRescaleThresh = QUANT ? 1.8f : 8.0f;
   static constexpr float kPScale = QUANT ? 7.0f : 0.0f;
-  static constexpr int kRegsLow = 64;    // loader / MMA warpgroup (two-tile variant)
-  static constexpr int kRegsHigh = 216;  // softmax warpgroups (two-tile variant)
+  // Registers per thread at launch (65536 / (threads * CTAs per SM), rounded
+  // down to a multiple of 8) and their split between warpgroups: the
+  // loader/MMA warpgroup needs few, the softmax warpgroups many.
+  static constexpr int kRegsLaunch = (65536 / (kThreads * kCtasPerSm)) / 8 * 8;
+  static constexpr int kRegsLow = NQT == 2 ? 64 : 56;
+  static constexpr int kRegsHigh = NQT == 2 ? 216 : 200;
 };
 
 template <bool F16>
@@ -198,7 +205,8 @@ __device__ __forceinline__ void softmax_emit(const float (&x)[128], float cj, fl
 }
 
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT>
-__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
+                                  FwdCfg<D, NQT, QUANT, SPLIT>::kCtasPerSm)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -287,12 +295,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // Split variant: the merge kernel may be scheduled now; it waits for this
+  // grid's completion (and memory flush) before reading the partials.
+  if constexpr (SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // Two-tile variant: 384 threads launched at 168 registers each (64512).  The
   // loader/MMA warpgroup needs few, the softmax warpgroups many:
   // 128 x 56 + 256 x 224 = 64512, exactly the launch budget.
-  static_assert(NQT != 2 || 128 * C::kRegsLow + 256 * C::kRegsHigh <= C::kThreads * 168,
-                "register split");
+  static_assert(128 * C::kRegsLow + (C::kThreads - 128) * C::kRegsHigh <=
+                    C::kThreads * C::kRegsLaunch,
+                "register split exceeds the launch allocation");
 
   auto raise = [&]() {
     *abort_flag = 1;
@@ -300,7 +312,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
   };
 
   if (warp < 4) {
-  if constexpr (NQT == 2) regs_dec<C::kRegsLow>();
+  regs_dec<C::kRegsLow>();
   if (warp == 0) {
     // ======================================================== TMA producer
     if (lane == 0) {
@@ -465,7 +477,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads, 1)
     }
   }
   } else {
-    if constexpr (NQT == 2) regs_inc<C::kRegsHigh>();
+    regs_inc<C::kRegsHigh>();
     // ============================================================ softmax
     const int q = (warp - 4) >> 2;            // query tile of this warpgroup
     const int wq = warp & 3;                  // TMEM lane quarter
