@@ -325,7 +325,7 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
                                                                p.kv_len, nbk);                 \
       v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(           \
           X(v), c->v_amax, p.kv_len);                                                          \
-      v_quant_kernel<DD, FF><<<dim3(nbk, BHk), 256, 0, st>>>(X(v), c->v_amax, qb->v_t,         \
+      v_quant_kernel<DD, FF><<<dim3(nbk, BHk), 2 * DD, 0, st>>>(X(v), c->v_amax, qb->v_t,      \
                                                               qb->v_scale, p.kv_len, S_pad);   \
     }                                                                                          \
   } while (0)

@@ -37,6 +37,26 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
   }
 }
 
+// x / s correctly rounded (the float32 division) from the block's reciprocal:
+// y = RN(x * r) with r = RN(1/s) is within an ulp of x / s, the residual
+// x - y * s is exact under one fused multiply-add, and RN(y + residual * r) is
+// the correctly rounded quotient (Markstein's theorem on division through a
+// correctly rounded reciprocal; Markstein, IBM J. Res. Dev. 34(1), 1990).
+// Valid while s, 1/s and the quotient stay normal, which the callers check
+// block-wide (else they use the plain division).
+// The sign is copied from x (s > 0): the correction step would turn -0 into +0.
+__device__ __forceinline__ float div_by_recip(float x, float s, float r) {
+  const float y = x * r;
+  const float e = fmaf(-y, s, x);
+  return copysignf(fmaf(e, r, y), x);
+}
+
+// True when div_by_recip(x, s, r) is exact for every |x| <= 127.5 * s (and for
+// x = 0): s and 1/s comfortably inside the normal range.
+__device__ __forceinline__ bool recip_ok(float s) {
+  return s >= 1.0e-30f && s <= 1.0e30f;
+}
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -85,6 +105,8 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const uint16_t* __restric
 
   const float s = __fdiv_rn(amax, 127.0f);
   if (threadIdx.x == 0) scales[bh * nblk + t] = s;
+  const float r = __frcp_rn(s);
+  const bool fast = recip_ok(s);
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
     const int c = threadIdx.x + k * 256;
@@ -95,7 +117,10 @@ __global__ void __launch_bounds__(256) quant_qk_kernel(const uint16_t* __restric
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         int qv = 0;
-        if (s > 0.0f) qv = max(-127, min(127, __float2int_rn(__fdiv_rn(f[e], s))));
+        if (s > 0.0f) {
+          const float qf = fast ? div_by_recip(f[e], s, r) : __fdiv_rn(f[e], s);
+          qv = max(-127, min(127, __float2int_rn(qf)));
+        }
         packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
       }
       *reinterpret_cast<uint2*>(codes + base + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
@@ -134,49 +159,52 @@ __global__ void __launch_bounds__(256) v_amax_kernel(const uint16_t* __restrict_
   for (int c = threadIdx.x; c < D; c += 256) atomicMax(&amax_bits[u * D + c], smax[c]);
 }
 
-// grid: (S_pad/128, B*Hkv), 256 threads.  Quantise a 128-token tile of V and
-// write it transposed.
+// grid: (S_pad/128, B*Hkv), 2*D threads.  Quantise a 128-token tile of V and
+// write it transposed.  Thread (channel c, token half h) converts tokens
+// [64h, 64h + 64) of channel c: every load instruction of a warp reads 32
+// neighbouring channels of one token (64 contiguous bytes) and every store
+// writes 16 consecutive codes of one channel row.
 template <int D, bool F16>
-__global__ void __launch_bounds__(256) v_quant_kernel(const uint16_t* __restrict__ v,
-                                                      const unsigned* __restrict__ amax_bits,
-                                                      uint8_t* __restrict__ vt,
-                                                      float* __restrict__ v_scale, int S,
-                                                      int S_pad) {
-  constexpr int kCC = D / 8;
-  constexpr int kPitch = 128 + 16;  // bytes per transposed row in shared memory
-  __shared__ float sc[D];
-  __shared__ __align__(16) uint8_t tile[D * kPitch];
+__global__ void __launch_bounds__(2 * D) v_quant_kernel(const uint16_t* __restrict__ v,
+                                                        const unsigned* __restrict__ amax_bits,
+                                                        uint8_t* __restrict__ vt,
+                                                        float* __restrict__ v_scale, int S,
+                                                        int S_pad) {
   const size_t u = blockIdx.y;
   const int tok0 = blockIdx.x * 128;
-  for (int c = threadIdx.x; c < D; c += 256) {
-    const float s = __fdiv_rn(__uint_as_float(amax_bits[u * D + c]), 448.0f);
-    sc[c] = s;
-    if (blockIdx.x == 0) v_scale[u * D + c] = s;
-  }
-  __syncthreads();
-  for (int ch = threadIdx.x; ch < 128 * kCC; ch += 256) {
-    const int tk = ch / kCC;
-    const int cc = ch % kCC;
-    const int tok = tok0 + tk;
-    float f[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (tok < S) unpack8<F16>(ld_nc_v4(v + ((u * S + tok) * D + cc * 8)), f);
+  const int c = threadIdx.x % D;
+  const int half = threadIdx.x / D;
+  const float s = __fdiv_rn(__uint_as_float(amax_bits[u * D + c]), 448.0f);
+  if (blockIdx.x == 0 && half == 0) v_scale[u * D + c] = s;
+  const float r = __frcp_rn(s);
+  const bool fast = recip_ok(s);
+  const uint16_t* src = v + (u * S) * D + c;
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const int c0 = cc * 8 + e;
-      const float s0 = sc[c0], s1 = sc[c0 + 1];
-      const float a0 = (tok < S && s0 > 0.0f) ? __fdiv_rn(f[e], s0) : 0.0f;
-      const float a1 = (tok < S && s1 > 0.0f) ? __fdiv_rn(f[e + 1], s1) : 0.0f;
-      const uint16_t p = f32x2_to_e4m3x2(a0, a1);
-      tile[c0 * kPitch + tk] = static_cast<uint8_t>(p & 0xFF);
-      tile[(c0 + 1) * kPitch + tk] = static_cast<uint8_t>(p >> 8);
+  for (int g = 0; g < 4; ++g) {                 // 4 groups of 16 tokens
+    const int t0 = tok0 + half * 64 + g * 16;
+    uint16_t raw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) raw[i] = (t0 + i < S) ? __ldg(src + (size_t)(t0 + i) * D) : 0;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      float f0, f1;
+      if constexpr (F16) {
+        f0 = __half2float(__ushort_as_half(raw[i]));
+        f1 = __half2float(__ushort_as_half(raw[i + 1]));
+      } else {
+        f0 = __bfloat162float(__ushort_as_bfloat16(raw[i]));
+        f1 = __bfloat162float(__ushort_as_bfloat16(raw[i + 1]));
+      }
+      float a0 = 0.0f, a1 = 0.0f;
+      if (s > 0.0f) {
+        a0 = (t0 + i < S) ? (fast ? div_by_recip(f0, s, r) : __fdiv_rn(f0, s)) : 0.0f;
+        a1 = (t0 + i + 1 < S) ? (fast ? div_by_recip(f1, s, r) : __fdiv_rn(f1, s)) : 0.0f;
+      }
+      w[i / 4] |= uint32_t(f32x2_to_e4m3x2(a0, a1)) << (16 * ((i / 2) & 1));
     }
-  }
-  __syncthreads();
-  for (int ch = threadIdx.x; ch < D * 8; ch += 256) {
-    const int c = ch / 8;
-    const int part = ch % 8;
-    const uint4 w = *reinterpret_cast<const uint4*>(tile + c * kPitch + part * 16);
-    *reinterpret_cast<uint4*>(vt + (u * D + c) * (size_t)S_pad + tok0 + part * 16) = w;
+    *reinterpret_cast<uint4*>(vt + (u * D + c) * (size_t)S_pad + t0) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 

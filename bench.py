@@ -90,9 +90,11 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the sources that define the fused attention kernel (the one whose
+    DRAM traffic profiles/traffic.txt records)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_forward_flash_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in ("flash_fwd.cuh", "ptx.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
