@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     }
     for (int q = 0; q < NQT; ++q) {
       mbar_init(s_ready(q), 1);
-      mbar_init(p_ready(q), 128);
+      mbar_init(p_ready(q), 4);  // one arrive per softmax warp
     }
     mbar_init(o_final, 1);
     *abort_flag = 0;
@@ -502,9 +502,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     float l = 0.0f;            // row sum of the P values P.V uses (relative to m_used)
     float lf = 0.0f;           // row sum of the float32 P values (for lse)
     bool ok = true;
+    // Quantised: the K block scale of tile j is loaded one tile ahead (a pinned
+    // load, so that its latency hides behind the previous tile's softmax).
+    const float* ksrc = QUANT ? a.k_scale + (size_t)u * a.nblk_k + jt0 : nullptr;
+    float ksc_next = 1.0f;
+    if constexpr (QUANT)
+      if (n > 0) ksc_next = ld_global_f32(ksrc);
     for (int j = 0; j < n; ++j) {
-      float ksc = 1.0f;
-      if constexpr (QUANT) ksc = a.k_scale[(size_t)u * a.nblk_k + jt0 + j];
+      const float ksc = ksc_next;
+      if constexpr (QUANT)
+        if (j + 1 < n) ksc_next = ld_global_f32(ksrc + j + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(s_ready(q), j & 1, abort_flag));
       if (!ok) { if (lane == 0) raise(); break; }
       tc_fence_after();
@@ -601,7 +608,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         softmax_emit<F16, QUANT, true>(x, cj, mb, tS, l, lf);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_ready(q));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready(q));
     }
 
     // ----------------------------------------------------------- epilogue
