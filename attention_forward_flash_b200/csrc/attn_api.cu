@@ -80,12 +80,12 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT>
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF = SPLIT>
 attn_status launch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                        cudaStream_t st) {
   using Cfg = FwdCfg<D, NQT, QUANT, SPLIT>;
-  auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT>;
+  auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF>;
   static bool attr_ok = set_smem(kern, Cfg::kSmemBytes);
   if (!attr_ok) return ATTN_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
@@ -97,6 +97,9 @@ attn_status dispatch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtenso
                          const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                          cudaStream_t st) {
   if (c->split_path) return launch_fwd<D, 1, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
+  // Exact mode keeps a second (float32) row sum only when the caller asks for lse.
+  if (!QUANT && a.lse != nullptr)
+    return launch_fwd<D, 2, QUANT, F16, false, true>(c, tq, tk, tv, to, a, grid, st);
   return launch_fwd<D, 2, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
 }
 

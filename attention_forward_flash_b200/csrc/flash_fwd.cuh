@@ -87,8 +87,9 @@ struct FwdCfg {
   static constexpr int kStageOff = NQT * kQTile;
   static constexpr int kRingOff = kFixed;
   static constexpr int kBarOff = kRingOff + kNS * kSlot;
-  // barriers: q_full, full[NS], empty[NS], s_ready[NQT], p_ready[NQT], o_final
-  static constexpr int kNumBars = 1 + 2 * kNS + 2 * NQT + 1;
+  // barriers: q_full, full[NS], empty[NS], s_ready[NQT], p_ready[NQT][2] (one per
+  // 64-key half of P), o_final
+  static constexpr int kNumBars = 1 + 2 * kNS + 3 * NQT + 1;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;      // tmem base, abort flag
   static constexpr int kSvOff = kMiscOff + 16;                  // v scales (quant)
   static constexpr int kSmemBytes = kSvOff + (QUANT ? D * 4 : 0) + 1024;  // + alignment slack
@@ -108,7 +109,7 @@ struct FwdCfg {
   // down to a multiple of 8) and their split between warpgroups: the
   // loader/MMA warpgroup needs few, the softmax warpgroups many.
   static constexpr int kRegsLaunch = (65536 / (kThreads * kCtasPerSm)) / 8 * 8;
-  static constexpr int kRegsLow = NQT == 2 ? 64 : 56;
+  static constexpr int kRegsLow = NQT == 2 ? 72 : 56;
   static constexpr int kRegsHigh = NQT == 2 ? 216 : 200;
 };
 
@@ -135,35 +136,54 @@ __device__ __forceinline__ void unpack_16x2(uint32_t v, float& lo, float& hi) {
   }
 }
 
-// P = 2^(x * cj - mb) for one 128-key row chunk: written over S in tensor memory
-// (16-bit pairs, or E4M3 quads in the quantised mode) and added to the row sums.
-// POLY: every fourth exponential runs on the FMA pipe instead of the MUFU.
-template <bool F16, bool QUANT, bool POLY>
-__device__ __forceinline__ void softmax_emit(const float (&x)[128], float cj, float mb,
-                                             uint32_t tS, float& l, float& lf) {
-  const f32x2 cc{cj, cj}, mm{-mb, -mb};
-  f32x2 fs0{0.0f, 0.0f}, fs1{0.0f, 0.0f}, rs0{0.0f, 0.0f}, rs1{0.0f, 0.0f};
+// Share of the exponentials that run on the FMA pipe (poly_ex2x2) instead of the
+// MUFU, on key tiles without masked scores: one pair in this many (0: none).
+#ifndef ATTN_POLY_EVERY
+#define ATTN_POLY_EVERY 0
+#endif
+#ifndef ATTN_POLY_EVERY_Q
+#define ATTN_POLY_EVERY_Q 0
+#endif
+
+// Per-tile row-sum accumulators of one softmax thread: r[] adds the 16-bit P
+// values that P.V multiplies (exact mode), f0/f1 the float32 P values.
+struct RowSums {
+  float r[4];
+  f32x2 f0, f1;
+};
+
+// P = 2^(x * c - m) for one half (64 keys) of a 128-key row, written over S in
+// tensor memory as 16-bit pairs (exact) or E4M3 quads (quantised), and added to
+// the row sums.  `cm` = {c, c}, `mm` = {-m, -m}; in the quantised mode x holds
+// the integer scores offset by 1.5 * 2^23 (their float bit pattern), and mm
+// already subtracts that offset times c.  POLY: one pair in POLY takes the FMA
+// pipe exponential (0: all on the MUFU).  LF: keep the float32 sum (exact mode;
+// the quantised mode always keeps it, it is its only sum).
+template <bool F16, bool QUANT, int POLY, bool LF, int H>
+__device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 cm, f32x2 mm,
+                                                  uint32_t tS, RowSums& rs) {
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
+  for (int ch = 2 * H; ch < 2 * H + 2; ++ch) {
     if constexpr (QUANT) {
       uint32_t pk[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int e = 32 * ch + 4 * c;
-        const f32x2 t0 = ffma2(f32x2{x[e], x[e + 1]}, cc, mm);
-        const f32x2 t1 = ffma2(f32x2{x[e + 2], x[e + 3]}, cc, mm);
-        float p0, p1;
-        if (POLY && (c % 2 == 0)) {
-          p0 = poly_ex2(t0.x);
-          p1 = poly_ex2(t0.y);
+        const f32x2 t0 = ffma2(f32x2{x[e], x[e + 1]}, cm, mm);
+        const f32x2 t1 = ffma2(f32x2{x[e + 2], x[e + 3]}, cm, mm);
+        f32x2 p01, p23;
+        if (POLY > 0 && ((2 * c) % (POLY > 0 ? POLY : 1)) == 0) {
+          p01 = poly_ex2x2(t0);
         } else {
-          p0 = ex2(t0.x);
-          p1 = ex2(t0.y);
+          p01.x = ex2(t0.x);
+          p01.y = ex2(t0.y);
         }
-        const float p2 = ex2(t1.x), p3 = ex2(t1.y);
-        pk[c] = uint32_t(f32x2_to_e4m3x2(p0, p1)) | (uint32_t(f32x2_to_e4m3x2(p2, p3)) << 16);
-        fs0 = fadd2(fs0, f32x2{p0, p1});
-        fs1 = fadd2(fs1, f32x2{p2, p3});
+        p23.x = ex2(t1.x);
+        p23.y = ex2(t1.y);
+        pk[c] = uint32_t(f32x2_to_e4m3x2(p01.x, p01.y)) |
+                (uint32_t(f32x2_to_e4m3x2(p23.x, p23.y)) << 16);
+        rs.f0 = fadd2(rs.f0, p01);
+        rs.f1 = fadd2(rs.f1, p23);
       }
       tmem_st8(tS + 8 * ch, pk);
     } else {
@@ -171,40 +191,34 @@ __device__ __forceinline__ void softmax_emit(const float (&x)[128], float cj, fl
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const int e = 32 * ch + 2 * c;
-        const f32x2 t = ffma2(f32x2{x[e], x[e + 1]}, cc, mm);
-        float p0, p1;
-        if (POLY && (c % 4 == 0)) {
-          p0 = poly_ex2(t.x);
-          p1 = poly_ex2(t.y);
+        const f32x2 t = ffma2(f32x2{x[e], x[e + 1]}, cm, mm);
+        f32x2 p;
+        if (POLY > 0 && (c % (POLY > 0 ? POLY : 1)) == 0) {
+          p = poly_ex2x2(t);
         } else {
-          p0 = ex2(t.x);
-          p1 = ex2(t.y);
+          p.x = ex2(t.x);
+          p.y = ex2(t.y);
         }
-        pk[c] = pack_16x2<F16>(p0, p1);
-        float r0, r1;
-        unpack_16x2<F16>(pk[c], r0, r1);
-        if (c & 1) {
-          rs1 = fadd2(rs1, f32x2{r0, r1});
-          fs1 = fadd2(fs1, f32x2{p0, p1});
-        } else {
-          rs0 = fadd2(rs0, f32x2{r0, r1});
-          fs0 = fadd2(fs0, f32x2{p0, p1});
+        pk[c] = pack_16x2<F16>(p.x, p.y);
+        if (c & 1)
+          add_16x2<F16>(pk[c], rs.r[2], rs.r[3]);
+        else
+          add_16x2<F16>(pk[c], rs.r[0], rs.r[1]);
+        if constexpr (LF) {
+          if (c & 1)
+            rs.f1 = fadd2(rs.f1, p);
+          else
+            rs.f0 = fadd2(rs.f0, p);
         }
       }
       tmem_st16(tS + 16 * ch, pk);
     }
   }
-  const float fsum = (fs0.x + fs0.y) + (fs1.x + fs1.y);
-  if constexpr (QUANT) {
-    l += fsum;
-    lf += fsum;
-  } else {
-    l += (rs0.x + rs0.y) + (rs1.x + rs1.y);
-    lf += fsum;
-  }
 }
 
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT>
+// LF: the kernel also keeps the float32 row sum for the log-sum-exp (exact mode;
+// needed by the split variant and when the caller asks for lse).
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF>
 __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
                                   FwdCfg<D, NQT, QUANT, SPLIT>::kCtasPerSm)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -212,6 +226,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
   using C = FwdCfg<D, NQT, QUANT, SPLIT>;
+  static_assert(!SPLIT || LF, "the split variant always needs the float32 row sum");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -263,8 +278,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
   auto full_bar = [&](int s) { return bar(1 + s); };
   auto empty_bar = [&](int s) { return bar(1 + C::kNS + s); };
   auto s_ready = [&](int q) { return bar(1 + 2 * C::kNS + q); };
-  auto p_ready = [&](int q) { return bar(1 + 2 * C::kNS + NQT + q); };
-  const uint32_t o_final = bar(1 + 2 * C::kNS + 2 * NQT);
+  auto p_ready = [&](int q, int h) { return bar(1 + 2 * C::kNS + NQT + 2 * q + h); };
+  const uint32_t o_final = bar(1 + 2 * C::kNS + 3 * NQT);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   float* sv_smem = reinterpret_cast<float*>(smem + C::kSvOff);
@@ -277,7 +292,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     }
     for (int q = 0; q < NQT; ++q) {
       mbar_init(s_ready(q), 1);
-      mbar_init(p_ready(q), 4);  // one arrive per softmax warp
+      mbar_init(p_ready(q, 0), 4);  // one arrive per softmax warp
+      mbar_init(p_ready(q, 1), 4);
     }
     mbar_init(o_final, 1);
     *abort_flag = 0;
@@ -412,18 +428,23 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
           }
         }
       };
-      auto issue_pv = [&](int q, uint32_t v_lo, uint32_t accum) {
+      // O += P V over one 64-key half h of the tile (P columns of that half).
+      auto issue_pv = [&](int q, int h, uint32_t v_lo, uint32_t accum) {
         const uint32_t d = tmem + NQT * 128 + q * D;
         const uint32_t p = tmem + q * 128;
         if constexpr (QUANT) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 32 keys (8 columns of 4 e4m3) per step
+          for (int k2 = 0; k2 < 2; ++k2) {  // 32 keys (8 columns of 4 e4m3) per step
+            const int kk = 2 * h + k2;
             mma_f8_ts(d, p + kk * 8, desc_pack(v_lo + kk * 2, hi_v), idesc_pv, (accum | kk) != 0);
+          }
         } else {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)   // 16 keys (8 columns of 2 x 16-bit) per step
+          for (int k2 = 0; k2 < 4; ++k2) {  // 16 keys (8 columns of 2 x 16-bit) per step
+            const int kk = 4 * h + k2;
             mma_f16_ts(d, p + kk * 8, desc_pack(v_lo + kk * 128, hi_v), idesc_pv,
                        (accum | kk) != 0);
+          }
         }
       };
 
@@ -458,9 +479,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         const uint32_t v_lo = ring_lo_v + sv * (C::kSlot >> 4);
         const uint32_t k_lo = ring_lo + sk * (C::kSlot >> 4);
         for (int q = 0; q < NQT && ok; ++q) {
-          if (!mbar_wait(p_ready(q), j & 1, abort_flag)) { raise(); ok = false; break; }
-          tc_fence_after();
-          issue_pv(q, v_lo, j > 0);
+          // The first half of P.V runs while the softmax still writes the second.
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(p_ready(q, h), j & 1, abort_flag)) { raise(); ok = false; break; }
+            tc_fence_after();
+            issue_pv(q, h, v_lo, j > 0);
+          }
+          if (!ok) break;
           if (q == NQT - 1) tc_commit(empty_bar(sv));
           if (has_next) {
             issue_qk(q, k_lo);
@@ -508,6 +533,25 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     float ksc_next = 1.0f;
     if constexpr (QUANT)
       if (n > 0) ksc_next = ld_global_f32(ksrc);
+    constexpr int kPoly = QUANT ? ATTN_POLY_EVERY_Q : ATTN_POLY_EVERY;
+    // Quantised scores arrive as int32 s; adding 0x4B400000 to the bits gives the
+    // float F = 1.5 * 2^23 + s exactly (|s| < 2^22).  The offset is removed in the
+    // maximum and folded into the exponent's FMA: 2^(F * c - K) with
+    // K = 1.5 * 2^23 * c + m.  K is exact (so the FMA rounds s * c - m once, as a
+    // plain conversion would) because c is trimmed to 21 significant bits (the
+    // product with 3 * 2^22 then has at most 23) and the running max m is kept on
+    // integers in this mode.
+    constexpr float kMagic = QUANT ? 12582912.0f : 0.0f;
+    auto to_score = [](uint32_t v) {
+      return QUANT ? __uint_as_float(v + 0x4B400000u) : __uint_as_float(v);
+    };
+    // Hands one 64-key half of P to the MMA warp.
+    auto p_half_done = [&](int h) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready(q, h));
+    };
     for (int j = 0; j < n; ++j) {
       const float ksc = ksc_next;
       if constexpr (QUANT)
@@ -518,72 +562,67 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       const int kv0 = (jt0 + j) * 128;
       const bool need_mask =
           (kv0 < a.window_lo) || (kv0 + 128 > a.Skv) || (a.causal && kv0 + 127 > pos_min);
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tS + 0, s0);
-      tmem_ld32(tS + 32, s1);
-      tmem_ld32(tS + 64, s2);
-      tmem_ld32(tS + 96, s3);
-      tmem_ld_wait(s0);
-      tmem_ld_wait(s1);
-      tmem_ld_wait(s2);
-      tmem_ld_wait(s3);
+      // S is read in two 64-column halves: the second half's load overlaps the
+      // masking and maximum of the first.  Row max: four chains of three-input maxima.
       float x[128];
-      if constexpr (QUANT) {
-        // s32 -> f32 exactly: the integer plus 1.5*2^23 is a float whose low
-        // mantissa bits hold it; subtract 1.5*2^23 again (packed, two per op).
-        const f32x2 magic{-12582912.0f, -12582912.0f};
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          f32x2 v = fadd2(f32x2{__uint_as_float(s0[c] + 0x4B400000u),
-                                __uint_as_float(s0[c + 1] + 0x4B400000u)}, magic);
-          x[c] = v.x;
-          x[c + 1] = v.y;
-          v = fadd2(f32x2{__uint_as_float(s1[c] + 0x4B400000u),
-                          __uint_as_float(s1[c + 1] + 0x4B400000u)}, magic);
-          x[32 + c] = v.x;
-          x[33 + c] = v.y;
-          v = fadd2(f32x2{__uint_as_float(s2[c] + 0x4B400000u),
-                          __uint_as_float(s2[c + 1] + 0x4B400000u)}, magic);
-          x[64 + c] = v.x;
-          x[65 + c] = v.y;
-          v = fadd2(f32x2{__uint_as_float(s3[c] + 0x4B400000u),
-                          __uint_as_float(s3[c + 1] + 0x4B400000u)}, magic);
-          x[96 + c] = v.x;
-          x[97 + c] = v.y;
-        }
-      } else {
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(tS + 0, s0);
+        tmem_ld32(tS + 32, s1);
+        tmem_ld_wait(s0);
+        tmem_ld_wait(s1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(s0[c]);
-          x[32 + c] = __uint_as_float(s1[c]);
-          x[64 + c] = __uint_as_float(s2[c]);
-          x[96 + c] = __uint_as_float(s3[c]);
+          x[c] = to_score(s0[c]);
+          x[32 + c] = to_score(s1[c]);
         }
       }
-      // raw score -> base-2 scaled score factor (quantised: kept positive so that
-      // masked -inf scores stay -inf for an all-zero block)
-      const float cj = QUANT ? fmaxf(qsc * ksc * a.scale_log2, 1e-30f) : a.scale_log2;
+      uint32_t s2[32], s3[32];
+      tmem_ld32(tS + 64, s2);
+      tmem_ld32(tS + 96, s3);
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
+        for (int c = 0; c < 64; ++c) {
           const int kj = kv0 + c;
           if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
         }
       }
-      // row max: four chains of three-input maxima
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < 128; c += 8)
+      for (int c = 0; c < 64; c += 8)
 #pragma unroll
         for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
-      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+      tmem_ld_wait(s2);
+      tmem_ld_wait(s3);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[64 + c] = to_score(s2[c]);
+        x[96 + c] = to_score(s3[c]);
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int c = 64; c < 128; ++c) {
+          const int kj = kv0 + c;
+          if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int c = 64; c < 128; c += 8)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
+      // raw score -> base-2 scaled score factor (quantised: kept positive so that
+      // masked -inf scores stay -inf for an all-zero block)
+      const float cj =
+          QUANT ? __uint_as_float(__float_as_uint(fmaxf(qsc * ksc * a.scale_log2, 1e-30f)) & ~7u)
+                : a.scale_log2;
+      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) - kMagic;  // exact
       const float m_tile = mx * cj;  // cj > 0; -inf stays -inf
       const float m_prev = m_used;
       const float m_new = fmaxf(m_prev, m_tile);
       const bool need = (m_prev != -INFINITY) && (m_new > m_prev + C::kRescaleThresh);
-      if (m_prev == -INFINITY || need) m_used = m_new;
+      if (m_prev == -INFINITY || need) m_used = QUANT ? ceilf(m_new) : m_new;
       if (__any_sync(0xffffffffu, need)) {
-        const float f = need ? ex2(m_prev - m_new) : 1.0f;
+        const float f = need ? ex2(m_prev - m_used) : 1.0f;
         l *= f;
         lf *= f;
 #pragma unroll 1
@@ -597,19 +636,33 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         }
       }
       // P = 2^(x * cj - m)  (quantised: times 2^7 before the E4M3 cast), written
-      // over S in 32-key chunks.  Exact mode: the row sum l adds the 16-bit values
+      // over S in two 64-key halves; the MMA warp starts on the first half while
+      // the second is computed.  Exact mode: the row sum l adds the 16-bit values
       // that the P.V product actually uses, so O is a convex combination of V rows;
-      // lf adds the float32 values (for lse).  On tiles without masked keys a
-      // quarter of the exponentials run on the FMA pipe (poly_ex2).
+      // lf adds the float32 values (for lse).  On tiles without masked keys a share
+      // of the exponentials run on the FMA pipe (poly_ex2x2).
       const float mb = (m_used == -INFINITY ? 0.0f : m_used) - C::kPScale;
-      if (need_mask)
-        softmax_emit<F16, QUANT, false>(x, cj, mb, tS, l, lf);
-      else
-        softmax_emit<F16, QUANT, true>(x, cj, mb, tS, l, lf);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready(q));
+      const float kq = QUANT ? fmaf(kMagic, cj, mb) : mb;  // quantised: offset folded in
+      const f32x2 cm{cj, cj}, mm{-kq, -kq};
+      RowSums rs{{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f}, {0.0f, 0.0f}};
+      if (need_mask) {
+        softmax_emit_half<F16, QUANT, 0, LF, 0>(x, cm, mm, tS, rs);
+        p_half_done(0);
+        softmax_emit_half<F16, QUANT, 0, LF, 1>(x, cm, mm, tS, rs);
+      } else {
+        softmax_emit_half<F16, QUANT, kPoly, LF, 0>(x, cm, mm, tS, rs);
+        p_half_done(0);
+        softmax_emit_half<F16, QUANT, kPoly, LF, 1>(x, cm, mm, tS, rs);
+      }
+      p_half_done(1);
+      const float fsum = (rs.f0.x + rs.f0.y) + (rs.f1.x + rs.f1.y);
+      if constexpr (QUANT) {
+        l += fsum;
+        lf += fsum;
+      } else {
+        l += (rs.r[0] + rs.r[1]) + (rs.r[2] + rs.r[3]);
+        if constexpr (LF) lf += fsum;
+      }
     }
 
     // ----------------------------------------------------------- epilogue

@@ -312,24 +312,6 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe (keeps the MUFU free for the other exponentials).
-// Cody-Waite style range reduction x = n + f, n = round-to-nearest(x) through
-// the 1.5*2^23 addition, f in [-1/2, 1/2]; 2^f from a degree-3 polynomial
-// fitted to minimise the maximum relative error on that interval (fit in
-// float64, coefficients rounded to float32: max relative error 7.5e-5, about
-// 13.7 bits, enough for the 16-bit and 8-bit P it feeds); 2^n is added to the
-// exponent field.  Arguments are clamped to -125 (so the result stays a normal
-// float); callers only use this where no score is masked.
-__device__ __forceinline__ float poly_ex2(float x) {
-  x = fmaxf(x, -125.0f);
-  const float r = x + 12582912.0f;  // 1.5 * 2^23: rounds x to an integer in the low bits
-  const float f = x - (r - 12582912.0f);
-  float p = fmaf(0.05517113208770752f, f, 0.24261008203029633f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999281167984009f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -358,6 +340,55 @@ __device__ __forceinline__ f32x2 fadd2(f32x2 a, f32x2 b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
   return d;
+}
+
+__device__ __forceinline__ f32x2 fsub2(f32x2 a, f32x2 b) {
+  uint64_t ra, rb, rd;
+  f32x2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+
+// 2^x for a pair of arguments on the FMA pipe (keeps the MUFU free for the
+// other exponentials).  Cody-Waite style range reduction x = n + f with
+// n = round-to-nearest(x) through the 1.5*2^23 addition and f in [-1/2, 1/2];
+// 2^f from a degree-3 polynomial fitted to minimise the maximum relative error
+// on that interval (fit in float64, coefficients rounded to float32: max
+// relative error 7.5e-5, about 13.7 bits, enough for the 16-bit and 8-bit P it
+// feeds); 2^n is added to the exponent field.  Arguments are clamped to -125
+// (so the result stays a normal float); callers only use this where no score
+// is masked.  Packed float32 pairs: one instruction serves both lanes.
+__device__ __forceinline__ f32x2 poly_ex2x2(f32x2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const f32x2 big{12582912.0f, 12582912.0f};  // 1.5 * 2^23
+  const f32x2 r = fadd2(x, big);              // x rounded to an integer in the low bits
+  const f32x2 f = fsub2(x, fsub2(r, big));
+  f32x2 p = ffma2(f32x2{0.05517113208770752f, 0.05517113208770752f}, f,
+                  f32x2{0.24261008203029633f, 0.24261008203029633f});
+  p = ffma2(p, f, f32x2{0.6932609677314758f, 0.6932609677314758f});
+  p = ffma2(p, f, f32x2{0.9999281167984009f, 0.9999281167984009f});
+  return f32x2{__int_as_float(__float_as_int(p.x) + (__float_as_int(r.x) << 23)),
+               __int_as_float(__float_as_int(p.y) + (__float_as_int(r.y) << 23))};
+}
+__device__ __forceinline__ float poly_ex2(float x) { return poly_ex2x2(f32x2{x, x}).x; }
+
+// acc_lo + (low 16-bit value of w), acc_hi + (high 16-bit value of w), for a
+// pair of bf16 (or f16) values packed in one word: mixed-precision adds with a
+// 16-bit operand and a float32 accumulator (exact widening, one rounding).
+template <bool F16>
+__device__ __forceinline__ void add_16x2(uint32_t w, float& acc_lo, float& acc_hi) {
+  if constexpr (F16)
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi) : "r"(w));
+  else
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi) : "r"(w));
 }
 
 // Two floats -> packed e4m3 pair, `lo` in the low byte (round to nearest even,
