@@ -138,12 +138,11 @@ __device__ __forceinline__ void unpack_16x2(uint32_t v, float& lo, float& hi) {
 
 // Share of the exponentials that run on the FMA pipe (poly_ex2x2) instead of the
 // MUFU, on key tiles without masked scores: one pair in this many (0: none).
-#ifndef ATTN_POLY_EVERY
-#define ATTN_POLY_EVERY 0
-#endif
-#ifndef ATTN_POLY_EVERY_Q
-#define ATTN_POLY_EVERY_Q 0
-#endif
+// Measured on the video workload, every share tried (1/4, 1/8, 1/16) was slower
+// than none in both modes: the polynomial's extra instructions cost more issue
+// slots than the MUFU time they free.
+constexpr int kPolyEvery = 0;   // exact mode
+constexpr int kPolyEveryQ = 0;  // quantised mode
 
 // Per-tile row-sum accumulators of one softmax thread: r[] adds the 16-bit P
 // values that P.V multiplies (exact mode), f0/f1 the float32 P values.
@@ -378,13 +377,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       // Never leave with copies in flight into this CTA's shared memory.
       {
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(q_full, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+        while (!mbar_try_wait_sleep(q_full, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
         }
       }
       for (int s = 0; s < C::kNS; ++s)
         if (last_issue[s] >= 0) {
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full_bar(s), (last_issue[s] / C::kNS) & 1) &&
+          while (!mbar_try_wait_sleep(full_bar(s), (last_issue[s] / C::kNS) & 1) &&
                  globaltimer_ns() - t0 < kWaitTimeoutNs) {
           }
         }
@@ -497,7 +496,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       tc_commit(o_final);
       // Leave only once every issued MMA has finished (TMEM is freed at exit).
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(o_final, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!mbar_try_wait_sleep(o_final, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
   }
@@ -533,7 +532,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     float ksc_next = 1.0f;
     if constexpr (QUANT)
       if (n > 0) ksc_next = ld_global_f32(ksrc);
-    constexpr int kPoly = QUANT ? ATTN_POLY_EVERY_Q : ATTN_POLY_EVERY;
+    constexpr int kPoly = QUANT ? kPolyEveryQ : kPolyEvery;
     // Quantised scores arrive as int32 s; adding 0x4B400000 to the bits gives the
     // float F = 1.5 * 2^23 + s exactly (|s| < 2^22).  The offset is removed in the
     // maximum and folded into the exponent's FMA: 2^(F * c - K) with

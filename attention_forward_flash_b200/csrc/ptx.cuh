@@ -55,17 +55,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the waiting warp sleeps in hardware until
+// the phase completes (or the hint, in ns, runs out) instead of spinning, so
+// it takes no issue slots from the warps that share its scheduler.
+constexpr uint32_t kWaitHintNs = 1000000;  // 1 ms
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(kWaitHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of parity `parity` to complete.  Returns false if it
 // did not complete within kWaitTimeoutNs, or if another role of the CTA has
-// already raised `abort_flag` (a shared-memory word).
+// already raised `abort_flag` (a shared-memory word).  Each sleeping try_wait
+// lasts at most kWaitHintNs, so the flag and the clock are checked at
+// least that often.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           const volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
   }
