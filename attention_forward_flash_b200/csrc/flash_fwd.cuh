@@ -109,8 +109,8 @@ struct FwdCfg {
   // down to a multiple of 8) and their split between warpgroups: the
   // loader/MMA warpgroup needs few, the softmax warpgroups many.
   static constexpr int kRegsLaunch = (65536 / (kThreads * kCtasPerSm)) / 8 * 8;
-  static constexpr int kRegsLow = NQT == 2 ? 72 : 56;
-  static constexpr int kRegsHigh = NQT == 2 ? 216 : 200;
+  static constexpr int kRegsLow = NQT == 2 ? 88 : 56;
+  static constexpr int kRegsHigh = NQT == 2 ? 208 : 200;
 };
 
 template <bool F16>
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
 
   // Two-tile variant: 384 threads launched at 168 registers each (64512).  The
   // loader/MMA warpgroup needs few, the softmax warpgroups many:
-  // 128 x 56 + 256 x 224 = 64512, exactly the launch budget.
+  // 128 x 88 + 256 x 208 = 64512, exactly the launch budget.
   static_assert(128 * C::kRegsLow + (C::kThreads - 128) * C::kRegsHigh <=
                     C::kThreads * C::kRegsLaunch,
                 "register split exceeds the launch allocation");
