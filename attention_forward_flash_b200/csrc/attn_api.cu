@@ -320,12 +320,18 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
 
 #define ATTN_QUANT_LAUNCH(DD, FF)                                                              \
   do {                                                                                         \
-    if (nbq > 0)                                                                               \
-      quant_qk_kernel<DD, FF><<<dim3(nbq, BHq), 256, 0, st>>>(X(q), qb->q, qb->q_scale,        \
-                                                               p.q_len, nbq);                  \
+    static bool qk_attr = set_smem(quant_qk_kernel<DD, FF>, QuantQkCfg<DD>::kSmemBytes);        \
+    if (!qk_attr) return ATTN_ERR_CUDA;                                                        \
+    const int qk_ctas = QuantQkCfg<DD>::kCtasPerSm * c->num_sms;                               \
+    if (nbq > 0) {                                                                             \
+      const int tot = nbq * static_cast<int>(BHq);                                             \
+      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
+          X(q), qb->q, qb->q_scale, p.q_len, nbq, tot, c->err);                                \
+    }                                                                                          \
     if (nbk > 0) {                                                                             \
-      quant_qk_kernel<DD, FF><<<dim3(nbk, BHk), 256, 0, st>>>(X(k), qb->k, qb->k_scale,        \
-                                                               p.kv_len, nbk);                 \
+      const int tot = nbk * static_cast<int>(BHk);                                             \
+      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
+          X(k), qb->k, qb->k_scale, p.kv_len, nbk, tot, c->err);                               \
       v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(           \
           X(v), c->v_amax, p.kv_len);                                                          \
       v_quant_kernel<DD, FF><<<dim3(nbk, BHk), 2 * DD, 0, st>>>(X(v), c->v_amax, qb->v_t,      \

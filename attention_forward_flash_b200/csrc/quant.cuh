@@ -65,65 +65,151 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return r;
 }
 
-// grid: (ceil(S/128), B*H), 256 threads.  One CTA quantises one 128-token block.
+// Persistent: grid of a few CTAs per SM, 256 threads, each CTA walking the
+// 128-token blocks b = blockIdx.x, blockIdx.x + gridDim.x, ...  A block of one
+// (b, h) is contiguous (128 tokens x D, 16-bit), so one bulk copy brings it into
+// shared memory; two buffers let the next block stream in while this one is
+// reduced and quantised, keeping HBM busy.  Waits are bounded: on a timeout the
+// CTA records kErrTimeout in `err` and stops.
+template <int D>
+struct QuantQkCfg {
+  static constexpr int kBlockBytes = 128 * D * 2;
+  static constexpr int kSmemBytes = 2 * kBlockBytes + 64 + 128;  // buffers, barriers, reduction
+  static constexpr int kCtasPerSm = D == 128 ? 3 : 6;
+};
+
 template <int D, bool F16>
-__global__ void __launch_bounds__(256) quant_qk_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(256, QuantQkCfg<D>::kCtasPerSm) quant_qk_kernel(const uint16_t* __restrict__ x,
                                                        int8_t* __restrict__ codes,
                                                        float* __restrict__ scales, int S,
-                                                       int nblk) {
+                                                       int nblk, int total, unsigned* err) {
+  using C = QuantQkCfg<D>;
   constexpr int kChunks = 128 * D / 8;  // 16-byte chunks of a full block
   constexpr int kPer = kChunks / 256;
-  __shared__ float red[8];
-  const int t = blockIdx.x;
-  const size_t bh = blockIdx.y;
-  const int tok0 = t * 128;
-  const int nelem = min(128, S - tok0) * D;
-  const size_t base = (bh * S + tok0) * D;
-
-  uint4 w[kPer];
-  float amax = 0.0f;
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int c = threadIdx.x + k * 256;
-    if (c * 8 < nelem) {
-      w[k] = ld_nc_v4(x + base + (size_t)c * 8);
-      float f[8];
-      unpack8<F16>(w[k], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
-    } else {
-      w[k] = make_uint4(0, 0, 0, 0);
-    }
+  extern __shared__ __align__(128) uint8_t qsm[];
+  const uint32_t sbase = smem_u32(qsm);
+  const uint32_t bar0 = sbase + 2 * C::kBlockBytes;
+  float* red = reinterpret_cast<float*>(qsm + 2 * C::kBlockBytes + 64);
+  volatile int* stop = reinterpret_cast<volatile int*>(qsm + 2 * C::kBlockBytes + 32);
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    *stop = 0;
+    fence_mbar_init();
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
   __syncthreads();
-  amax = red[0];
-#pragma unroll
-  for (int k = 1; k < 8; ++k) amax = fmaxf(amax, red[k]);
-
-  const float s = __fdiv_rn(amax, 127.0f);
-  if (threadIdx.x == 0) scales[bh * nblk + t] = s;
-  const float r = __frcp_rn(s);
-  const bool fast = recip_ok(s);
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int c = threadIdx.x + k * 256;
-    if (c * 8 < nelem) {
-      float f[8];
-      unpack8<F16>(w[k], f);
-      uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        int qv = 0;
-        if (s > 0.0f) {
-          const float qf = fast ? div_by_recip(f[e], s, r) : __fdiv_rn(f[e], s);
-          qv = max(-127, min(127, __float2int_rn(qf)));
-        }
-        packed[e >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (e & 3));
+  auto block_bytes = [&](int b) {
+    const int t = b % nblk;
+    return (uint32_t)(min(128, S - t * 128) * D * 2);
+  };
+  auto issue = [&](int b, int stage) {  // thread 0
+    const size_t bh = b / nblk;
+    const int t = b % nblk;
+    const uint32_t bytes = block_bytes(b);
+    mbar_arrive_expect_tx(bar0 + 8 * stage, bytes);
+    bulk_load(sbase + stage * C::kBlockBytes, x + (bh * S + (size_t)t * 128) * D, bytes,
+              bar0 + 8 * stage);
+  };
+  if (threadIdx.x == 0) {
+    if (blockIdx.x < total) issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < total) issue(blockIdx.x + gridDim.x, 1);
+  }
+  int it = 0;
+  for (int b = blockIdx.x; b < total; b += gridDim.x, ++it) {
+    const int stage = it & 1;
+    const uint32_t bar = bar0 + 8 * stage;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar, (it >> 1) & 1, stop))) {
+      if ((threadIdx.x & 31) == 0) {
+        *stop = 1;
+        atomicOr(err, 1u);
       }
-      *reinterpret_cast<uint2*>(codes + base + (size_t)c * 8) = make_uint2(packed[0], packed[1]);
+      break;
+    }
+    const size_t bh = b / nblk;
+    const int t = b % nblk;
+    const int nelem = min(128, S - t * 128) * D;
+    const uint4* src = reinterpret_cast<const uint4*>(qsm + stage * C::kBlockBytes);
+    uint4 w[kPer];
+    float amax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int c = threadIdx.x + k * 256;
+      if (c * 8 < nelem) {
+        w[k] = src[c];
+        float f[8];
+        unpack8<F16>(w[k], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+      } else {
+        w[k] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();  // every thread holds its data: the buffer may be refilled
+    if (threadIdx.x == 0 && b + 2 * gridDim.x < total) {
+      fence_proxy_async_smem();  // the generic reads above come before the async refill
+      issue(b + 2 * gridDim.x, stage);
+    }
+    amax = red[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) amax = fmaxf(amax, red[k]);
+
+    const float s = __fdiv_rn(amax, 127.0f);
+    if (threadIdx.x == 0) scales[bh * nblk + t] = s;
+    const float r = __frcp_rn(s);
+    const bool fast = recip_ok(s);
+    const size_t base = (bh * S + (size_t)t * 128) * D;
+    // code = rint_half_even(x / s).  |x| <= amax, so |x / s| <= 127 (1 + 2^-24) < 127.5
+    // and the clamp to +-127 never acts; -0 and +0 both give code 0.  Fast path:
+    // the correctly rounded quotient through the reciprocal (packed pairs), then
+    // round-half-even by adding 1.5 * 2^23 (the integer lands in the low bits:
+    // its low byte is the code).
+    const f32x2 rr{r, r}, ns{-s, -s}, big{12582912.0f, 12582912.0f};
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int c = threadIdx.x + k * 256;
+      if (c * 8 < nelem) {
+        float f[8];
+        unpack8<F16>(w[k], f);
+        uint32_t bits[8];
+        if (fast) {
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const f32x2 xv{f[e], f[e + 1]};
+            const f32x2 y = fmul2(xv, rr);
+            const f32x2 q = ffma2(ffma2(y, ns, xv), rr, y);  // Markstein correction
+            const f32x2 m = fadd2(q, big);
+            bits[e] = __float_as_uint(m.x);
+            bits[e + 1] = __float_as_uint(m.y);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int qv = (s > 0.0f) ? max(-127, min(127, __float2int_rn(__fdiv_rn(f[e], s)))) : 0;
+            bits[e] = static_cast<uint32_t>(qv);
+          }
+        }
+        const uint32_t w0 = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
+                                        __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
+        const uint32_t w1 = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
+                                        __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
+        *reinterpret_cast<uint2*>(codes + base + (size_t)c * 8) = make_uint2(w0, w1);
+      }
+    }
+    __syncthreads();  // red[] is rewritten by the next block
+  }
+  // Never leave with a copy in flight into this CTA's shared memory.
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < 2; ++k) {
+      const int b = blockIdx.x + (it + k) * gridDim.x;
+      if (b < total) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(bar0 + 8 * ((it + k) & 1), ((it + k) >> 1) & 1) &&
+               globaltimer_ns() - t0 < kWaitTimeoutNs) {
+        }
+      }
     }
   }
 }
