@@ -334,8 +334,11 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
           X(k), qb->k, qb->k_scale, p.kv_len, nbk, tot, c->err);                               \
       v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(           \
           X(v), c->v_amax, p.kv_len);                                                          \
-      v_quant_kernel<DD, FF><<<dim3(nbk, BHk), 2 * DD, 0, st>>>(X(v), c->v_amax, qb->v_t,      \
-                                                              qb->v_scale, p.kv_len, S_pad);   \
+      static bool vq_attr = set_smem(v_quant_kernel<DD, FF>, VQuantCfg<DD>::kSmemBytes);       \
+      if (!vq_attr) return ATTN_ERR_CUDA;                                                      \
+      const int vq_ctas = std::min(tot, VQuantCfg<DD>::kCtasPerSm * c->num_sms);               \
+      v_quant_kernel<DD, FF><<<vq_ctas, 256, VQuantCfg<DD>::kSmemBytes, st>>>(                 \
+          X(v), c->v_amax, qb->v_t, qb->v_scale, p.kv_len, S_pad, nbk, tot, c->err);           \
     }                                                                                          \
   } while (0)
 

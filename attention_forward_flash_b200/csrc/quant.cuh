@@ -37,6 +37,18 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
   }
 }
 
+template <bool F16>
+__device__ __forceinline__ void unpack_16x2_v(uint32_t w, float& lo, float& hi) {
+  if constexpr (F16) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&w);
+    lo = __low2float(h);
+    hi = __high2float(h);
+  } else {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+  }
+}
+
 // x / s correctly rounded (the float32 division) from the block's reciprocal:
 // y = RN(x * r) with r = RN(1/s) is within an ulp of x / s, the residual
 // x - y * s is exact under one fused multiply-add, and RN(y + residual * r) is
@@ -245,52 +257,150 @@ __global__ void __launch_bounds__(256) v_amax_kernel(const uint16_t* __restrict_
   for (int c = threadIdx.x; c < D; c += 256) atomicMax(&amax_bits[u * D + c], smax[c]);
 }
 
-// grid: (S_pad/128, B*Hkv), 2*D threads.  Quantise a 128-token tile of V and
-// write it transposed.  Thread (channel c, token half h) converts tokens
-// [64h, 64h + 64) of channel c: every load instruction of a warp reads 32
-// neighbouring channels of one token (64 contiguous bytes) and every store
-// writes 16 consecutive codes of one channel row.
+// Quantise 128-token tiles of V and write them transposed.  Persistent, like
+// quant_qk_kernel: tiles (unit u, tile t) in turn, each brought into shared
+// memory by one bulk copy (a tile of one unit is contiguous) while the previous
+// one is converted.  Thread (channel pair cp, token group tg) converts channels
+// 2cp, 2cp + 1 for a run of tokens: each 32-bit shared load gives both channels
+// of one token (a warp reads one token row without bank conflicts), divisions
+// are paired along tokens, and each channel's codes leave as 16-byte stores of
+// consecutive tokens.  s = amax / 448 per (u, channel); the code is the E4M3
+// value of x / s (correctly rounded quotient, nearest even, saturating), with
+// the sign of a zero following x; tokens past S and all-zero channels give 0.
+template <int D>
+struct VQuantCfg {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kSmemBytes = 2 * kTileBytes + 64;
+  static constexpr int kPairs = D / 2;              // channel pairs
+  static constexpr int kGroups = 256 / kPairs;      // token groups
+  static constexpr int kRun = 128 / kGroups;        // tokens per thread
+  static constexpr int kCtasPerSm = D == 128 ? 3 : 6;
+};
+
 template <int D, bool F16>
-__global__ void __launch_bounds__(2 * D) v_quant_kernel(const uint16_t* __restrict__ v,
-                                                        const unsigned* __restrict__ amax_bits,
-                                                        uint8_t* __restrict__ vt,
-                                                        float* __restrict__ v_scale, int S,
-                                                        int S_pad) {
-  const size_t u = blockIdx.y;
-  const int tok0 = blockIdx.x * 128;
-  const int c = threadIdx.x % D;
-  const int half = threadIdx.x / D;
-  const float s = __fdiv_rn(__uint_as_float(amax_bits[u * D + c]), 448.0f);
-  if (blockIdx.x == 0 && half == 0) v_scale[u * D + c] = s;
-  const float r = __frcp_rn(s);
-  const bool fast = recip_ok(s);
-  const uint16_t* src = v + (u * S) * D + c;
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {                 // 4 groups of 16 tokens
-    const int t0 = tok0 + half * 64 + g * 16;
-    uint16_t raw[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) raw[i] = (t0 + i < S) ? __ldg(src + (size_t)(t0 + i) * D) : 0;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      float f0, f1;
-      if constexpr (F16) {
-        f0 = __half2float(__ushort_as_half(raw[i]));
-        f1 = __half2float(__ushort_as_half(raw[i + 1]));
-      } else {
-        f0 = __bfloat162float(__ushort_as_bfloat16(raw[i]));
-        f1 = __bfloat162float(__ushort_as_bfloat16(raw[i + 1]));
-      }
-      float a0 = 0.0f, a1 = 0.0f;
-      if (s > 0.0f) {
-        a0 = (t0 + i < S) ? (fast ? div_by_recip(f0, s, r) : __fdiv_rn(f0, s)) : 0.0f;
-        a1 = (t0 + i + 1 < S) ? (fast ? div_by_recip(f1, s, r) : __fdiv_rn(f1, s)) : 0.0f;
-      }
-      w[i / 4] |= uint32_t(f32x2_to_e4m3x2(a0, a1)) << (16 * ((i / 2) & 1));
+__global__ void __launch_bounds__(256, VQuantCfg<D>::kCtasPerSm)
+    v_quant_kernel(const uint16_t* __restrict__ v, const unsigned* __restrict__ amax_bits,
+                   uint8_t* __restrict__ vt, float* __restrict__ v_scale, int S, int S_pad,
+                   int nbk, int total, unsigned* err) {
+  using C = VQuantCfg<D>;
+  extern __shared__ __align__(128) uint8_t vsm[];
+  const uint32_t sbase = smem_u32(vsm);
+  const uint32_t bar0 = sbase + 2 * C::kTileBytes;
+  volatile int* stop = reinterpret_cast<volatile int*>(vsm + 2 * C::kTileBytes + 32);
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    *stop = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int b, int stage) {  // thread 0
+    const size_t u = b / nbk;
+    const int t = b % nbk;
+    const uint32_t bytes = (uint32_t)(min(128, S - t * 128) * D * 2);
+    mbar_arrive_expect_tx(bar0 + 8 * stage, bytes);
+    bulk_load(sbase + stage * C::kTileBytes, v + (u * S + (size_t)t * 128) * D, bytes,
+              bar0 + 8 * stage);
+  };
+  if (threadIdx.x == 0) {
+    if (blockIdx.x < total) issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < total) issue(blockIdx.x + gridDim.x, 1);
+  }
+  const int cp = threadIdx.x % C::kPairs;
+  const int tg = threadIdx.x / C::kPairs;
+  const int c0 = 2 * cp;
+  int it = 0;
+  for (int b = blockIdx.x; b < total; b += gridDim.x, ++it) {
+    const int stage = it & 1;
+    const size_t u = b / nbk;
+    const int t = b % nbk;
+    // scales of this thread's two channels
+    const float s0 = __fdiv_rn(__uint_as_float(amax_bits[u * D + c0]), 448.0f);
+    const float s1 = __fdiv_rn(__uint_as_float(amax_bits[u * D + c0 + 1]), 448.0f);
+    if (t == 0 && tg == 0) {
+      v_scale[u * D + c0] = s0;
+      v_scale[u * D + c0 + 1] = s1;
     }
-    *reinterpret_cast<uint4*>(vt + (u * D + c) * (size_t)S_pad + t0) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+    const bool fast = recip_ok(s0) && recip_ok(s1);
+    const float r0 = __frcp_rn(s0), r1 = __frcp_rn(s1);
+    if (!__all_sync(0xffffffffu, mbar_wait(bar0 + 8 * stage, (it >> 1) & 1, stop))) {
+      if ((threadIdx.x & 31) == 0) {
+        *stop = 1;
+        atomicOr(err, 1u);
+      }
+      break;
+    }
+    const int ntok = min(128, S - t * 128);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(vsm + stage * C::kTileBytes) + cp;
+    const int tk0 = tg * C::kRun;
+    uint32_t out0[C::kRun / 4], out1[C::kRun / 4];  // codes of channel c0, c0 + 1
+#pragma unroll
+    for (int i = 0; i < C::kRun; i += 2) {
+      const int ta = tk0 + i, tb = tk0 + i + 1;
+      const uint32_t wa = ta < ntok ? src[ta * (D / 2)] : 0u;
+      const uint32_t wb = tb < ntok ? src[tb * (D / 2)] : 0u;
+      float xa0, xa1, xb0, xb1;  // token a / b, channel c0 / c0 + 1
+      unpack_16x2_v<F16>(wa, xa0, xa1);
+      unpack_16x2_v<F16>(wb, xb0, xb1);
+      float q0a = 0.0f, q0b = 0.0f, q1a = 0.0f, q1b = 0.0f;
+      if (fast) {
+        const f32x2 x0{xa0, xb0}, x1{xa1, xb1};
+        const f32x2 y0 = fmul2(x0, f32x2{r0, r0}), y1 = fmul2(x1, f32x2{r1, r1});
+        const f32x2 z0 = ffma2(ffma2(y0, f32x2{-s0, -s0}, x0), f32x2{r0, r0}, y0);
+        const f32x2 z1 = ffma2(ffma2(y1, f32x2{-s1, -s1}, x1), f32x2{r1, r1}, y1);
+        q0a = copysignf(z0.x, xa0);
+        q0b = copysignf(z0.y, xb0);
+        q1a = copysignf(z1.x, xa1);
+        q1b = copysignf(z1.y, xb1);
+      } else {
+        if (s0 > 0.0f) {
+          q0a = __fdiv_rn(xa0, s0);
+          q0b = __fdiv_rn(xb0, s0);
+        }
+        if (s1 > 0.0f) {
+          q1a = __fdiv_rn(xa1, s1);
+          q1b = __fdiv_rn(xb1, s1);
+        }
+      }
+      if (s0 <= 0.0f) q0a = q0b = 0.0f;
+      if (s1 <= 0.0f) q1a = q1b = 0.0f;
+      if (ta >= ntok) q0a = q1a = 0.0f;  // padding tokens: code 0x00
+      if (tb >= ntok) q0b = q1b = 0.0f;
+      const uint32_t h0 = f32x2_to_e4m3x2(q0a, q0b), h1 = f32x2_to_e4m3x2(q1a, q1b);
+      if (i % 4 == 0) {
+        out0[i / 4] = h0;
+        out1[i / 4] = h1;
+      } else {
+        out0[i / 4] |= h0 << 16;
+        out1[i / 4] |= h1 << 16;
+      }
+    }
+    __syncthreads();  // every thread has read the tile: the buffer may be refilled
+    if (threadIdx.x == 0 && b + 2 * gridDim.x < total) {
+      fence_proxy_async_smem();
+      issue(b + 2 * gridDim.x, stage);
+    }
+    uint8_t* d0 = vt + (u * D + c0) * (size_t)S_pad + (size_t)t * 128 + tk0;
+    uint8_t* d1 = d0 + S_pad;
+#pragma unroll
+    for (int k = 0; k < C::kRun / 16; ++k) {
+      reinterpret_cast<uint4*>(d0)[k] =
+          make_uint4(out0[4 * k], out0[4 * k + 1], out0[4 * k + 2], out0[4 * k + 3]);
+      reinterpret_cast<uint4*>(d1)[k] =
+          make_uint4(out1[4 * k], out1[4 * k + 1], out1[4 * k + 2], out1[4 * k + 3]);
+    }
+  }
+  // Never leave with a copy in flight into this CTA's shared memory.
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < 2; ++k) {
+      const int b = blockIdx.x + (it + k) * gridDim.x;
+      if (b < total) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(bar0 + 8 * ((it + k) & 1), ((it + k) >> 1) & 1) &&
+               globaltimer_ns() - t0 < kWaitTimeoutNs) {
+        }
+      }
+    }
   }
 }
 
