@@ -20,79 +20,105 @@ namespace attn {
 constexpr int kMergeMaxSplits = 128;
 constexpr int kMergeWarps = 4;
 
-// grid: rows, 128 threads; one CTA per output row.  Warp 0 computes every
-// split's weight once (cached in shared memory) and the denominator; then warp w
-// accumulates splits w, w + 4, ... with all of its loads in flight, and the four
-// partial sums are added in shared memory.
+// grid: rows, 128 threads; one CTA per output row.  Every warp loads all
+// splits' weight exponents (one per lane) together with the partial outputs of
+// its own splits w, w + 4, ..., so that both arrive in one memory round trip;
+// each warp then forms the maximum, its splits' weights and the denominator
+// itself, and the four partial sums are added in shared memory.
 template <int D, bool F16>
 __global__ void __launch_bounds__(32 * kMergeWarps) splitkv_merge_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
     uint16_t* __restrict__ out, float* __restrict__ lse, int rows, int splits) {
-  constexpr int kPer = D / 32;  // channels per lane
-  __shared__ float wts[kMergeMaxSplits];
+  constexpr int kPer = D / 32;                    // channels per lane
+  constexpr int kMaxPerWarp = kMergeMaxSplits / kMergeWarps;
   __shared__ float red[kMergeWarps][D];
-  __shared__ float inv_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x;
   // Launched as a programmatic dependent of the split kernel: wait until that
   // grid has completed and its partials are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (warp == 0) {
-    float M = -INFINITY;
-    for (int s = lane; s < splits; s += 32) M = fmaxf(M, lse_part[(size_t)s * rows + row]);
+  // this lane's share of the weight exponents (splits lane, lane + 32, ...)
+  float W[kMergeMaxSplits / 32];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float wsum = 0.0f;
-    for (int s = lane; s < splits; s += 32) {
-      const float L = lse_part[(size_t)s * rows + row];
-      const float w = (M == -INFINITY) ? 0.0f : ex2(L - M);
-      wts[s] = w;
-      wsum += w;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    if (lane == 0) inv_s = (wsum > 0.0f) ? 1.0f / wsum : 0.0f;
-    if (lse != nullptr) {
-      const float* lf = lse_part + (size_t)splits * rows;
-      float ML = -INFINITY;
-      for (int s = lane; s < splits; s += 32) ML = fmaxf(ML, lf[(size_t)s * rows + row]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ML = fmaxf(ML, __shfl_xor_sync(0xffffffffu, ML, o));
-      float ls = 0.0f;
-      for (int s = lane; s < splits; s += 32)
-        ls += (ML == -INFINITY) ? 0.0f : ex2(lf[(size_t)s * rows + row] - ML);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-      if (lane == 0)
-        lse[row] = (ls > 0.0f) ? (ML + lg2(ls)) * 0.69314718055994531f : -INFINITY;
-    }
+  for (int k = 0; k < kMergeMaxSplits / 32; ++k) {
+    const int sp = lane + 32 * k;
+    W[k] = sp < splits ? lse_part[(size_t)sp * rows + row] : -INFINITY;
   }
-  __syncthreads();
+  // this warp's partial outputs, all loads in flight
+  float part[kMaxPerWarp / 4][kPer];  // splits warp + 4 i, in groups processed below
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.0f;
-#pragma unroll 8
-  for (int s = warp; s < splits; s += kMergeWarps) {
-    const float w = wts[s];
-    if (w == 0.0f) continue;  // empty or negligible split: its partials are never read
-    const float* src = o_part + ((size_t)s * rows + row) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
-      acc[2] += w * v.z;
-      acc[3] += w * v.w;
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(src);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
+  float M = -INFINITY, wsum = 0.0f;
+  // splits warp + 4 i in groups of kMaxPerWarp / 4; the first group's loads are
+  // issued before the weight exponents are used, so both are in flight together
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    const int i0 = g * (kMaxPerWarp / 4);
+    if (g > 0 && warp + 4 * i0 >= splits) break;
+#pragma unroll
+    for (int i = 0; i < kMaxPerWarp / 4; ++i) {
+      const int sp = warp + 4 * (i0 + i);
+      const float* src = o_part + ((size_t)sp * rows + row) * D + lane * kPer;
+      if (sp < splits) {
+        if constexpr (kPer == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          part[i][0] = v.x; part[i][1] = v.y; part[i][2] = v.z; part[i][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          part[i][0] = v.x; part[i][1] = v.y;
+        }
+      }
+    }
+    if (g == 0) {
+#pragma unroll
+      for (int k = 0; k < kMergeMaxSplits / 32; ++k) M = fmaxf(M, W[k]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+#pragma unroll
+      for (int k = 0; k < kMergeMaxSplits / 32; ++k)
+        wsum += (M == -INFINITY || W[k] == -INFINITY) ? 0.0f : ex2(W[k] - M);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxPerWarp / 4; ++i) {
+      const int sp = warp + 4 * (i0 + i);
+      // weight of split sp from the lane that holds its exponent (all lanes take part)
+      const int k = sp >> 5;
+      const float Wk = k == 0 ? W[0] : k == 1 ? W[1] : k == 2 ? W[2] : W[3];
+      const float Ws = __shfl_sync(0xffffffffu, Wk, sp & 31);
+      if (sp < splits) {
+        const float w = (M == -INFINITY || Ws == -INFINITY) ? 0.0f : ex2(Ws - M);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] += w * part[i][e];
+      }
     }
   }
 #pragma unroll
   for (int e = 0; e < kPer; ++e) red[warp][lane * kPer + e] = acc[e];
+  if (warp == 1 && lse != nullptr) {
+    const float* lf = lse_part + (size_t)splits * rows;
+    float ML = -INFINITY, F[kMergeMaxSplits / 32];
+#pragma unroll
+    for (int k = 0; k < kMergeMaxSplits / 32; ++k) {
+      const int sp = lane + 32 * k;
+      F[k] = sp < splits ? lf[(size_t)sp * rows + row] : -INFINITY;
+      ML = fmaxf(ML, F[k]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ML = fmaxf(ML, __shfl_xor_sync(0xffffffffu, ML, o));
+    float ls = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kMergeMaxSplits / 32; ++k)
+      ls += (ML == -INFINITY || F[k] == -INFINITY) ? 0.0f : ex2(F[k] - ML);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) lse[row] = (ls > 0.0f) ? (ML + lg2(ls)) * 0.69314718055994531f : -INFINITY;
+  }
   __syncthreads();
   if (warp == 0) {
-    const float inv = inv_s;
+    const float inv = (wsum > 0.0f) ? 1.0f / wsum : 0.0f;
     uint16_t h[kPer];
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
