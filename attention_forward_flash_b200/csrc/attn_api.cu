@@ -326,12 +326,12 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
     if (nbq > 0) {                                                                             \
       const int tot = nbq * static_cast<int>(BHq);                                             \
       quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
-          X(q), qb->q, qb->q_scale, p.q_len, nbq, tot, c->err);                                \
+          X(q), qb->q, qb->q_scale, p.q_len, nbq, tot, c->err, c->debug);                      \
     }                                                                                          \
     if (nbk > 0) {                                                                             \
       const int tot = nbk * static_cast<int>(BHk);                                             \
       quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
-          X(k), qb->k, qb->k_scale, p.kv_len, nbk, tot, c->err);                               \
+          X(k), qb->k, qb->k_scale, p.kv_len, nbk, tot, c->err, 0u);                           \
       v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(           \
           X(v), c->v_amax, p.kv_len);                                                          \
       static bool vq_attr = set_smem(v_quant_kernel<DD, FF>, VQuantCfg<DD>::kSmemBytes);       \

@@ -94,7 +94,8 @@ template <int D, bool F16>
 __global__ void __launch_bounds__(256, QuantQkCfg<D>::kCtasPerSm) quant_qk_kernel(const uint16_t* __restrict__ x,
                                                        int8_t* __restrict__ codes,
                                                        float* __restrict__ scales, int S,
-                                                       int nblk, int total, unsigned* err) {
+                                                       int nblk, int total, unsigned* err,
+                                                       unsigned debug) {
   using C = QuantQkCfg<D>;
   constexpr int kChunks = 128 * D / 8;  // 16-byte chunks of a full block
   constexpr int kPer = kChunks / 256;
@@ -124,7 +125,9 @@ __global__ void __launch_bounds__(256, QuantQkCfg<D>::kCtasPerSm) quant_qk_kerne
   };
   if (threadIdx.x == 0) {
     if (blockIdx.x < total) issue(blockIdx.x, 0);
-    if (blockIdx.x + gridDim.x < total) issue(blockIdx.x + gridDim.x, 1);
+    // timeout test (bit 1): CTA 0 never loads its second block
+    if (blockIdx.x + gridDim.x < total && !((debug & 2u) && blockIdx.x == 0))
+      issue(blockIdx.x + gridDim.x, 1);
   }
   int it = 0;
   for (int b = blockIdx.x; b < total; b += gridDim.x, ++it) {

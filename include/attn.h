@@ -144,8 +144,10 @@ int attn_num_splits(const attn_ctx *c);
 
 /* TEST HOOK.  Bit 0 of `flags` makes the next attn_forward's loader skip the
  * second key tile of every CTA, so that the waits on it run out: the kernel then
- * records ATTN_ERR_TIMEOUT in the context and returns without hanging.  The
- * hook exists only to test that error path; 0 restores normal operation. */
+ * records ATTN_ERR_TIMEOUT in the context and returns without hanging.  Bit 1
+ * does the same to attn_quantize_qk: the first CTA of the Q quantiser never
+ * loads its second block.  The hook exists only to test that error path; 0
+ * restores normal operation. */
 attn_status attn_debug_set(attn_ctx *c, unsigned flags);
 
 /* TEST HOOK.  y[i] = 2^x[i] (device pointers, n floats) computed by the

@@ -74,3 +74,25 @@ def test_quantiser_bit_exact_full_workloads(name):
     w = WORKLOADS[name]
     q, k, v = make_qkv(w)
     _check_quant(q, k, v, w.torch_dtype)
+
+
+def test_quantiser_wait_timeout_is_reported_and_context_survives():
+    """A block copy that never arrives (test hook: the Q quantiser's first CTA skips
+    its second block) ends in a bounded wait: ATTN_ERR_TIMEOUT is reported, nothing
+    hangs, and the next call on the same context is bit-exact again."""
+    from attention_forward_flash_b200 import _abi
+    B, Hq, Hk, S, D = 1, 32, 8, 4096, 128   # 1024 Q blocks: more than the quantiser CTAs
+    g = torch.Generator().manual_seed(21)
+    q, k, v = (torch.randn(B, h, S, D, generator=g).to(torch.bfloat16) for h in (Hq, Hk, Hk))
+    att = Attention(B, Hq, Hk, S, S, D, precision="quant")
+    _abi.attn_debug_set(att.ctx, 2)
+    att.quantize(q.cuda(), k.cuda(), v.cuda())
+    with pytest.raises(_abi.AttnError) as e:
+        att.check_error()
+    assert e.value.status == _abi.ATTN_ERR_TIMEOUT
+    _abi.attn_debug_set(att.ctx, 0)
+    qb = att.quantize(q.cuda(), k.cuda(), v.cuda())
+    att.check_error()
+    rq, rqs = quantize_qk_int8(q.float().numpy())
+    assert np.array_equal(qb.q_scale.cpu().numpy().view(np.uint32), rqs.view(np.uint32))
+    assert np.array_equal(qb.q.cpu().numpy(), rq)
