@@ -28,4 +28,4 @@ from ._abi import (  # noqa: F401
     lib,
     lib_path,
 )
-from .api import Attention, QuantBuffers  # noqa: F401
+from .api import Attention, DeviceStaging, QuantBuffers  # noqa: F401

@@ -12,7 +12,7 @@ ATTN_EXACT, ATTN_INT8QK_FP8PV = 0, 1
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
-            "attn_debug_exp2", "attn_forward_splitkv_noalloc")
+            "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -77,6 +77,8 @@ def lib():
         L.attn_forward_splitkv_noalloc.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp,
                                                    vp, vp]
         L.attn_forward_splitkv_noalloc.restype = c_int
+        L.attn_forward_host.argtypes = [vp] * 11 + [ctypes.POINTER(AttnQBufs), c_int, vp]
+        L.attn_forward_host.restype = c_int
         _LIB = L
     return _LIB
 
@@ -134,3 +136,11 @@ def attn_debug_exp2(x, y, n, stream):
 def attn_forward_splitkv_noalloc(params: AttnParams, q, k, v, o, lse, err, stream):
     _check(lib().attn_forward_splitkv_noalloc(ctypes.byref(params), q, k, v, o, lse, err, stream),
            "attn_forward_splitkv_noalloc")
+
+
+def attn_forward_host(ctx, q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev,
+                      lse_dev, qbufs, chunks, stream):
+    qb = ctypes.byref(qbufs) if qbufs is not None else None
+    _check(lib().attn_forward_host(ctx, q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev,
+                                   v_dev, o_dev, lse_dev, qb, chunks, stream),
+           "attn_forward_host")

@@ -39,6 +39,21 @@ class QuantBuffers:
                          self.k_scale.data_ptr(), self.v_t.data_ptr(), self.v_scale.data_ptr())
 
 
+class DeviceStaging:
+    """Device buffers that ``Attention.forward_host`` copies through (full problem size)."""
+
+    def __init__(self, params: AttnParams, dtype, device, quant, with_lse):
+        B, Hq, Hk = params.batch, params.n_q_heads, params.n_kv_heads
+        Sq, Sk, D = params.q_len, params.kv_len, params.head_dim
+        self.q = torch.empty((B, Hq, Sq, D), dtype=dtype, device=device)
+        self.k = torch.empty((B, Hk, Sk, D), dtype=dtype, device=device)
+        self.v = torch.empty((B, Hk, Sk, D), dtype=dtype, device=device)
+        self.o = torch.empty((B, Hq, Sq, D), dtype=dtype, device=device)
+        self.lse = (torch.empty((B, Hq, Sq), dtype=torch.float32, device=device)
+                    if with_lse else None)
+        self.qbufs = QuantBuffers(params, device) if quant else None
+
+
 class Attention:
     """One attention problem shape bound to a library context."""
 
@@ -59,14 +74,16 @@ class Attention:
     def num_splits(self):
         return _abi.attn_num_splits(self.ctx)
 
-    def _check_inputs(self, q, k, v):
+    def _check_inputs(self, q, k, v, on_cuda=True):
         p = self.params
         want_q = (p.batch, p.n_q_heads, p.q_len, p.head_dim)
         want_kv = (p.batch, p.n_kv_heads, p.kv_len, p.head_dim)
+        where = "CUDA" if on_cuda else "host"
         for name, t, shape in (("q", q, want_q), ("k", k, want_kv), ("v", v, want_kv)):
-            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous() or not t.is_cuda:
-                raise ValueError(f"{name}: expected contiguous CUDA {self.dtype} of shape {shape}, "
-                                 f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+            if (tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous()
+                    or t.is_cuda != on_cuda):
+                raise ValueError(f"{name}: expected contiguous {where} {self.dtype} of shape "
+                                 f"{shape}, got {t.dtype} {tuple(t.shape)} on {t.device}")
 
     def quantize(self, q, k, v, qbufs=None, stream=None):
         if self.precision != "quant":
@@ -99,6 +116,45 @@ class Attention:
         return (out, lse) if return_lse else out
 
     __call__ = forward
+
+    def forward_host(self, q, k, v, *, out=None, lse=None, return_lse=False, staging=None,
+                     chunks=0, stream=None, device=None):
+        """End-to-end forward from host tensors through ``attn_forward_host``.
+
+        q, k, v: contiguous CPU tensors (page-locked ones let the copies overlap the
+        kernels).  out / lse: CPU tensors to write (page-locked ones are allocated if
+        None).  staging: the ``DeviceStaging`` to copy through; one is allocated on
+        ``device`` (default: the current CUDA device) and kept for later calls if
+        None.  Calls that share a staging must be ordered (one stream).  The call is
+        asynchronous on ``stream``: synchronise it before reading the outputs.
+        """
+        p = self.params
+        self._check_inputs(q, k, v, on_cuda=False)
+        want_lse = return_lse or lse is not None
+        if staging is None:
+            cached = getattr(self, "_staging", None)
+            if cached is None or (want_lse and cached.lse is None):
+                dev = (device if device is not None
+                       else torch.device("cuda", torch.cuda.current_device()))
+                cached = DeviceStaging(p, self.dtype, dev, self.precision == "quant", want_lse)
+                self._staging = cached
+            staging = cached
+        if out is None:
+            out = torch.empty((p.batch, p.n_q_heads, p.q_len, p.head_dim), dtype=self.dtype,
+                              pin_memory=True)
+        if lse is None and return_lse:
+            lse = torch.empty((p.batch, p.n_q_heads, p.q_len), dtype=torch.float32,
+                              pin_memory=True)
+        if lse is not None and staging.lse is None:
+            raise ValueError("lse requested but the staging has no lse buffer")
+        lse_host = lse.data_ptr() if lse is not None else None
+        lse_dev = staging.lse.data_ptr() if lse is not None else None
+        qb = staging.qbufs.struct() if staging.qbufs is not None else None
+        _abi.attn_forward_host(self.ctx, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse_host, staging.q.data_ptr(), staging.k.data_ptr(),
+                               staging.v.data_ptr(), staging.o.data_ptr(), lse_dev, qb, chunks,
+                               _stream_handle(stream))
+        return (out, lse) if return_lse else out
 
     def check_error(self, stream=None):
         """Synchronise and raise AttnError if a kernel recorded a failed wait."""

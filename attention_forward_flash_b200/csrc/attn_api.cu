@@ -17,6 +17,10 @@
 
 using namespace attn;
 
+namespace {
+constexpr int kMaxHostChunks = 64;  // ranges of units of one attn_forward_host call
+}  // namespace
+
 struct attn_ctx {
   attn_params p;
   int device;
@@ -36,6 +40,13 @@ struct attn_ctx {
   unsigned* v_amax;
   unsigned* err;
   unsigned debug;
+  // attn_forward_host's pipeline, created by its first call: stream 0 carries the
+  // host-to-device copies, 1 and 2 the kernels of even and odd ranges, 3 the
+  // device-to-host copies.
+  bool pipe_ready;
+  cudaStream_t pipe[4];
+  cudaEvent_t pev_start, pev_join[4];
+  cudaEvent_t pev_in[kMaxHostChunks], pev_done[kMaxHostChunks];
 };
 
 namespace {
@@ -145,6 +156,248 @@ attn_status validate(const attn_params* p) {
   if (rows > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->start_pos) + p->q_len > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
+}
+
+// Pointer checks of attn_forward.  Buffers of zero length may be NULL (an empty
+// tensor has no storage); every other one must be non-NULL and 16-byte aligned.
+bool bad_ptr(const void* ptr, bool needed) {
+  return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));
+}
+
+bool bad_qbufs(const attn_params& p, const attn_qbufs* qb) {
+  const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
+  return !qb || bad_ptr(qb->q, need_q) || bad_ptr(qb->q_scale, need_q) ||
+         bad_ptr(qb->k, need_kv) || bad_ptr(qb->k_scale, need_kv) || bad_ptr(qb->v_t, need_kv) ||
+         bad_ptr(qb->v_scale, need_kv);
+}
+
+attn_status check_forward_buffers(const attn_ctx* c, const void* q, const void* k, const void* v,
+                                  const attn_qbufs* qb, const void* o, const float* lse) {
+  const attn_params& p = c->p;
+  const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
+  if (bad_ptr(o, need_q) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
+  if (p.precision == ATTN_INT8QK_FP8PV) {
+    if (bad_qbufs(p, qb)) return ATTN_ERR_INVALID_ARG;
+  } else {
+    if (qb) return ATTN_ERR_INVALID_ARG;
+    if (bad_ptr(q, need_q) || bad_ptr(k, need_kv) || bad_ptr(v, need_kv))
+      return ATTN_ERR_INVALID_ARG;
+  }
+  return ATTN_OK;
+}
+
+// Launches the quantisers on `st` for the units [u0, u0 + nu) (unit = one
+// (batch, kv head) pair with its query heads).  Pointers are those of the whole
+// problem, already validated.
+attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const void* k,
+                           const void* v, const attn_qbufs* qb, cudaStream_t st) {
+  const attn_params& p = c->p;
+  const int D = p.head_dim;
+  const bool f16 = p.dtype == ATTN_FP16;
+  const int nbq = ceil_div(p.q_len, 128), nbk = ceil_div(p.kv_len, 128);
+  const int S_pad = nbk * 128;
+  const unsigned BHq = static_cast<unsigned>(nu) * c->G;  // query heads of the range
+  const unsigned BHk = static_cast<unsigned>(nu);
+  // Every tensor is unit-major, so the range [u0, u0 + nu) is a contiguous slice of each.
+  const size_t qe = static_cast<size_t>(u0) * c->R * D;         // Q elements / codes before u0
+  const size_t ke = static_cast<size_t>(u0) * p.kv_len * D;     // K, V elements before u0
+  const uint16_t* qx = static_cast<const uint16_t*>(q) + (nbq > 0 ? qe : 0);
+  const uint16_t* kx = static_cast<const uint16_t*>(k) + (nbk > 0 ? ke : 0);
+  const uint16_t* vx = static_cast<const uint16_t*>(v) + (nbk > 0 ? ke : 0);
+  int8_t* qc = nbq > 0 ? qb->q + qe : nullptr;
+  float* qs = nbq > 0 ? qb->q_scale + static_cast<size_t>(u0) * c->G * nbq : nullptr;
+  int8_t* kc = nbk > 0 ? qb->k + ke : nullptr;
+  float* ks = nbk > 0 ? qb->k_scale + static_cast<size_t>(u0) * nbk : nullptr;
+  uint8_t* vt = nbk > 0 ? qb->v_t + static_cast<size_t>(u0) * D * S_pad : nullptr;
+  float* vs = nbk > 0 ? qb->v_scale + static_cast<size_t>(u0) * D : nullptr;
+  unsigned* vamax = nbk > 0 ? c->v_amax + static_cast<size_t>(u0) * D : nullptr;
+
+#define ATTN_QUANT_LAUNCH(DD, FF)                                                             \
+  do {                                                                                        \
+    static bool qk_attr = set_smem(quant_qk_kernel<DD, FF>, QuantQkCfg<DD>::kSmemBytes);      \
+    if (!qk_attr) return ATTN_ERR_CUDA;                                                       \
+    const int qk_ctas = QuantQkCfg<DD>::kCtasPerSm * c->num_sms;                              \
+    if (nbq > 0) {                                                                            \
+      const int tot = nbq * static_cast<int>(BHq);                                            \
+      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
+          qx, qc, qs, p.q_len, nbq, tot, c->err, c->debug);                                   \
+    }                                                                                         \
+    if (nbk > 0) {                                                                            \
+      const int tot = nbk * static_cast<int>(BHk);                                            \
+      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
+          kx, kc, ks, p.kv_len, nbk, tot, c->err, 0u);                                        \
+      v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(            \
+          vx, vamax, p.kv_len);                                                               \
+      static bool vq_attr = set_smem(v_quant_kernel<DD, FF>, VQuantCfg<DD>::kSmemBytes);      \
+      if (!vq_attr) return ATTN_ERR_CUDA;                                                     \
+      const int vq_ctas = std::min(tot, VQuantCfg<DD>::kCtasPerSm * c->num_sms);              \
+      v_quant_kernel<DD, FF><<<vq_ctas, 256, VQuantCfg<DD>::kSmemBytes, st>>>(                \
+          vx, vamax, vt, vs, p.kv_len, S_pad, nbk, tot, c->err);                              \
+    }                                                                                         \
+  } while (0)
+
+  if (nbk > 0 &&
+      cudaMemsetAsync(vamax, 0, static_cast<size_t>(nu) * D * 4, st) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (D == 128) {
+    if (f16) ATTN_QUANT_LAUNCH(128, true);
+    else ATTN_QUANT_LAUNCH(128, false);
+  } else {
+    if (f16) ATTN_QUANT_LAUNCH(64, true);
+    else ATTN_QUANT_LAUNCH(64, false);
+  }
+#undef ATTN_QUANT_LAUNCH
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Launches the forward on `st` for the units [u0, u0 + nu).  Pointers are those
+// of the whole problem, already validated.  The split-KV path keeps its partials
+// in the context's workspace, so it only runs on the whole problem at once.
+attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void* k,
+                          const void* v, const attn_qbufs* qb, void* o, float* lse,
+                          cudaStream_t st) {
+  if (c->split_path && (u0 != 0 || nu != c->units)) return ATTN_ERR_INVALID_ARG;
+  const attn_params& p = c->p;
+  const bool quant = p.precision == ATTN_INT8QK_FP8PV;
+  const int D = p.head_dim;
+  const bool f16 = p.dtype == ATTN_FP16;
+  const size_t rows = static_cast<size_t>(nu) * c->R;
+  if (rows == 0) return ATTN_OK;
+  // Every tensor is unit-major: move each base to unit u0 (the kernels index
+  // from their base, so a range of units is just a smaller problem).
+  const size_t qe = static_cast<size_t>(u0) * c->R * D;      // Q, O elements before u0
+  const size_t ke = static_cast<size_t>(u0) * p.kv_len * D;  // K, V elements before u0
+  o = static_cast<uint16_t*>(o) + qe;
+  if (lse) lse += static_cast<size_t>(u0) * c->R;
+  if (p.kv_len == 0) {  // every row sees no key
+    if (cudaMemsetAsync(o, 0, rows * D * 2, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (lse) fill_lse_kernel<<<ceil_div(rows, 256), 256, 0, st>>>(lse, rows);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  attn_qbufs qo{};
+  if (quant) {
+    const int nbq = ceil_div(p.q_len, 128), nbk = ceil_div(p.kv_len, 128);
+    qo.q = qb->q + qe;
+    qo.k = qb->k + ke;
+    qo.q_scale = qb->q_scale + static_cast<size_t>(u0) * c->G * nbq;
+    qo.k_scale = qb->k_scale + static_cast<size_t>(u0) * nbk;
+    qo.v_t = qb->v_t + static_cast<size_t>(u0) * D * (static_cast<size_t>(nbk) * 128);
+    qo.v_scale = qb->v_scale + static_cast<size_t>(u0) * D;
+    qb = &qo;
+  } else {
+    q = static_cast<const uint16_t*>(q) + qe;
+    k = static_cast<const uint16_t*>(k) + ke;
+    v = static_cast<const uint16_t*>(v) + ke;
+  }
+
+  // Tensor maps.  Q, O: [units][R][D]; K, V: [units][Skv][D]; V^T: [units][D][S_pad].
+  const CUtensorMapDataType t16 =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t R = c->R, Sk = p.kv_len, U = nu;
+  CUtensorMap tq, tk, tv, to;
+  bool ok = true;
+  if (quant) {
+    const CUtensorMapSwizzle sw8 =
+        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const uint64_t S_pad = static_cast<uint64_t>(ceil_div(p.kv_len, 128)) * 128;
+    ok &= make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, D, R, U, D, R * D, D, 128, sw8);
+    ok &= make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, D, Sk, U, D, Sk * D, D, 128, sw8);
+    ok &= make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->v_t, S_pad, D, U, S_pad, S_pad * D, 128,
+                   D, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok &= make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return ATTN_ERR_CUDA;
+
+  FwdArgs a{};
+  a.R = c->R;
+  a.Sq = p.q_len;
+  a.Skv = p.kv_len;
+  a.G = c->G;
+  a.units = nu;
+  a.row_tiles = c->row_tiles;
+  a.splits = c->splits;
+  a.tiles_per_split = c->tiles_per_split;
+  a.start_pos = p.start_pos;
+  a.causal = p.causal;
+  a.window_lo = p.window_lo;
+  a.scale_log2 = c->scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.o_part = c->o_part;
+  a.lse_part = c->lse_part;
+  if (quant) {
+    a.q_scale = qb->q_scale;
+    a.k_scale = qb->k_scale;
+    a.v_scale = qb->v_scale;
+  }
+  a.nblk_q = ceil_div(p.q_len, 128);
+  a.nblk_k = ceil_div(p.kv_len, 128);
+  a.err = c->err;
+  a.debug = c->debug;
+  const int grid = nu * c->row_tiles * (c->split_path ? c->splits : 1);
+
+  attn_status s;
+  if (D == 128) {
+    if (quant) s = f16 ? dispatch_fwd<128, true, true>(c, tq, tk, tv, to, a, grid, st)
+                       : dispatch_fwd<128, true, false>(c, tq, tk, tv, to, a, grid, st);
+    else s = f16 ? dispatch_fwd<128, false, true>(c, tq, tk, tv, to, a, grid, st)
+                 : dispatch_fwd<128, false, false>(c, tq, tk, tv, to, a, grid, st);
+  } else {
+    if (quant) s = f16 ? dispatch_fwd<64, true, true>(c, tq, tk, tv, to, a, grid, st)
+                       : dispatch_fwd<64, true, false>(c, tq, tk, tv, to, a, grid, st);
+    else s = f16 ? dispatch_fwd<64, false, true>(c, tq, tk, tv, to, a, grid, st)
+                 : dispatch_fwd<64, false, false>(c, tq, tk, tv, to, a, grid, st);
+  }
+  if (s != ATTN_OK) return s;
+  if (c->split_path) {
+    if (D == 128) s = f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
+    else s = f16 ? launch_merge<64, true>(c, o, lse, st) : launch_merge<64, false>(c, o, lse, st);
+  }
+  return s;
+}
+
+// Creates attn_forward_host's streams and events on the current device (all or none).
+attn_status ensure_pipeline(attn_ctx* c) {
+  if (c->pipe_ready) return ATTN_OK;
+  constexpr int kEvents = 1 + 4 + 2 * kMaxHostChunks;
+  cudaStream_t st[4] = {};
+  cudaEvent_t ev[kEvents] = {};
+  int ns = 0, ne = 0;
+  while (ns < 4 && cudaStreamCreateWithFlags(&st[ns], cudaStreamNonBlocking) == cudaSuccess) ++ns;
+  if (ns == 4)
+    while (ne < kEvents && cudaEventCreateWithFlags(&ev[ne], cudaEventDisableTiming) == cudaSuccess)
+      ++ne;
+  if (ns < 4 || ne < kEvents) {  // release what was created
+    for (int i = 0; i < ne; ++i) cudaEventDestroy(ev[i]);
+    for (int i = 0; i < ns; ++i) cudaStreamDestroy(st[i]);
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  for (int i = 0; i < 4; ++i) c->pipe[i] = st[i];
+  c->pev_start = ev[0];
+  for (int i = 0; i < 4; ++i) c->pev_join[i] = ev[1 + i];
+  for (int i = 0; i < kMaxHostChunks; ++i) {
+    c->pev_in[i] = ev[5 + i];
+    c->pev_done[i] = ev[5 + kMaxHostChunks + i];
+  }
+  c->pipe_ready = true;
+  return ATTN_OK;
+}
+
+// Number of unit ranges attn_forward_host cuts a problem into when the caller
+// leaves it to the library: about 8 MiB of inputs per range, at most
+// kMaxHostChunks.  The pipeline's fill and drain (the first range's inputs, the
+// last range's outputs) shrink with the range; a range still moves megabytes, so
+// the per-copy and per-launch costs (microseconds) stay small beside it.
+int default_host_chunks(const attn_ctx* c) {
+  const attn_params& p = c->p;
+  const double in_bytes = static_cast<double>(c->units) *
+                          (static_cast<double>(c->R) + 2.0 * p.kv_len) * p.head_dim * 2.0;
+  const int n = static_cast<int>(in_bytes / (8.0 * 1024 * 1024));
+  return std::max(1, std::min(n, kMaxHostChunks));
 }
 
 }  // namespace
@@ -263,6 +516,17 @@ void attn_destroy(attn_ctx* c) {
   if (!c) return;
   cudaDeviceSynchronize();
   cudaFree(c->ws);
+  if (c->pipe_ready) {
+    for (int i = 0; i < 4; ++i) {
+      cudaStreamDestroy(c->pipe[i]);
+      cudaEventDestroy(c->pev_join[i]);
+    }
+    for (int i = 0; i < kMaxHostChunks; ++i) {
+      cudaEventDestroy(c->pev_in[i]);
+      cudaEventDestroy(c->pev_done[i]);
+    }
+    cudaEventDestroy(c->pev_start);
+  }
   delete c;
 }
 
@@ -299,162 +563,87 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
                              const attn_qbufs* qb, void* stream) {
   if (!c || !qb) return ATTN_ERR_INVALID_ARG;
   if (c->p.precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
-  // Buffers of zero length may be NULL (an empty tensor has no storage).
   const bool need_q = c->p.q_len > 0, need_kv = c->p.kv_len > 0;
-  auto bad = [](const void* ptr, bool needed) {
-    return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));
-  };
-  if (bad(q, need_q) || bad(qb->q, need_q) || bad(qb->q_scale, need_q) || bad(k, need_kv) ||
-      bad(v, need_kv) || bad(qb->k, need_kv) || bad(qb->k_scale, need_kv) ||
-      bad(qb->v_t, need_kv) || bad(qb->v_scale, need_kv))
+  if (bad_ptr(q, need_q) || bad_ptr(k, need_kv) || bad_ptr(v, need_kv) || bad_qbufs(c->p, qb))
     return ATTN_ERR_INVALID_ARG;
-  const attn_params& p = c->p;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int D = p.head_dim;
-  const bool f16 = p.dtype == ATTN_FP16;
-  const int nbq = ceil_div(p.q_len, 128), nbk = ceil_div(p.kv_len, 128);
-  const int S_pad = nbk * 128;
-  const unsigned BHq = p.batch * p.n_q_heads;
-  const unsigned BHk = c->units;
-  auto X = [](const void* ptr) { return static_cast<const uint16_t*>(ptr); };
-
-#define ATTN_QUANT_LAUNCH(DD, FF)                                                              \
-  do {                                                                                         \
-    static bool qk_attr = set_smem(quant_qk_kernel<DD, FF>, QuantQkCfg<DD>::kSmemBytes);        \
-    if (!qk_attr) return ATTN_ERR_CUDA;                                                        \
-    const int qk_ctas = QuantQkCfg<DD>::kCtasPerSm * c->num_sms;                               \
-    if (nbq > 0) {                                                                             \
-      const int tot = nbq * static_cast<int>(BHq);                                             \
-      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
-          X(q), qb->q, qb->q_scale, p.q_len, nbq, tot, c->err, c->debug);                      \
-    }                                                                                          \
-    if (nbk > 0) {                                                                             \
-      const int tot = nbk * static_cast<int>(BHk);                                             \
-      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
-          X(k), qb->k, qb->k_scale, p.kv_len, nbk, tot, c->err, 0u);                           \
-      v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(           \
-          X(v), c->v_amax, p.kv_len);                                                          \
-      static bool vq_attr = set_smem(v_quant_kernel<DD, FF>, VQuantCfg<DD>::kSmemBytes);       \
-      if (!vq_attr) return ATTN_ERR_CUDA;                                                      \
-      const int vq_ctas = std::min(tot, VQuantCfg<DD>::kCtasPerSm * c->num_sms);               \
-      v_quant_kernel<DD, FF><<<vq_ctas, 256, VQuantCfg<DD>::kSmemBytes, st>>>(                 \
-          X(v), c->v_amax, qb->v_t, qb->v_scale, p.kv_len, S_pad, nbk, tot, c->err);           \
-    }                                                                                          \
-  } while (0)
-
-  if (nbk > 0 &&
-      cudaMemsetAsync(c->v_amax, 0, static_cast<size_t>(c->units) * D * 4, st) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  if (D == 128) {
-    if (f16) ATTN_QUANT_LAUNCH(128, true);
-    else ATTN_QUANT_LAUNCH(128, false);
-  } else {
-    if (f16) ATTN_QUANT_LAUNCH(64, true);
-    else ATTN_QUANT_LAUNCH(64, false);
-  }
-#undef ATTN_QUANT_LAUNCH
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return quantize_units(c, 0, c->units, q, k, v, qb, static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* v,
                          const attn_qbufs* qb, void* o, float* lse, void* stream) {
   if (!c) return ATTN_ERR_INVALID_ARG;
+  const attn_status s = check_forward_buffers(c, q, k, v, qb, o, lse);
+  if (s != ATTN_OK) return s;
+  return forward_units(c, 0, c->units, q, k, v, qb, o, lse, static_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_host,
+                              const void* v_host, void* o_host, float* lse_host, void* q_dev,
+                              void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                              const attn_qbufs* qb, int chunks, void* stream) {
+  if (!c || chunks < 0 || chunks > kMaxHostChunks) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
   const bool quant = p.precision == ATTN_INT8QK_FP8PV;
-  // Buffers of zero length may be NULL (an empty tensor has no storage).
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
-  auto bad = [](const void* ptr, bool needed) {
-    return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));
-  };
-  if (bad(o, need_q) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
-  if (quant) {
-    if (!qb) return ATTN_ERR_INVALID_ARG;
-    if (bad(qb->q, need_q) || bad(qb->q_scale, need_q) || bad(qb->k, need_kv) ||
-        bad(qb->k_scale, need_kv) || bad(qb->v_t, need_kv) || bad(qb->v_scale, need_kv))
-      return ATTN_ERR_INVALID_ARG;
-  } else {
-    if (qb) return ATTN_ERR_INVALID_ARG;
-    if (bad(q, need_q) || bad(k, need_kv) || bad(v, need_kv)) return ATTN_ERR_INVALID_ARG;
-  }
-
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int D = p.head_dim;
-  const bool f16 = p.dtype == ATTN_FP16;
-  const size_t rows = static_cast<size_t>(c->units) * c->R;
-  if (rows == 0) return ATTN_OK;
-  if (p.kv_len == 0) {  // every row sees no key
-    if (cudaMemsetAsync(o, 0, rows * D * 2, st) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (lse) fill_lse_kernel<<<ceil_div(rows, 256), 256, 0, st>>>(lse, rows);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-  }
-
-  // Tensor maps.  Q, O: [units][R][D]; K, V: [units][Skv][D]; V^T: [units][D][S_pad].
-  const CUtensorMapDataType t16 =
-      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const uint64_t R = c->R, Sk = p.kv_len, U = c->units;
-  CUtensorMap tq, tk, tv, to;
-  bool ok = true;
-  if (quant) {
-    const CUtensorMapSwizzle sw8 =
-        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    const uint64_t S_pad = static_cast<uint64_t>(ceil_div(p.kv_len, 128)) * 128;
-    ok &= make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, D, R, U, D, R * D, D, 128, sw8);
-    ok &= make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, D, Sk, U, D, Sk * D, D, 128, sw8);
-    ok &= make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->v_t, S_pad, D, U, S_pad, S_pad * D, 128,
-                   D, CU_TENSOR_MAP_SWIZZLE_128B);
-  } else {
-    ok &= make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  }
-  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return ATTN_ERR_CUDA;
-
-  FwdArgs a{};
-  a.R = c->R;
-  a.Sq = p.q_len;
-  a.Skv = p.kv_len;
-  a.G = c->G;
-  a.units = c->units;
-  a.row_tiles = c->row_tiles;
-  a.splits = c->splits;
-  a.tiles_per_split = c->tiles_per_split;
-  a.start_pos = p.start_pos;
-  a.causal = p.causal;
-  a.window_lo = p.window_lo;
-  a.scale_log2 = c->scale * 1.4426950408889634f;
-  a.lse = lse;
-  a.o_part = c->o_part;
-  a.lse_part = c->lse_part;
-  if (quant) {
-    a.q_scale = qb->q_scale;
-    a.k_scale = qb->k_scale;
-    a.v_scale = qb->v_scale;
-  }
-  a.nblk_q = ceil_div(p.q_len, 128);
-  a.nblk_k = ceil_div(p.kv_len, 128);
-  a.err = c->err;
-  a.debug = c->debug;
-  const int grid = c->units * c->row_tiles * (c->split_path ? c->splits : 1);
-
-  attn_status s;
-  if (D == 128) {
-    if (quant) s = f16 ? dispatch_fwd<128, true, true>(c, tq, tk, tv, to, a, grid, st)
-                       : dispatch_fwd<128, true, false>(c, tq, tk, tv, to, a, grid, st);
-    else s = f16 ? dispatch_fwd<128, false, true>(c, tq, tk, tv, to, a, grid, st)
-                 : dispatch_fwd<128, false, false>(c, tq, tk, tv, to, a, grid, st);
-  } else {
-    if (quant) s = f16 ? dispatch_fwd<64, true, true>(c, tq, tk, tv, to, a, grid, st)
-                       : dispatch_fwd<64, true, false>(c, tq, tk, tv, to, a, grid, st);
-    else s = f16 ? dispatch_fwd<64, false, true>(c, tq, tk, tv, to, a, grid, st)
-                 : dispatch_fwd<64, false, false>(c, tq, tk, tv, to, a, grid, st);
-  }
+  if ((need_q && (!q_host || !o_host)) || (need_kv && (!k_host || !v_host)))
+    return ATTN_ERR_INVALID_ARG;
+  if ((lse_host == nullptr) != (lse_dev == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (bad_ptr(q_dev, need_q) || bad_ptr(k_dev, need_kv) || bad_ptr(v_dev, need_kv) ||
+      bad_ptr(o_dev, need_q) || (lse_dev && !aligned16(lse_dev)))
+    return ATTN_ERR_INVALID_ARG;
+  if (quant ? bad_qbufs(p, qb) : qb != nullptr) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<size_t>(c->units) * c->R == 0) return ATTN_OK;
+  attn_status s = ensure_pipeline(c);
   if (s != ATTN_OK) return s;
-  if (c->split_path) {
-    if (D == 128) s = f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
-    else s = f16 ? launch_merge<64, true>(c, o, lse, st) : launch_merge<64, false>(c, o, lse, st);
+
+  const int U = c->units;
+  int n = chunks > 0 ? chunks : default_host_chunks(c);
+  n = c->split_path ? 1 : std::min(n, U);
+  const size_t qU = static_cast<size_t>(c->R) * p.head_dim * 2;   // Q or O bytes per unit
+  const size_t kU = static_cast<size_t>(p.kv_len) * p.head_dim * 2;  // K or V bytes per unit
+  const size_t lU = static_cast<size_t>(c->R) * 4;                // lse bytes per unit
+  auto copy = [](void* dst, const void* src, size_t off, size_t bytes, cudaMemcpyKind kind,
+                 cudaStream_t cs) {
+    if (bytes == 0) return true;
+    return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
+                           bytes, kind, cs) == cudaSuccess;
+  };
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t h2d = c->pipe[0], d2h = c->pipe[3];
+  bool ok = cudaEventRecord(c->pev_start, st) == cudaSuccess;
+  for (int i = 0; i < 4 && ok; ++i)
+    ok = cudaStreamWaitEvent(c->pipe[i], c->pev_start, 0) == cudaSuccess;
+  for (int i = 0; i < n && ok; ++i) {
+    const int u0 = static_cast<int>(static_cast<long long>(i) * U / n);
+    const int nu = static_cast<int>(static_cast<long long>(i + 1) * U / n) - u0;
+    cudaStream_t cs = c->pipe[1 + (i & 1)];
+    const cudaMemcpyKind in = cudaMemcpyHostToDevice, out = cudaMemcpyDeviceToHost;
+    ok = copy(q_dev, q_host, u0 * qU, nu * qU, in, h2d) &&
+         copy(k_dev, k_host, u0 * kU, nu * kU, in, h2d) &&
+         copy(v_dev, v_host, u0 * kU, nu * kU, in, h2d) &&
+         cudaEventRecord(c->pev_in[i], h2d) == cudaSuccess &&
+         cudaStreamWaitEvent(cs, c->pev_in[i], 0) == cudaSuccess;
+    if (!ok) break;
+    if (quant) {
+      s = quantize_units(c, u0, nu, q_dev, k_dev, v_dev, qb, cs);
+      if (s == ATTN_OK)
+        s = forward_units(c, u0, nu, nullptr, nullptr, nullptr, qb, o_dev, lse_dev, cs);
+    } else {
+      s = forward_units(c, u0, nu, q_dev, k_dev, v_dev, nullptr, o_dev, lse_dev, cs);
+    }
+    if (s != ATTN_OK) break;
+    ok = cudaEventRecord(c->pev_done[i], cs) == cudaSuccess &&
+         cudaStreamWaitEvent(d2h, c->pev_done[i], 0) == cudaSuccess &&
+         copy(o_host, o_dev, u0 * qU, nu * qU, out, d2h) &&
+         (!lse_dev || copy(lse_host, lse_dev, u0 * lU, nu * lU, out, d2h));
   }
-  return s;
+  // Join every pipeline stream back into the caller's stream, after an error too.
+  for (int i = 0; i < 4; ++i)
+    if (cudaEventRecord(c->pev_join[i], c->pipe[i]) != cudaSuccess ||
+        cudaStreamWaitEvent(st, c->pev_join[i], 0) != cudaSuccess)
+      ok = false;
+  if (s != ATTN_OK) return s;
+  return ok ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // extern "C"

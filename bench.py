@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=0,
+                    help="unit ranges of the end-to-end call (0: the library's choice)")
     ap.add_argument("--kv-heads", type=int, default=0,
                     help="run the workload with this many kv heads (same group size); for "
                          "profiling captures on a smaller case")
@@ -346,24 +348,20 @@ def measure(w: Workload, precision, steps, warmup, device):
                 launches=launches_per_step(att, precision))
 
 
-def measure_e2e(w: Workload, precision, m, steps, warmup):
-    """Same metric through the public API with host buffers: every step copies
-    Q, K, V from pinned host memory, runs the call, and copies O back."""
+def measure_e2e(w: Workload, precision, m, steps, warmup, chunks=0):
+    """Same metric through the public API with host buffers: every step is one
+    ``Attention.forward_host`` call (C ABI ``attn_forward_host``), which copies Q,
+    K, V from pinned host memory, runs the quantiser (quantised mode) and the
+    forward, and copies O back; the copies of each range of units overlap the
+    kernels of its neighbours.  ``chunks`` = 0 leaves the range count to the library."""
+    from attention_forward_flash_b200 import DeviceStaging
     att = m["att"]
     hq, hk, hv = (t.cpu().pin_memory() for t in (m["q"], m["k"], m["v"]))
     ho = torch.empty(m["out"].shape, dtype=m["out"].dtype).pin_memory()
-    dq, dk, dv, do = (torch.empty_like(t) for t in (m["q"], m["k"], m["v"], m["out"]))
+    staging = DeviceStaging(att.params, att.dtype, m["q"].device, precision == "quant", False)
 
     def step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        if precision == "quant":
-            qb = att.quantize(dq, dk, dv, qbufs=m["qb"])
-            att.forward(qbufs=qb, out=do)
-        else:
-            att.forward(dq, dk, dv, out=do)
-        ho.copy_(do, non_blocking=True)
+        att.forward_host(hq, hk, hv, out=ho, staging=staging, chunks=chunks)
 
     ms = time_steps(step, steps, warmup)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
@@ -439,10 +437,12 @@ def run_native(args):
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(3, min(args.steps, 10))
-    e2e_ms, h2d, d2h = measure_e2e(w, precision, m, e2e_steps, 2)
+    e2e_ms, h2d, d2h = measure_e2e(w, precision, m, e2e_steps, 3, args.e2e_chunks)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "call": "Attention.forward_host (attn_forward_host), pinned host buffers",
+           "unit_ranges": args.e2e_chunks or "library default"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,

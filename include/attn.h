@@ -123,6 +123,48 @@ attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const vo
 attn_status attn_forward(attn_ctx *c, const void *q, const void *k, const void *v,
                          const attn_qbufs *qb, void *o, float *lse, void *stream);
 
+/* End-to-end forward from host memory.
+ * No counterpart on the source pages: it is for callers whose Q, K and V sit in
+ * host memory.  It copies q, k and v from the host into the caller's device
+ * buffers, runs the forward (preceded by the quantiser in the quantised mode)
+ * and copies o, and lse if asked for, back to the host, overlapping the copies
+ * with the kernels.  The problem's units (one per batch entry and kv head, with
+ * that head's query heads) are independent and every tensor is unit-major, so
+ * the call cuts the units into `chunks` contiguous ranges.  For each range the
+ * host-to-device copies, the kernels and the device-to-host copies run in that
+ * order, on four streams that the context owns: while one range computes, the
+ * next range's inputs arrive and the previous range's outputs leave, each
+ * direction on its own copy engine.  The kernels of consecutive ranges go to
+ * two streams, so the last wave of one range overlaps the first of the next.
+ * Every result is bit-identical to attn_forward's (and attn_quantize_qk's) on
+ * the same inputs.  All of the work is ordered after the work already queued on
+ * `stream`, and work queued on `stream` afterwards waits for all of it:
+ * synchronise `stream` before reading o_host.
+ *
+ * Arguments: q_host, k_host, v_host (read) and o_host, lse_host (written) are
+ * host pointers in the layouts above.  lse_host may be NULL, and must be NULL
+ * exactly when lse_dev is.  Page-locked host memory (cudaHostAlloc or
+ * cudaHostRegister) lets the copies overlap the kernels; pageable memory gives
+ * the same results with the copies serialised by the driver.  q_dev, k_dev,
+ * v_dev, o_dev and lse_dev are device buffers of the full sizes, 16-byte
+ * aligned, which the call uses as staging (q_dev, k_dev and v_dev hold the
+ * 16-bit inputs in both modes).  qb: in the quantised mode, the quantiser's
+ * output buffers as for attn_forward (filled by this call); NULL in exact mode.
+ * chunks: 0 lets the library choose (about 8 MiB of inputs per range, at most
+ * 64 ranges); 1 to 64 asks for that many ranges; either is capped at the number
+ * of units.
+ * A problem on the split-KV path runs as one range.  Every buffer must stay
+ * valid until the work completes.  The first call creates the context's streams
+ * and events on the current device, which must be the context's.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL host pointer, NULL or misaligned device
+ * pointer, lse_host and lse_dev not both given or both NULL, qb presence not
+ * matching the mode, chunks out of range), ATTN_ERR_CUDA (stream or event
+ * creation, copy, tensor-map encode or launch failure). */
+attn_status attn_forward_host(attn_ctx *c, const void *q_host, const void *k_host,
+                              const void *v_host, void *o_host, float *lse_host, void *q_dev,
+                              void *k_dev, void *v_dev, void *o_dev, float *lse_dev,
+                              const attn_qbufs *qb, int chunks, void *stream);
+
 /* Synchronises `stream`, reads and clears the context's device error word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last call,
  * ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK. */
