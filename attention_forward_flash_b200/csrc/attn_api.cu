@@ -388,16 +388,31 @@ attn_status ensure_pipeline(attn_ctx* c) {
 }
 
 // Number of unit ranges attn_forward_host cuts a problem into when the caller
-// leaves it to the library: about 8 MiB of inputs per range, at most
+// leaves it to the library: about 24 MiB of inputs per range, at most
 // kMaxHostChunks.  The pipeline's fill and drain (the first range's inputs, the
-// last range's outputs) shrink with the range; a range still moves megabytes, so
-// the per-copy and per-launch costs (microseconds) stay small beside it.
+// last range's kernels and outputs) shrink with the range, but a range's kernel
+// cannot finish faster than its longest CTA, which sits on the pipeline's
+// critical path once per range.  On a PCIe 5.0 x16 host both the 1 x 40 x
+// 32760 x 128 MHA problem (40 ranges) and the 4 x 32/8 x 8192 x 128 causal GQA
+// one (16 ranges) ran fastest near this size.
 int default_host_chunks(const attn_ctx* c) {
   const attn_params& p = c->p;
   const double in_bytes = static_cast<double>(c->units) *
                           (static_cast<double>(c->R) + 2.0 * p.kv_len) * p.head_dim * 2.0;
-  const int n = static_cast<int>(in_bytes / (8.0 * 1024 * 1024));
+  const int n = static_cast<int>(in_bytes / (24.0 * 1024 * 1024) + 0.5);
   return std::max(1, std::min(n, kMaxHostChunks));
+}
+
+// Size of the pieces attn_forward_host copies O back in.  Host-to-device and
+// device-to-host copies share the PCIe link unevenly: measured on a PCIe 5.0 x16
+// host, with the outputs copied back in 1 MiB pieces the inputs kept ~51 GB/s and
+// the outputs got ~23 GB/s; in 8 MiB pieces 49 and 40; as one large copy 37 and
+// 47.  The inputs are the larger stream, so the pieces are the smallest whose
+// rate still keeps up with the inputs at the problem's output/input byte ratio.
+size_t d2h_piece_bytes(size_t out_per_unit, size_t in_per_unit) {
+  const double ratio = static_cast<double>(out_per_unit) / static_cast<double>(in_per_unit);
+  const size_t mib = size_t(1) << 20;
+  return ratio <= 0.4 ? mib : ratio <= 0.6 ? 2 * mib : ratio <= 0.8 ? 4 * mib : 8 * mib;
 }
 
 }  // namespace
@@ -610,14 +625,34 @@ attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_hos
   };
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaStream_t h2d = c->pipe[0], d2h = c->pipe[3];
+  const size_t piece = d2h_piece_bytes(qU, qU + 2 * kU);
+  auto bounds = [&](int i, int* u0, int* nu) {
+    *u0 = static_cast<int>(static_cast<long long>(i) * U / n);
+    *nu = static_cast<int>(static_cast<long long>(i + 1) * U / n) - *u0;
+  };
+  // Range j's outputs go back once its kernels are done and range j+1's inputs
+  // are in, so that they never split the link with the input copy that the next
+  // kernels wait on.
+  auto copy_out = [&](int j) {
+    int u0, nu;
+    bounds(j, &u0, &nu);
+    if (cudaStreamWaitEvent(d2h, c->pev_done[j], 0) != cudaSuccess) return false;
+    if (j + 1 < n && cudaStreamWaitEvent(d2h, c->pev_in[j + 1], 0) != cudaSuccess) return false;
+    for (size_t off = 0; off < nu * qU; off += piece)
+      if (!copy(o_host, o_dev, u0 * qU + off, std::min(piece, nu * qU - off),
+                cudaMemcpyDeviceToHost, d2h))
+        return false;
+    return !lse_dev || copy(lse_host, lse_dev, u0 * lU, nu * lU, cudaMemcpyDeviceToHost, d2h);
+  };
   bool ok = cudaEventRecord(c->pev_start, st) == cudaSuccess;
   for (int i = 0; i < 4 && ok; ++i)
     ok = cudaStreamWaitEvent(c->pipe[i], c->pev_start, 0) == cudaSuccess;
+  int issued = 0;  // ranges whose kernels are queued
   for (int i = 0; i < n && ok; ++i) {
-    const int u0 = static_cast<int>(static_cast<long long>(i) * U / n);
-    const int nu = static_cast<int>(static_cast<long long>(i + 1) * U / n) - u0;
+    int u0, nu;
+    bounds(i, &u0, &nu);
     cudaStream_t cs = c->pipe[1 + (i & 1)];
-    const cudaMemcpyKind in = cudaMemcpyHostToDevice, out = cudaMemcpyDeviceToHost;
+    const cudaMemcpyKind in = cudaMemcpyHostToDevice;
     ok = copy(q_dev, q_host, u0 * qU, nu * qU, in, h2d) &&
          copy(k_dev, k_host, u0 * kU, nu * kU, in, h2d) &&
          copy(v_dev, v_host, u0 * kU, nu * kU, in, h2d) &&
@@ -632,11 +667,11 @@ attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_hos
       s = forward_units(c, u0, nu, q_dev, k_dev, v_dev, nullptr, o_dev, lse_dev, cs);
     }
     if (s != ATTN_OK) break;
-    ok = cudaEventRecord(c->pev_done[i], cs) == cudaSuccess &&
-         cudaStreamWaitEvent(d2h, c->pev_done[i], 0) == cudaSuccess &&
-         copy(o_host, o_dev, u0 * qU, nu * qU, out, d2h) &&
-         (!lse_dev || copy(lse_host, lse_dev, u0 * lU, nu * lU, out, d2h));
+    ok = cudaEventRecord(c->pev_done[i], cs) == cudaSuccess;
+    issued = i + 1;
+    if (ok && i > 0) ok = copy_out(i - 1);
   }
+  if (ok && s == ATTN_OK && issued == n) ok = copy_out(n - 1);
   // Join every pipeline stream back into the caller's stream, after an error too.
   for (int i = 0; i < 4; ++i)
     if (cudaEventRecord(c->pev_join[i], c->pipe[i]) != cudaSuccess ||

@@ -136,6 +136,9 @@ attn_status attn_forward(attn_ctx *c, const void *q, const void *k, const void *
  * next range's inputs arrive and the previous range's outputs leave, each
  * direction on its own copy engine.  The kernels of consecutive ranges go to
  * two streams, so the last wave of one range overlaps the first of the next.
+ * A range's outputs leave once the next range's inputs are in, in pieces of 1
+ * to 8 MiB sized from the problem's output/input byte ratio, so that the
+ * inputs, the larger stream, keep most of the link.
  * Every result is bit-identical to attn_forward's (and attn_quantize_qk's) on
  * the same inputs.  All of the work is ordered after the work already queued on
  * `stream`, and work queued on `stream` afterwards waits for all of it:
@@ -150,7 +153,7 @@ attn_status attn_forward(attn_ctx *c, const void *q, const void *k, const void *
  * aligned, which the call uses as staging (q_dev, k_dev and v_dev hold the
  * 16-bit inputs in both modes).  qb: in the quantised mode, the quantiser's
  * output buffers as for attn_forward (filled by this call); NULL in exact mode.
- * chunks: 0 lets the library choose (about 8 MiB of inputs per range, at most
+ * chunks: 0 lets the library choose (about 24 MiB of inputs per range, at most
  * 64 ranges); 1 to 64 asks for that many ranges; either is capped at the number
  * of units.
  * A problem on the split-KV path runs as one range.  Every buffer must stay
