@@ -221,6 +221,30 @@ def test_wait_timeout_is_reported_and_context_survives():
     check_exact(o.double().cpu().numpy(), ro)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_quantised_wait_timeout_is_reported_and_context_survives(D):
+    """The same test hook in the quantised mode, whose kernel hands P to the MMA
+    warp through shared memory and has waits of its own: the loader never loads
+    the second key tile, every wait ends, the timeout is reported, and the next
+    call is correct."""
+    from attention_forward_flash_b200 import _abi
+    w = Workload("timeout_q", 1, 2, 2, 512, 1024, D, "bf16", seed=9)
+    q, k, v = (t.cuda() for t in make_qkv(w))
+    att = Attention(1, 2, 2, 512, 1024, D, num_splits=1, precision="quant")
+    qb = att.quantize(q, k, v)
+    att.check_error()
+    _abi.attn_debug_set(att.ctx, 1)
+    att.forward(qbufs=qb)
+    with pytest.raises(_abi.AttnError) as e:
+        att.check_error()
+    assert e.value.status == _abi.ATTN_ERR_TIMEOUT
+    _abi.attn_debug_set(att.ctx, 0)
+    o = att.forward(qbufs=qb)
+    att.check_error()
+    ro, _ = oracle_for(w, *(t.cpu() for t in (q, k, v)))
+    assert rel_rmse(o.double().cpu().numpy(), ro) <= QUANT_RMSE
+
+
 def test_polynomial_exp2_against_cuda_exp2():
     """The FMA-pipe exponential used for part of the softmax against torch's
     float32 exp2 on the GPU: relative error below 1e-4 on [-125, 126]."""
