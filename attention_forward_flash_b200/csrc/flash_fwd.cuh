@@ -154,7 +154,7 @@ struct RowSums {
 // P = 2^(x * c - m) for one half (64 keys) of a 128-key row, written over S in
 // tensor memory as 16-bit pairs (exact) or E4M3 quads (quantised), and added to
 // the row sums.  `cm` = {c, c}, `mm` = {-m, -m}; in the quantised mode x holds
-// the integer scores offset by 1.5 * 2^23 (their float bit pattern), and mm
+// the int32 scores' bits (offset by 1.5 * 2^23 into a float here), and mm
 // already subtracts that offset times c.  POLY: one pair in POLY takes the FMA
 // pipe exponential (0: all on the MUFU).  LF: keep the float32 sum (exact mode;
 // the quantised mode always keeps it, it is its only sum).
@@ -164,12 +164,14 @@ __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 c
 #pragma unroll
   for (int ch = 2 * H; ch < 2 * H + 2; ++ch) {
     if constexpr (QUANT) {
+      // x holds the int32 scores' bits; adding 0x4B400000 gives 1.5 * 2^23 + s exactly
+      auto sc = [](float v) { return __uint_as_float(__float_as_uint(v) + 0x4B400000u); };
       uint32_t pk[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int e = 32 * ch + 4 * c;
-        const f32x2 t0 = ffma2(f32x2{x[e], x[e + 1]}, cm, mm);
-        const f32x2 t1 = ffma2(f32x2{x[e + 2], x[e + 3]}, cm, mm);
+        const f32x2 t0 = ffma2(f32x2{sc(x[e]), sc(x[e + 1])}, cm, mm);
+        const f32x2 t1 = ffma2(f32x2{sc(x[e + 2]), sc(x[e + 3])}, cm, mm);
         f32x2 p01, p23;
         if (POLY > 0 && ((2 * c) % (POLY > 0 ? POLY : 1)) == 0) {
           p01 = poly_ex2x2(t0);
@@ -555,6 +557,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       const float ksc = ksc_next;
       if constexpr (QUANT)
         if (j + 1 < n) ksc_next = ld_global_f32(ksrc + j + 1);
+      // raw score -> base-2 scaled score factor (quantised: kept positive so that
+      // masked -inf scores stay -inf for an all-zero block); known before S lands
+      const float cj =
+          QUANT ? __uint_as_float(__float_as_uint(fmaxf(qsc * ksc * a.scale_log2, 1e-30f)) & ~7u)
+                : a.scale_log2;
       ok = __all_sync(0xffffffffu, mbar_wait(s_ready(q), j & 1, abort_flag));
       if (!ok) { if (lane == 0) raise(); break; }
       tc_fence_after();
@@ -563,8 +570,27 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
           (kv0 < a.window_lo) || (kv0 + 128 > a.Skv) || (a.causal && kv0 + 127 > pos_min);
       // S is read in two 64-column halves: the second half's load overlaps the
       // masking and maximum of the first.  Row max: four chains of three-input maxima.
+      // Quantised: x keeps the int32 scores' bits, the row max runs on the integers
+      // (eight chains) and the float offset is added in the emit; a masked score is
+      // the bit pattern that the offset turns into -inf (below every real score).
+      constexpr uint32_t kMaskedBits = 0xFF800000u - 0x4B400000u;
+      const float masked = QUANT ? __uint_as_float(kMaskedBits) : -INFINITY;
       float x[128];
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      constexpr int kIntMin = -2147483647 - 1;
+      int mi[8] = {kIntMin, kIntMin, kIntMin, kIntMin, kIntMin, kIntMin, kIntMin, kIntMin};
+      auto row_max = [&](int c0) {
+#pragma unroll
+        for (int c = c0; c < c0 + 64; c += 8) {
+          if constexpr (QUANT) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mi[e] = max(mi[e], static_cast<int>(__float_as_uint(x[c + e])));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
+          }
+        }
+      };
       {
         uint32_t s0[32], s1[32];
         tmem_ld32(tS + 0, s0);
@@ -573,8 +599,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         tmem_ld_wait(s1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          x[c] = to_score(s0[c]);
-          x[32 + c] = to_score(s1[c]);
+          x[c] = __uint_as_float(s0[c]);
+          x[32 + c] = __uint_as_float(s1[c]);
         }
       }
       uint32_t s2[32], s3[32];
@@ -584,37 +610,33 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int kj = kv0 + c;
-          if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
+          if (kj < lo_r || kj > hi_r) x[c] = masked;
         }
       }
-#pragma unroll
-      for (int c = 0; c < 64; c += 8)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
+      row_max(0);
       tmem_ld_wait(s2);
       tmem_ld_wait(s3);
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        x[64 + c] = to_score(s2[c]);
-        x[96 + c] = to_score(s3[c]);
+        x[64 + c] = __uint_as_float(s2[c]);
+        x[96 + c] = __uint_as_float(s3[c]);
       }
       if (need_mask) {
 #pragma unroll
         for (int c = 64; c < 128; ++c) {
           const int kj = kv0 + c;
-          if (kj < lo_r || kj > hi_r) x[c] = -INFINITY;
+          if (kj < lo_r || kj > hi_r) x[c] = masked;
         }
       }
-#pragma unroll
-      for (int c = 64; c < 128; c += 8)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
-      // raw score -> base-2 scaled score factor (quantised: kept positive so that
-      // masked -inf scores stay -inf for an all-zero block)
-      const float cj =
-          QUANT ? __uint_as_float(__float_as_uint(fmaxf(qsc * ksc * a.scale_log2, 1e-30f)) & ~7u)
-                : a.scale_log2;
-      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) - kMagic;  // exact
+      row_max(64);
+      float mx;
+      if constexpr (QUANT) {
+        int mr = max(max(max(mi[0], mi[1]), max(mi[2], mi[3])),
+                     max(max(mi[4], mi[5]), max(mi[6], mi[7])));
+        mx = to_score(static_cast<uint32_t>(mr)) - kMagic;  // exact; -inf if all masked
+      } else {
+        mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+      }
       const float m_tile = mx * cj;  // cj > 0; -inf stays -inf
       const float m_prev = m_used;
       const float m_new = fmaxf(m_prev, m_tile);
