@@ -157,10 +157,13 @@ struct RowSums {
 // the int32 scores' bits (offset by 1.5 * 2^23 into a float here), and mm
 // already subtracts that offset times c.  POLY: one pair in POLY takes the FMA
 // pipe exponential (0: all on the MUFU).  LF: keep the float32 sum (exact mode;
-// the quantised mode always keeps it, it is its only sum).
-template <bool F16, bool QUANT, int POLY, bool LF, int H>
+// the quantised mode always keeps it, it is its only sum).  `mid` runs in the
+// second half once its first 32 keys are computed and before they are stored:
+// the hand-off of the first half waits for that half's stores to complete, and
+// by then they have.
+template <bool F16, bool QUANT, int POLY, bool LF, int H, typename Mid>
 __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 cm, f32x2 mm,
-                                                  uint32_t tS, RowSums& rs) {
+                                                  uint32_t tS, RowSums& rs, Mid&& mid) {
 #pragma unroll
   for (int ch = 2 * H; ch < 2 * H + 2; ++ch) {
     if constexpr (QUANT) {
@@ -186,6 +189,7 @@ __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 c
         rs.f0 = fadd2(rs.f0, p01);
         rs.f1 = fadd2(rs.f1, p23);
       }
+      if (ch == 2) mid();
       tmem_st8(tS + 8 * ch, pk);
     } else {
       uint32_t pk[16];
@@ -212,6 +216,7 @@ __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 c
             rs.f0 = fadd2(rs.f0, p);
         }
       }
+      if (ch == 2) mid();
       tmem_st16(tS + 16 * ch, pk);
     }
   }
@@ -666,14 +671,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       const float kq = QUANT ? fmaf(kMagic, cj, mb) : mb;  // quantised: offset folded in
       const f32x2 cm{cj, cj}, mm{-kq, -kq};
       RowSums rs{{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f}, {0.0f, 0.0f}};
+      auto none = [] {};
+      auto first_half_done = [&] { p_half_done(0); };
       if (need_mask) {
-        softmax_emit_half<F16, QUANT, 0, LF, 0>(x, cm, mm, tS, rs);
-        p_half_done(0);
-        softmax_emit_half<F16, QUANT, 0, LF, 1>(x, cm, mm, tS, rs);
+        softmax_emit_half<F16, QUANT, 0, LF, 0>(x, cm, mm, tS, rs, none);
+        softmax_emit_half<F16, QUANT, 0, LF, 1>(x, cm, mm, tS, rs, first_half_done);
       } else {
-        softmax_emit_half<F16, QUANT, kPoly, LF, 0>(x, cm, mm, tS, rs);
-        p_half_done(0);
-        softmax_emit_half<F16, QUANT, kPoly, LF, 1>(x, cm, mm, tS, rs);
+        softmax_emit_half<F16, QUANT, kPoly, LF, 0>(x, cm, mm, tS, rs, none);
+        softmax_emit_half<F16, QUANT, kPoly, LF, 1>(x, cm, mm, tS, rs, first_half_done);
       }
       p_half_done(1);
       const float fsum = (rs.f0.x + rs.f0.y) + (rs.f1.x + rs.f1.y);
