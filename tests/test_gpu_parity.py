@@ -264,3 +264,46 @@ def test_polynomial_exp2_against_cuda_exp2():
     _abi.attn_debug_exp2(z.data_ptr(), w.data_ptr(), 2, torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert torch.all(w == y[-1])  # clamped to the value at -125
+
+
+# Long contexts: one CTA runs 1024 key tiles (131072 keys) in the single-pass
+# kernel (forced: the library would split a single unit of 1024 rows), and decode
+# problems with 32768 keys reach the library's split count for a few rows (merge
+# over ~37 partials, most of them empty under the window).
+LONG = [
+    ("long_prefill", Workload("long_prefill", 1, 2, 1, 512, 131072, 128, "bf16",
+                              modes=("exact", "quant"), seed=5101, oracle_rows=64)),
+    ("long_decode", Workload("long_decode", 1, 16, 8, 4, 32768, 128, "fp16", causal=True,
+                             start_pos=32764, seed=5102)),
+    ("long_decode_window", Workload("long_decode_window", 1, 16, 8, 1, 32768, 128, "fp16",
+                                    causal=True, start_pos=32767, window_lo=28672, seed=5103)),
+]
+
+
+@pytest.mark.parametrize("name,w", LONG, ids=[n for n, _ in LONG])
+def test_long_context_exact(name, w):
+    q, k, v = make_qkv(w)
+    o, lse, att = run_gpu(w, q, k, v, num_splits=1 if name == "long_prefill" else 0)
+    rows = sample_rows(w).numpy()
+    ro, rl = oracle_for(w, q, k, v, rows=rows)
+    check_exact(o[:, :, rows], ro, name)
+    check_lse(lse[:, :, rows], rl, name)
+    if name.startswith("long_decode"):
+        assert att.num_splits > 8
+    else:
+        assert att.num_splits == 1
+
+
+# The quantised mode on both kernels: the single-pass one (forced) and the
+# split-KV one with its merge (the library's choice for these shapes).
+@pytest.mark.parametrize("name,num_splits", [("long_prefill", 1), ("long_prefill", 0),
+                                             ("long_decode", 0)])
+def test_long_context_quant(name, num_splits):
+    w = dict(LONG)[name]
+    q, k, v = make_qkv(w)
+    o, _, att = run_gpu(w, q, k, v, precision="quant", num_splits=num_splits)
+    assert (att.num_splits == 1) == (num_splits == 1)
+    rows = sample_rows(w).numpy()
+    ro, _ = oracle_for(w, q, k, v, rows=rows)
+    e = rel_rmse(o[:, :, rows], ro)
+    assert e <= QUANT_RMSE, f"{name}: quantised rel_rmse {e:.3e}"
