@@ -19,6 +19,15 @@ using namespace attn;
 
 namespace {
 constexpr int kMaxHostChunks = 64;  // ranges of units of one attn_forward_host call
+
+// Tensor maps of one launch, kept with the base pointers and unit count they were
+// encoded for: a later launch on the same buffers reuses them.
+struct MapCache {
+  bool valid;
+  const void* key[4];  // Q, K, V (or their INT8/E4M3 codes) and O of the launch
+  int nu;
+  CUtensorMap tq, tk, tv, to;
+};
 }  // namespace
 
 struct attn_ctx {
@@ -47,6 +56,9 @@ struct attn_ctx {
   cudaStream_t pipe[4];
   cudaEvent_t pev_start, pev_join[4];
   cudaEvent_t pev_in[kMaxHostChunks], pev_done[kMaxHostChunks];
+  // Encoded tensor maps: slot 0 for attn_forward, slot 1 + i for range i of
+  // attn_forward_host.
+  MapCache maps[1 + kMaxHostChunks];
 };
 
 namespace {
@@ -255,7 +267,7 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
 // in the context's workspace, so it only runs on the whole problem at once.
 attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void* k,
                           const void* v, const attn_qbufs* qb, void* o, float* lse,
-                          cudaStream_t st) {
+                          cudaStream_t st, int slot) {
   if (c->split_path && (u0 != 0 || nu != c->units)) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
   const bool quant = p.precision == ATTN_INT8QK_FP8PV;
@@ -294,9 +306,19 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
   const CUtensorMapDataType t16 =
       f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t R = c->R, Sk = p.kv_len, U = nu;
-  CUtensorMap tq, tk, tv, to;
+  MapCache& mc = c->maps[slot];
+  const void* key[4] = {quant ? static_cast<const void*>(qb->q) : q,
+                        quant ? static_cast<const void*>(qb->k) : k,
+                        quant ? static_cast<const void*>(qb->v_t) : v, o};
+  const bool hit = mc.valid && mc.nu == nu && mc.key[0] == key[0] && mc.key[1] == key[1] &&
+                   mc.key[2] == key[2] && mc.key[3] == key[3];
+  CUtensorMap& tq = mc.tq;
+  CUtensorMap& tk = mc.tk;
+  CUtensorMap& tv = mc.tv;
+  CUtensorMap& to = mc.to;
   bool ok = true;
-  if (quant) {
+  if (hit) {
+  } else if (quant) {
     const CUtensorMapSwizzle sw8 =
         D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const uint64_t S_pad = static_cast<uint64_t>(ceil_div(p.kv_len, 128)) * 128;
@@ -309,7 +331,12 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
     ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   }
-  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!hit) {
+    ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    mc.valid = ok;
+    mc.nu = nu;
+    for (int i = 0; i < 4; ++i) mc.key[i] = key[i];
+  }
   if (!ok) return ATTN_ERR_CUDA;
 
   FwdArgs a{};
@@ -589,7 +616,8 @@ attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* 
   if (!c) return ATTN_ERR_INVALID_ARG;
   const attn_status s = check_forward_buffers(c, q, k, v, qb, o, lse);
   if (s != ATTN_OK) return s;
-  return forward_units(c, 0, c->units, q, k, v, qb, o, lse, static_cast<cudaStream_t>(stream));
+  return forward_units(c, 0, c->units, q, k, v, qb, o, lse, static_cast<cudaStream_t>(stream),
+                       0);
 }
 
 attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_host,
@@ -662,9 +690,9 @@ attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_hos
     if (quant) {
       s = quantize_units(c, u0, nu, q_dev, k_dev, v_dev, qb, cs);
       if (s == ATTN_OK)
-        s = forward_units(c, u0, nu, nullptr, nullptr, nullptr, qb, o_dev, lse_dev, cs);
+        s = forward_units(c, u0, nu, nullptr, nullptr, nullptr, qb, o_dev, lse_dev, cs, 1 + i);
     } else {
-      s = forward_units(c, u0, nu, q_dev, k_dev, v_dev, nullptr, o_dev, lse_dev, cs);
+      s = forward_units(c, u0, nu, q_dev, k_dev, v_dev, nullptr, o_dev, lse_dev, cs, 1 + i);
     }
     if (s != ATTN_OK) break;
     ok = cudaEventRecord(c->pev_done[i], cs) == cudaSuccess;

@@ -435,6 +435,22 @@ def run_native(args):
                 (" x2 for INT8/FP8" if precision == "quant" else ""),
                 "kernel": "flash_fwd_kernel", "kernel_ms": ms_kernel}
 
+    # ---- the quantisers on their own (quantised mode): an HBM-bound pass whose
+    # algorithmic bytes are Q and K read once, V read twice (channel maxima, then
+    # the codes), and the codes and scales written once
+    quantiser = None
+    if precision == "quant":
+        ms_q = time_steps(lambda: att.quantize(q, k, v, qbufs=qb), args.steps, 2)
+        q_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, v))
+        q_bytes += sum(t.numel() * t.element_size()
+                       for t in (qb.q, qb.k, qb.q_scale, qb.k_scale, qb.v_t, qb.v_scale))
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        gbs = q_bytes / (ms_q * 1e-3) / 1e9
+        quantiser = {"bound": "hbm", "ms": ms_q, "bytes": q_bytes, "achieved": gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": gbs / hbm,
+                     "kernels": "quant_qk_kernel (Q, K), v_amax_kernel, v_quant_kernel"}
+    att.check_error()
+
     # ---- end to end through the public API with host buffers
     e2e_steps = max(3, min(args.steps, 10))
     e2e_ms, h2d, d2h = measure_e2e(w, precision, m, e2e_steps, 3, args.e2e_chunks)
@@ -453,6 +469,7 @@ def run_native(args):
         "config": workload_config(w, precision),
         "pct_of_peak": 100.0 * achieved / peak,
         "roofline": roofline, "e2e": e2e,
+        **({"quantiser": quantiser} if quantiser else {}),
         "gpu_launches": m["launches"] * args.steps,
         "clocks": clocks.summary(),
     }
@@ -492,7 +509,9 @@ def run_native(args):
         flops_s, dt, desc, threads = oracle_sample_time(w, target_s=12.0)
         line["cpu_baseline"] = {"value": flops_s / dt / 1e12, "unit": "TFLOP/s",
                                 "cores": threads, "kind": "oracle", "sample": desc,
-                                "seconds": dt}
+                                "seconds": dt,
+                                # the whole call at the sample's rate (linear in rows)
+                                "extrapolated_full_call_s": flops / (flops_s / dt)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
