@@ -32,6 +32,13 @@ Readings taken where the pages are silent (each is listed in the design doc):
   it sees keys ``j <= start_pos + i``;
 * ``window_lo`` is an inclusive absolute lower bound on the key index, applied
   with or without ``causal``;
+* ``window_size`` W > 0 adds a per-row sliding window: row ``i`` (position
+  ``p = start_pos + i``) sees keys ``j >= p - W + 1``, i.e. the last W positions
+  up to its own when causal.  The pages name only a window lower bound (the
+  "Summary" above) and position/window test cases ("round 21 track b -- qsa2",
+  section "experiment contract"); the per-row form is the usual sliding window
+  read from that lower bound, applied together with ``window_lo`` (the larger
+  bound wins);
 * a row that sees no key returns O = 0 and lse = -inf;
 * ``scale`` defaults to ``1/sqrt(D)``.
 """
@@ -43,13 +50,16 @@ import math
 import numpy as np
 
 
-def visible_range(i, *, kv_len, start_pos=0, causal=False, window_lo=0):
+def visible_range(i, *, kv_len, start_pos=0, causal=False, window_lo=0, window_size=0):
     """Inclusive key range ``[lo, hi]`` seen by query row ``i`` (empty if lo > hi).
 
     Row ``i`` is at absolute position ``start_pos + i`` (the ``pos`` of
     "Performance evidence", page "perf(metal): widen four-row flash KV tiles").
+    ``window_size`` W > 0 keeps only keys ``j >= start_pos + i - W + 1``.
     """
     lo = max(int(window_lo), 0)
+    if window_size > 0:
+        lo = max(lo, int(start_pos) + int(i) - int(window_size) + 1)
     hi = kv_len - 1
     if causal:
         hi = min(hi, int(start_pos) + int(i))
@@ -67,13 +77,13 @@ def _as_f64(x):
 
 
 def attention_f64(q, k, v, *, scale=None, causal=False, start_pos=0, window_lo=0,
-                  rows=None, return_probs=False):
+                  window_size=0, rows=None, return_probs=False):
     """Attention forward in float64.
 
     Arguments
       q : [B, Hq, Sq, D];  k, v : [B, Hkv, Skv, D]  (any float dtype; widened exactly)
       scale : multiplier of Q K^T (default 1/sqrt(D))
-      causal, start_pos, window_lo : mask parameters, see ``visible_range``
+      causal, start_pos, window_lo, window_size : mask parameters, see ``visible_range``
       rows : optional 1-D index array of query rows to evaluate (same rows for
              every (b, hq)); default all rows
       return_probs : also return the softmax matrix P [B, Hq, len(rows), Skv]
@@ -101,10 +111,15 @@ def attention_f64(q, k, v, *, scale=None, causal=False, start_pos=0, window_lo=0
     hi = np.empty(R, dtype=np.int64)
     for n, i in enumerate(rows):
         lo[n], hi[n] = visible_range(int(i), kv_len=Skv, start_pos=start_pos,
-                                     causal=causal, window_lo=window_lo)
+                                     causal=causal, window_lo=window_lo,
+                                     window_size=window_size)
     j = np.arange(Skv)
     vis = (j[None, :] >= lo[:, None]) & (j[None, :] <= hi[:, None])  # [R, Skv]
     any_vis = vis.any(axis=1)
+    # O sums over each row's visible keys only.  P is 0 at masked keys, and a key
+    # that no evaluated row sees is also removed from V, so that a non-finite value
+    # there (0 * inf or 0 * nan) cannot reach the product.
+    seen = vis.any(axis=0)                                            # [Skv]
 
     out = np.zeros((B, Hq, R, D), dtype=np.float64)
     lse = np.full((B, Hq, R), -np.inf, dtype=np.float64)
@@ -123,7 +138,7 @@ def attention_f64(q, k, v, *, scale=None, causal=False, start_pos=0, window_lo=0
             l = p.sum(axis=1)
             l_safe = np.where(any_vis, l, 1.0)
             p = p / l_safe[:, None]                         # softmax rows
-            out[b, hq] = p @ v[b, hk]
+            out[b, hq] = p @ np.where(seen[:, None], v[b, hk], 0.0)
             lse[b, hq] = np.where(any_vis, m_safe + np.log(l_safe), -np.inf)
             if return_probs:
                 probs[b, hq] = p

@@ -53,7 +53,7 @@ def test_hand_worked_example():
         np.testing.assert_allclose(lse[0, 0], want_lse, rtol=1e-15, atol=1e-15, err_msg=case["name"])
 
 
-def _brute(q, k, v, scale, causal, start_pos, window_lo):
+def _brute(q, k, v, scale, causal, start_pos, window_lo, window_size=0):
     """Independent restatement: explicit loops, softmax as exp(s)/sum(exp(s))."""
     B, Hq, Sq, D = q.shape
     Hkv, Skv = k.shape[1], k.shape[2]
@@ -66,7 +66,8 @@ def _brute(q, k, v, scale, causal, start_pos, window_lo):
             for i in range(Sq):
                 pos = start_pos + i
                 keys = [j for j in range(Skv)
-                        if j >= window_lo and (not causal or j <= pos)]
+                        if j >= window_lo and (not causal or j <= pos)
+                        and (window_size == 0 or pos - j < window_size)]
                 if not keys:
                     continue
                 e = {}
@@ -82,7 +83,7 @@ def _brute(q, k, v, scale, causal, start_pos, window_lo):
     return o, lse
 
 
-@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("seed", range(10))
 def test_brute_force_tiny(seed):
     rng = np.random.default_rng(seed)
     B = int(rng.integers(1, 3))
@@ -95,13 +96,14 @@ def test_brute_force_tiny(seed):
     causal = bool(seed % 2)
     start_pos = int(rng.integers(0, 5))
     window_lo = int(rng.integers(0, 3))
+    window_size = int(rng.integers(0, 4)) if seed >= 2 else 0
     scale = float(rng.uniform(0.2, 1.5))
     q = rng.standard_normal((B, Hq, Sq, D))
     k = rng.standard_normal((B, Hkv, Skv, D))
     v = rng.standard_normal((B, Hkv, Skv, D))
     o, lse = attention_f64(q, k, v, scale=scale, causal=causal, start_pos=start_pos,
-                           window_lo=window_lo)
-    bo, blse = _brute(q, k, v, scale, causal, start_pos, window_lo)
+                           window_lo=window_lo, window_size=window_size)
+    bo, blse = _brute(q, k, v, scale, causal, start_pos, window_lo, window_size)
     np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(lse, blse, rtol=1e-12, atol=1e-12)
 
@@ -244,3 +246,63 @@ def test_no_keys_at_all():
     k = np.zeros((1, 1, 0, 4))
     o, lse = attention_f64(q, k, k, causal=True)
     assert o.shape == (1, 2, 3, 4) and np.all(o == 0) and np.all(lse == -math.inf)
+
+
+# Per-row sliding window (window_size W): row i at position p sees keys
+# max(window_lo, p - W + 1) .. p (causal).
+@pytest.mark.parametrize("W,start_pos,window_lo", [(1, 0, 0), (3, 5, 0), (16, 40, 0), (7, 30, 33),
+                                                   (64, 0, 0)])
+def test_sliding_window_against_torch_sdpa(W, start_pos, window_lo):
+    g = torch.Generator().manual_seed(23)
+    B, Hq, Hkv, Sq, Skv, D = 1, 4, 2, 11, 57, 8
+    q = torch.randn(B, Hq, Sq, D, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, Skv, D, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, Skv, D, generator=g, dtype=torch.float64)
+    mask = torch.zeros(Sq, Skv, dtype=torch.bool)
+    for i in range(Sq):
+        p = start_pos + i
+        for j in range(Skv):
+            mask[i, j] = j >= window_lo and j <= p and p - j < W
+    ok_rows = mask.any(dim=1)
+    G = Hq // Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(G, dim=1), v.repeat_interleave(G, dim=1), attn_mask=mask)
+    o, lse = attention_f64(q, k, v, causal=True, start_pos=start_pos, window_lo=window_lo,
+                           window_size=W)
+    np.testing.assert_allclose(o[:, :, ok_rows.numpy()], ref[:, :, ok_rows].numpy(),
+                               rtol=1e-12, atol=1e-12)
+    assert np.all(o[:, :, ~ok_rows.numpy()] == 0.0)
+    assert np.all(lse[:, :, ~ok_rows.numpy()] == -math.inf)
+
+
+def test_window_of_one_returns_own_value_row():
+    """W = 1, causal: row i sees only key start_pos + i, so O is that row of V and
+    lse is its scaled score."""
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((1, 2, 6, 8))
+    k = rng.standard_normal((1, 2, 20, 8))
+    v = rng.standard_normal((1, 2, 20, 8))
+    o, lse = attention_f64(q, k, v, causal=True, start_pos=9, window_size=1)
+    np.testing.assert_allclose(o[0], v[0, :, 9:15], atol=1e-15)
+    s = np.einsum("hid,hid->hi", q[0], k[0, :, 9:15]) / math.sqrt(8)
+    np.testing.assert_allclose(lse[0], s, atol=1e-13)
+
+
+def test_keys_outside_the_sliding_window_have_no_influence():
+    rng = np.random.default_rng(32)
+    q = rng.standard_normal((1, 1, 5, 8))
+    k = rng.standard_normal((1, 1, 64, 8))
+    v = rng.standard_normal((1, 1, 64, 8))
+    kw = dict(causal=True, start_pos=50, window_size=10)   # rows see 41..50 .. 45..54
+    o1, l1 = attention_f64(q, k, v, **kw)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, :41] = np.nan
+    v2[:, :, :41] = 1e30
+    k2[:, :, 55:] = 1e30
+    v2[:, :, 55:] = np.nan
+    o2, l2 = attention_f64(q, k2, v2, **kw)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    # a window at least as long as every row's causal range changes nothing
+    o3, l3 = attention_f64(q, k, v, causal=True, start_pos=50, window_size=55)
+    o4, l4 = attention_f64(q, k, v, causal=True, start_pos=50)
+    assert np.array_equal(o3, o4) and np.array_equal(l3, l4)
