@@ -26,7 +26,7 @@ class AttnParams(ctypes.Structure):
                 ("q_len", ctypes.c_int), ("kv_len", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("start_pos", ctypes.c_int), ("causal", ctypes.c_int), ("window_lo", ctypes.c_int),
                 ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("precision", ctypes.c_int),
-                ("num_splits", ctypes.c_int)]
+                ("num_splits", ctypes.c_int), ("window_size", ctypes.c_int)]
 
 
 class AttnQBufs(ctypes.Structure):

@@ -59,7 +59,7 @@ class Attention:
 
     def __init__(self, batch, n_q_heads, n_kv_heads, q_len, kv_len, head_dim, *,
                  dtype=torch.bfloat16, causal=False, start_pos=0, window_lo=0, scale=0.0,
-                 precision="exact", num_splits=0):
+                 precision="exact", num_splits=0, window_size=0):
         if dtype not in (torch.bfloat16, torch.float16):
             raise ValueError("dtype must be torch.bfloat16 or torch.float16")
         self.dtype = dtype
@@ -67,7 +67,7 @@ class Attention:
         self.params = AttnParams(batch, n_q_heads, n_kv_heads, q_len, kv_len, head_dim, start_pos,
                                  int(bool(causal)), window_lo, float(scale),
                                  ATTN_FP16 if dtype == torch.float16 else ATTN_BF16,
-                                 _PRECISIONS[precision], num_splits)
+                                 _PRECISIONS[precision], num_splits, window_size)
         self.ctx = _abi.attn_create(self.params)
 
     @property

@@ -103,27 +103,39 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF = SPLIT>
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN>
 attn_status launch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                        cudaStream_t st) {
   using Cfg = FwdCfg<D, NQT, QUANT, SPLIT>;
-  auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF>;
+  auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN>;
   static bool attr_ok = set_smem(kern, Cfg::kSmemBytes);
   if (!attr_ok) return ATTN_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+template <int D, bool QUANT, bool F16, bool WIN>
+attn_status dispatch_win(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
+                         const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+                         cudaStream_t st) {
+  if (c->split_path)
+    return launch_fwd<D, 1, QUANT, F16, true, true, WIN>(c, tq, tk, tv, to, a, grid, st);
+  // Exact mode keeps a second (float32) row sum only when the caller asks for lse
+  // (the quantised mode's only sum is the float32 one).
+  if constexpr (!QUANT) {
+    if (a.lse != nullptr)
+      return launch_fwd<D, 2, QUANT, F16, false, true, WIN>(c, tq, tk, tv, to, a, grid, st);
+  }
+  return launch_fwd<D, 2, QUANT, F16, false, false, WIN>(c, tq, tk, tv, to, a, grid, st);
+}
+
 template <int D, bool QUANT, bool F16>
 attn_status dispatch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                          cudaStream_t st) {
-  if (c->split_path) return launch_fwd<D, 1, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
-  // Exact mode keeps a second (float32) row sum only when the caller asks for lse.
-  if (!QUANT && a.lse != nullptr)
-    return launch_fwd<D, 2, QUANT, F16, false, true>(c, tq, tk, tv, to, a, grid, st);
-  return launch_fwd<D, 2, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
+  if (a.window_size > 0) return dispatch_win<D, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
+  return dispatch_win<D, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
 }
 
 // The merge is a programmatic dependent launch of the split kernel: its launch
@@ -156,7 +168,8 @@ attn_status validate(const attn_params* p) {
   if (!p) return ATTN_ERR_INVALID_ARG;
   if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1) return ATTN_ERR_INVALID_ARG;
   if (p->n_q_heads % p->n_kv_heads != 0) return ATTN_ERR_INVALID_ARG;
-  if (p->q_len < 0 || p->kv_len < 0 || p->start_pos < 0 || p->window_lo < 0)
+  if (p->q_len < 0 || p->kv_len < 0 || p->start_pos < 0 || p->window_lo < 0 ||
+      p->window_size < 0)
     return ATTN_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_INVALID_ARG;
@@ -351,6 +364,7 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
   a.start_pos = p.start_pos;
   a.causal = p.causal;
   a.window_lo = p.window_lo;
+  a.window_size = p.window_size;
   a.scale_log2 = c->scale * 1.4426950408889634f;
   a.lse = lse;
   a.o_part = c->o_part;
@@ -838,6 +852,7 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   a.start_pos = p->start_pos;
   a.causal = p->causal;
   a.window_lo = p->window_lo;
+  a.window_size = p->window_size;
   a.scale_log2 = c.scale * 1.4426950408889634f;
   a.lse = lse;
   a.o_part = c.o_part;
@@ -848,13 +863,13 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   a.debug = 0;
   const int grid = c.units * c.row_tiles * c.splits;
   if (D == 128) {
-    st = f16 ? launch_fwd<128, 1, false, true, true>(&c, tq, tk, tv, to, a, grid, s)
-             : launch_fwd<128, 1, false, false, true>(&c, tq, tk, tv, to, a, grid, s);
+    st = f16 ? dispatch_fwd<128, false, true>(&c, tq, tk, tv, to, a, grid, s)
+             : dispatch_fwd<128, false, false>(&c, tq, tk, tv, to, a, grid, s);
     if (st == ATTN_OK)
       st = f16 ? launch_merge<128, true>(&c, o, lse, s) : launch_merge<128, false>(&c, o, lse, s);
   } else {
-    st = f16 ? launch_fwd<64, 1, false, true, true>(&c, tq, tk, tv, to, a, grid, s)
-             : launch_fwd<64, 1, false, false, true>(&c, tq, tk, tv, to, a, grid, s);
+    st = f16 ? dispatch_fwd<64, false, true>(&c, tq, tk, tv, to, a, grid, s)
+             : dispatch_fwd<64, false, false>(&c, tq, tk, tv, to, a, grid, s);
     if (st == ATTN_OK)
       st = f16 ? launch_merge<64, true>(&c, o, lse, s) : launch_merge<64, false>(&c, o, lse, s);
   }

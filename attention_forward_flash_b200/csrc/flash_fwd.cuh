@@ -48,6 +48,7 @@ struct FwdArgs {
   int start_pos;
   int causal;
   int window_lo;
+  int window_size;  // sliding window W (0: none): row at position p sees keys >= p - W + 1
   float scale_log2;  // scale * log2(e)
   float* lse;        // [units * R] natural-log lse or nullptr (non-split variant)
   float* o_part;     // [splits, units, R, D] float32 (split variant)
@@ -223,8 +224,10 @@ __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 c
 }
 
 // LF: the kernel also keeps the float32 row sum for the log-sum-exp (exact mode;
-// needed by the split variant and when the caller asks for lse).
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF>
+// needed by the split variant and when the caller asks for lse).  WIN: the
+// per-row sliding window (window_size) is applied; the kernels without it keep
+// the bounds they need in fewer registers.
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN>
 __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
                                   FwdCfg<D, NQT, QUANT, SPLIT>::kCtasPerSm)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -263,7 +266,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     pos_min = a.start_pos + r0 % a.Sq;
     pos_max = a.start_pos + r_last % a.Sq;
   }
-  const int kv_lo = a.window_lo;
+  // Lowest key any row of the CTA sees, and the highest of the rows' lower bounds
+  // (key tiles below it hold masked keys for some row).
+  const int W = WIN ? a.window_size : 0;  // folded away in the kernels without a window
+  const int kv_lo = W > 0 ? max(a.window_lo, pos_min - W + 1) : a.window_lo;
+  const int kv_lo_max = W > 0 ? max(a.window_lo, pos_max - W + 1) : a.window_lo;
   const int kv_hi = a.causal ? min(a.Skv - 1, pos_max) : a.Skv - 1;
   int jt0 = 0, jt1 = 0;  // absolute key-tile range [jt0, jt1)
   if (kv_hi >= kv_lo) {
@@ -518,7 +525,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     const int ri = rvalid ? r : a.R - 1;
     const int i = ri % a.Sq;
     const int pos = a.start_pos + i;
-    const int lo_r = a.window_lo;
+    const int lo_r = W > 0 ? max(a.window_lo, pos - W + 1) : a.window_lo;
     const int hi_r = a.causal ? min(pos, a.Skv - 1) : a.Skv - 1;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + q * 128;
@@ -572,7 +579,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       tc_fence_after();
       const int kv0 = (jt0 + j) * 128;
       const bool need_mask =
-          (kv0 < a.window_lo) || (kv0 + 128 > a.Skv) || (a.causal && kv0 + 127 > pos_min);
+          (kv0 < kv_lo_max) || (kv0 + 128 > a.Skv) || (a.causal && kv0 + 127 > pos_min);
       // S is read in two 64-column halves: the second half's load overlaps the
       // masking and maximum of the first.  Row max: four chains of three-input maxima.
       // Quantised: x keeps the int32 scores' bits, the row max runs on the integers

@@ -45,6 +45,7 @@ class Workload:
     causal: bool = False
     start_pos: int = 0
     window_lo: int = 0
+    window_size: int = 0                 # sliding window W (0: none)
     modes: tuple = ("exact",)    # precision modes this workload is run in
     seed: int = 1000
     k_channel_offset_var: float = 0.0   # per-(b,h) channel offset ~ N(0, var) added to K

@@ -178,7 +178,7 @@ def make_attention(w: Workload, precision):
     from attention_forward_flash_b200 import Attention
     return Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
                      dtype=w.torch_dtype, causal=w.causal, start_pos=w.start_pos,
-                     window_lo=w.window_lo, precision=precision)
+                     window_lo=w.window_lo, precision=precision, window_size=w.window_size)
 
 
 def launches_per_step(att, precision):
@@ -232,7 +232,7 @@ def oracle_sample_time(w: Workload, target_s=12.0, max_rows=None, seed=0):
         rows = np.linspace(0, small.q_len - 1, min(r, small.q_len)).astype(np.int64)
         t0 = time.perf_counter()
         attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
-                      rows=rows)
+                      window_size=w.window_size, rows=rows)
         dt = time.perf_counter() - t0
         if dt >= target_s / 4 or r >= min(rows_cap, small.q_len):
             break
@@ -243,13 +243,13 @@ def oracle_sample_time(w: Workload, target_s=12.0, max_rows=None, seed=0):
         rows = np.linspace(0, small.q_len - 1, r).astype(np.int64)
         t0 = time.perf_counter()
         attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
-                      rows=rows)
+                      window_size=w.window_size, rows=rows)
         dt = time.perf_counter() - t0
     from oracle import visible_range
     pairs = 0
     for i in rows:
         lo, hi = visible_range(int(i), kv_len=w.kv_len, start_pos=w.start_pos, causal=w.causal,
-                               window_lo=w.window_lo)
+                               window_lo=w.window_lo, window_size=w.window_size)
         pairs += max(0, hi - lo + 1)
     flops = 4.0 * w.batch * w.n_q_heads * pairs * w.head_dim
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
@@ -277,7 +277,7 @@ def run_reference(args):
 
     def step():
         attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
-                      rows=rows)
+                      window_size=w.window_size, rows=rows)
 
     for _ in range(args.warmup):
         step()
@@ -307,7 +307,8 @@ def workload_config(w: Workload, precision):
     return {"workload": w.name, "batch": w.batch, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "q_len": w.q_len, "kv_len": w.kv_len,
             "head_dim": w.head_dim, "causal": w.causal, "start_pos": w.start_pos,
-            "window_lo": w.window_lo, "precision": precision, "input_dtype": w.dtype,
+            "window_lo": w.window_lo, "window_size": w.window_size, "precision": precision,
+            "input_dtype": w.dtype,
             "l2": (f"inputs {in_bytes / 1e9:.2f} GB > 126 MB L2" if in_bytes > L2_BYTES
                    else "L2 flushed before every timed call (256 MB written, then 256 MB read)"),
             "parallelism": "replicas (independent problem per GPU)"}

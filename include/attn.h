@@ -24,7 +24,9 @@
  *     lse is [batch, n_q_heads, q_len] float32.
  *   - GQA: query head h reads key/value head h / (n_q_heads / n_kv_heads).
  *   - Query row i sits at absolute position start_pos + i.  With causal != 0
- *     it sees keys j <= start_pos + i.  Keys j < window_lo are never seen.
+ *     it sees keys j <= start_pos + i.  Keys j < window_lo are never seen.  With
+ *     window_size W > 0 it sees only keys j >= start_pos + i - W + 1 as well (the
+ *     last W positions up to its own when causal).
  *     A row that sees no key gets O = 0 and lse = -inf.
  *   - All tensor pointers are DEVICE pointers owned by the caller and must be
  *     16-byte aligned; the library never frees them.  A buffer of zero length
@@ -75,6 +77,8 @@ typedef struct {
   int dtype;       /* attn_dtype of Q, K, V and O */
   int precision;   /* attn_precision */
   int num_splits;  /* key/value splits: 0 = chosen by the library, 1 = none, >1 = forced */
+  int window_size; /* sliding window W >= 0: row i sees keys j >= start_pos + i - W + 1
+                      (0: none); combined with window_lo, the larger bound applies */
 } attn_params;
 
 /* Caller-owned device buffers of the quantised mode (all 16-byte aligned):

@@ -37,7 +37,8 @@ def max_abs(o, r):
 def attention_for(w, precision="exact", num_splits=0):
     return Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
                      dtype=w.torch_dtype, causal=w.causal, start_pos=w.start_pos,
-                     window_lo=w.window_lo, precision=precision, num_splits=num_splits)
+                     window_lo=w.window_lo, precision=precision, num_splits=num_splits,
+                     window_size=w.window_size)
 
 
 def run_gpu(w, q, k, v, precision="exact", num_splits=0):
@@ -51,6 +52,7 @@ def run_gpu(w, q, k, v, precision="exact", num_splits=0):
 
 def oracle_for(w, q, k, v, rows=None):
     return attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos, window_lo=w.window_lo,
+                         window_size=w.window_size,
                          rows=rows)
 
 

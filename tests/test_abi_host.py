@@ -43,6 +43,7 @@ def _params(**kw):
     (dict(kv_len=-5), _abi.ATTN_ERR_INVALID_ARG),
     (dict(start_pos=-1), _abi.ATTN_ERR_INVALID_ARG),
     (dict(window_lo=-1), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(window_size=-1), _abi.ATTN_ERR_INVALID_ARG),
     (dict(causal=2), _abi.ATTN_ERR_INVALID_ARG),
     (dict(dtype=7), _abi.ATTN_ERR_INVALID_ARG),
     (dict(precision=3), _abi.ATTN_ERR_INVALID_ARG),

@@ -26,7 +26,8 @@ pytestmark = pytest.mark.gpu
 def _att(w, precision="exact", num_splits=0):
     return Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
                      dtype=w.torch_dtype, causal=w.causal, start_pos=w.start_pos,
-                     window_lo=w.window_lo, precision=precision, num_splits=num_splits)
+                     window_lo=w.window_lo, precision=precision, num_splits=num_splits,
+                     window_size=w.window_size)
 
 
 def _device_result(att, q, k, v):
@@ -176,3 +177,14 @@ def test_full_size_video_default_chunks():
     torch.cuda.current_stream().synchronize()
     att.check_error()
     _same(o, ro.cpu(), "video O")
+
+
+def test_sliding_window_bit_identical_to_device_entry():
+    w = Workload("gqa_sliding", 4, 8, 2, 700, 1291, 128, "fp16", causal=True, start_pos=591,
+                 window_size=200, seed=4103)
+    q, k, v = make_qkv(w)
+    att = _att(w, num_splits=SINGLE_PASS)
+    ro, rl, _ = _device_result(att, q, k, v)
+    o, lse, _ = _host_result(att, q, k, v, chunks=3)
+    _same(o, ro, "sliding window O")
+    _same(lse, rl, "sliding window lse")

@@ -307,3 +307,46 @@ def test_long_context_quant(name, num_splits):
     ro, _ = oracle_for(w, q, k, v, rows=rows)
     e = rel_rmse(o[:, :, rows], ro)
     assert e <= QUANT_RMSE, f"{name}: quantised rel_rmse {e:.3e}"
+
+
+# Per-row sliding window (window_size W): row i at position p sees keys
+# max(window_lo, p - W + 1) .. p.  Windows narrower than, equal to and wider
+# than a key tile, crossing tile edges at ragged offsets, with and without
+# window_lo, in the single-pass and split-KV kernels.
+SLIDING = [
+    # D, Sq, Skv, start_pos, W, window_lo, causal, num_splits
+    (128, 700, 1291, 591, 1, 0, True, 1),
+    (128, 700, 1291, 591, 64, 0, True, 1),
+    (128, 700, 1291, 591, 127, 0, True, 1),
+    (128, 700, 1291, 591, 128, 0, True, 0),
+    (64, 700, 1291, 591, 129, 0, True, 1),
+    (64, 700, 1291, 591, 300, 650, True, 1),
+    (128, 1000, 1000, 0, 1000, 0, True, 1),
+    (128, 1000, 1000, 0, 5000, 0, True, 0),
+    (64, 513, 1111, 500, 300, 0, False, 1),
+    (128, 4, 32768, 32764, 1, 0, True, 0),
+    (128, 4, 32768, 32764, 100, 0, True, 0),
+    (128, 1, 32768, 32767, 4096, 0, True, 0),
+]
+
+
+@pytest.mark.parametrize("D,Sq,Skv,start_pos,W,window_lo,causal,num_splits", SLIDING)
+def test_sliding_window(D, Sq, Skv, start_pos, W, window_lo, causal, num_splits):
+    w = Workload("sliding", 1, 8, 2, Sq, Skv, D, "bf16" if D == 64 else "fp16", causal=causal,
+                 start_pos=start_pos, window_lo=window_lo, window_size=W, seed=6000 + W + Sq)
+    q, k, v = make_qkv(w)
+    o, lse, att = run_gpu(w, q, k, v, num_splits=num_splits)
+    if num_splits == 1:
+        assert att.num_splits == 1
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro, f"W={W}")
+    check_lse(lse, rl, f"W={W}")
+
+
+def test_sliding_window_quantised():
+    w = Workload("sliding_q", 2, 8, 2, 700, 1291, 128, "bf16", causal=True, start_pos=591,
+                 window_size=256, seed=6101)
+    q, k, v = make_qkv(w)
+    o, _, _ = run_gpu(w, q, k, v, precision="quant")
+    ro, _ = oracle_for(w, q, k, v)
+    assert rel_rmse(o, ro) <= QUANT_RMSE
