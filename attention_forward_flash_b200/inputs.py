@@ -17,6 +17,8 @@ Shapes mirror the pages' workloads:
   works on 1024px image diffusion), with a per-channel offset on K that gives
   the channel outliers per-block INT8 quantisation has to cope with.
 * ``llm``: a causal GQA prefill with 1% of K entries scaled by 20.
+* ``llm_window``: the same shape with a per-row sliding window of 1024 positions
+  (each query row sees the last 1024 keys up to its own).
 * ``tiny``: a small exact case the oracle finishes in well under a second.
 
 Recipe: a CPU ``torch.Generator`` seeded with the workload's seed draws float32
@@ -83,6 +85,10 @@ WORKLOADS = {
     "llm": Workload("llm", 4, 32, 8, 8192, 8192, 128, "bf16", causal=True,
                     modes=("exact", "quant"), seed=1004, k_outlier_frac=0.01,
                     k_outlier_mult=20.0, oracle_rows=256),
+    # the causal GQA prefill with a 1024-position sliding window per row
+    "llm_window": Workload("llm_window", 4, 32, 8, 8192, 8192, 128, "bf16", causal=True,
+                           window_size=1024, modes=("exact", "quant"), seed=1005,
+                           oracle_rows=256),
 }
 
 

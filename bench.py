@@ -301,6 +301,21 @@ def run_reference(args):
     return 0
 
 
+def work_flops(w: Workload):
+    """Work count of one call: the headline formula (4*B*Hq*Sq*Skv*D, halved for
+    causal), or, with a per-row sliding window, 4*B*Hq*D times the (q, k) pairs the
+    window leaves visible."""
+    if w.window_size <= 0:
+        return w.flops()
+    pairs = 0
+    for i in range(w.q_len):
+        p = w.start_pos + i
+        lo = max(w.window_lo, p - w.window_size + 1)
+        hi = min(p, w.kv_len - 1) if w.causal else w.kv_len - 1
+        pairs += max(0, hi - lo + 1)
+    return 4.0 * w.batch * w.n_q_heads * pairs * w.head_dim
+
+
 def workload_config(w: Workload, precision):
     in_bytes = (w.batch * w.n_q_heads * w.q_len + 2 * w.batch * w.n_kv_heads * w.kv_len) * \
         w.head_dim * 2
@@ -417,7 +432,7 @@ def run_native(args):
     att.check_error()
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local, world)
-    flops = w.flops()
+    flops = work_flops(w)
     value = flops * world / (ms * 1e-3) / 1e12
 
     # ---- dominant kernel (the fused attention kernel) for the roofline
@@ -480,12 +495,13 @@ def run_native(args):
         extra = {}
         for name, prec in (("video", "quant" if precision == "exact" else "exact"),
                            ("llm", "exact"), ("llm", "quant"), ("image", "exact"),
-                           ("image", "quant"), ("decode", "exact"), ("decode_window", "exact")):
+                           ("image", "quant"), ("decode", "exact"), ("decode_window", "exact"),
+                           ("llm_window", "exact")):
             if name == w.name and prec == precision:
                 continue
             wx = WORKLOADS[name]
             mx = measure(wx, prec, 10 if wx.flops() > 1e12 else 50, 3, device)
-            fl = wx.flops()
+            fl = work_flops(wx)
             entry = {"ms_per_step": mx["ms_step"], "ms_kernel": mx["ms_kernel"],
                      "tflops_step": fl / (mx["ms_step"] * 1e-3) / 1e12,
                      "tflops_kernel": fl / (mx["ms_kernel"] * 1e-3) / 1e12,

@@ -34,7 +34,7 @@ def test_exact_full(name):
         assert att.num_splits > 1  # few-row problems take the split-KV path
 
 
-@pytest.mark.parametrize("name", ["video", "llm"])
+@pytest.mark.parametrize("name", ["video", "llm", "llm_window"])
 def test_exact_full_size_sampled_rows(name):
     w = WORKLOADS[name]
     q, k, v = make_qkv(w)
@@ -350,3 +350,23 @@ def test_sliding_window_quantised():
     o, _, _ = run_gpu(w, q, k, v, precision="quant")
     ro, _ = oracle_for(w, q, k, v)
     assert rel_rmse(o, ro) <= QUANT_RMSE
+
+
+# The qsa2 audit's decode matrix ("build and reproduction"): a 32768-cell KV cache,
+# 1/2/4/8 query rows, first positions 0, 1, 63, 64, 512, 2047, 2048, 2050, 8192 and
+# 30000 (causal: the cells past each row's position are masked), each with and
+# without a 1024-position sliding window.
+QSA2_CELLS = 32768
+QSA2 = [(ntok, pos0, W) for ntok in (1, 2, 4, 8)
+        for pos0 in (0, 1, 63, 64, 512, 2047, 2048, 2050, 8192, 30000) for W in (0, 1024)]
+
+
+@pytest.mark.parametrize("ntok,pos0,W", QSA2)
+def test_decode_qsa2_positions(ntok, pos0, W):
+    w = _small(q_len=ntok, start_pos=pos0, kv_len=QSA2_CELLS, window_size=W,
+               seed=41 + 7 * pos0 + ntok + W)
+    q, k, v = make_qkv(w)
+    o, lse, _ = run_gpu(w, q, k, v)
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro, str((ntok, pos0, W)))
+    check_lse(lse, rl)
