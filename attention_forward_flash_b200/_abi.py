@@ -12,7 +12,8 @@ ATTN_EXACT, ATTN_INT8QK_FP8PV = 0, 1
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
-            "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host")
+            "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host",
+            "attn_forward_paged")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -79,6 +80,8 @@ def lib():
         L.attn_forward_splitkv_noalloc.restype = c_int
         L.attn_forward_host.argtypes = [vp] * 11 + [ctypes.POINTER(AttnQBufs), c_int, vp]
         L.attn_forward_host.restype = c_int
+        L.attn_forward_paged.argtypes = [vp, vp, vp, vp, vp, c_int, vp, vp, vp]
+        L.attn_forward_paged.restype = c_int
         _LIB = L
     return _LIB
 
@@ -144,3 +147,8 @@ def attn_forward_host(ctx, q_host, k_host, v_host, o_host, lse_host, q_dev, k_de
     _check(lib().attn_forward_host(ctx, q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev,
                                    v_dev, o_dev, lse_dev, qb, chunks, stream),
            "attn_forward_host")
+
+
+def attn_forward_paged(ctx, q, k_pool, v_pool, block_table, num_blocks, o, lse, stream):
+    _check(lib().attn_forward_paged(ctx, q, k_pool, v_pool, block_table, num_blocks, o, lse,
+                                    stream), "attn_forward_paged")

@@ -117,6 +117,40 @@ class Attention:
 
     __call__ = forward
 
+    def forward_paged(self, q, k_pool, v_pool, block_table, *, out=None, lse=None,
+                      return_lse=False, stream=None):
+        """Exact-mode forward over a paged key/value cache (``attn_forward_paged``).
+
+        k_pool, v_pool: [num_blocks, n_kv_heads, 128, head_dim] CUDA tensors of the
+        context's dtype; block_table: int32 CUDA tensor [batch, ceil(kv_len / 128)].
+        """
+        p = self.params
+        if self.precision != "exact":
+            raise ValueError("forward_paged() needs precision='exact'")
+        want = (p.n_kv_heads, 128, p.head_dim)
+        for name, t in (("k_pool", k_pool), ("v_pool", v_pool)):
+            if (t.dim() != 4 or tuple(t.shape[1:]) != want or t.dtype != self.dtype
+                    or not t.is_contiguous() or not t.is_cuda):
+                raise ValueError(f"{name}: expected contiguous CUDA {self.dtype} "
+                                 f"[blocks, {want[0]}, {want[1]}, {want[2]}]")
+        if v_pool.shape[0] != k_pool.shape[0]:
+            raise ValueError("k_pool and v_pool must hold the same number of blocks")
+        nbt = (p.kv_len + 127) // 128
+        if (block_table.dtype != torch.int32 or tuple(block_table.shape) != (p.batch, nbt)
+                or not block_table.is_contiguous() or not block_table.is_cuda):
+            raise ValueError(f"block_table: expected contiguous CUDA int32 [{p.batch}, {nbt}]")
+        if out is None:
+            out = torch.empty((p.batch, p.n_q_heads, p.q_len, p.head_dim), dtype=self.dtype,
+                              device=q.device)
+        if lse is None and return_lse:
+            lse = torch.empty((p.batch, p.n_q_heads, p.q_len), dtype=torch.float32,
+                              device=q.device)
+        _abi.attn_forward_paged(self.ctx, q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                block_table.data_ptr(), k_pool.shape[0], out.data_ptr(),
+                                lse.data_ptr() if lse is not None else None,
+                                _stream_handle(stream))
+        return (out, lse) if return_lse else out
+
     def forward_host(self, q, k, v, *, out=None, lse=None, return_lse=False, staging=None,
                      chunks=0, stream=None, device=None):
         """End-to-end forward from host tensors through ``attn_forward_host``.

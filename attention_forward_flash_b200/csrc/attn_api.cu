@@ -97,6 +97,22 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// 4-D tiled map of a paged key/value pool [blocks][kv heads][128 positions][D]:
+// dims (D, 128, kv heads, blocks), box (64 channels, 128 positions, 1, 1).
+bool make_pool_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t D,
+                   uint64_t hkv, uint64_t blocks) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {D, 128, hkv, blocks};
+  cuuint64_t strides[3] = {D * 2, 128 * D * 2, hkv * 128 * D * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename K>
 bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
@@ -632,6 +648,75 @@ attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* 
   if (s != ATTN_OK) return s;
   return forward_units(c, 0, c->units, q, k, v, qb, o, lse, static_cast<cudaStream_t>(stream),
                        0);
+}
+
+attn_status attn_forward_paged(attn_ctx* c, const void* q, const void* k_pool,
+                               const void* v_pool, const int32_t* block_table, int num_blocks,
+                               void* o, float* lse, void* stream) {
+  if (!c) return ATTN_ERR_INVALID_ARG;
+  const attn_params& p = c->p;
+  if (p.precision != ATTN_EXACT) return ATTN_ERR_UNSUPPORTED;
+  const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
+  if (bad_ptr(q, need_q) || bad_ptr(o, need_q) || (lse && !aligned16(lse)) ||
+      bad_ptr(k_pool, need_kv) || bad_ptr(v_pool, need_kv) ||
+      (need_kv && (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u))) ||
+      (need_kv && num_blocks < 1))
+    return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D = p.head_dim;
+  const bool f16 = p.dtype == ATTN_FP16;
+  const size_t rows = static_cast<size_t>(c->units) * c->R;
+  if (rows == 0) return ATTN_OK;
+  if (p.kv_len == 0) {  // every row sees no key
+    if (cudaMemsetAsync(o, 0, rows * D * 2, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (lse) fill_lse_kernel<<<ceil_div(rows, 256), 256, 0, st>>>(lse, rows);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  const CUtensorMapDataType t16 =
+      f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t R = c->R, U = c->units;
+  CUtensorMap tq, tk, tv, to;
+  bool ok = make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_pool_map(&tk, t16, k_pool, D, p.n_kv_heads, num_blocks);
+  ok &= make_pool_map(&tv, t16, v_pool, D, p.n_kv_heads, num_blocks);
+  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return ATTN_ERR_CUDA;
+  FwdArgs a{};
+  a.R = c->R;
+  a.Sq = p.q_len;
+  a.Skv = p.kv_len;
+  a.G = c->G;
+  a.units = c->units;
+  a.row_tiles = c->row_tiles;
+  a.splits = c->splits;
+  a.tiles_per_split = c->tiles_per_split;
+  a.start_pos = p.start_pos;
+  a.causal = p.causal;
+  a.window_lo = p.window_lo;
+  a.window_size = p.window_size;
+  a.block_table = block_table;
+  a.bt_stride = ceil_div(p.kv_len, 128);
+  a.n_kv_heads = p.n_kv_heads;
+  a.scale_log2 = c->scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.o_part = c->o_part;
+  a.lse_part = c->lse_part;
+  a.nblk_q = ceil_div(p.q_len, 128);
+  a.nblk_k = ceil_div(p.kv_len, 128);
+  a.err = c->err;
+  a.debug = c->debug;
+  const int grid = c->units * c->row_tiles * (c->split_path ? c->splits : 1);
+  attn_status s;
+  if (D == 128)
+    s = f16 ? dispatch_fwd<128, false, true>(c, tq, tk, tv, to, a, grid, st)
+            : dispatch_fwd<128, false, false>(c, tq, tk, tv, to, a, grid, st);
+  else
+    s = f16 ? dispatch_fwd<64, false, true>(c, tq, tk, tv, to, a, grid, st)
+            : dispatch_fwd<64, false, false>(c, tq, tk, tv, to, a, grid, st);
+  if (s != ATTN_OK || !c->split_path) return s;
+  if (D == 128)
+    return f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
+  return f16 ? launch_merge<64, true>(c, o, lse, st) : launch_merge<64, false>(c, o, lse, st);
 }
 
 attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_host,

@@ -49,6 +49,12 @@ struct FwdArgs {
   int causal;
   int window_lo;
   int window_size;  // sliding window W (0: none): row at position p sees keys >= p - W + 1
+  // Paged K/V (exact mode): if block_table is set, key tile t of batch entry b is
+  // block block_table[b * bt_stride + t] of a pool [blocks][n_kv_heads][128][D],
+  // and the K/V tensor maps are 4-D over that pool.
+  const int* block_table;
+  int bt_stride;
+  int n_kv_heads;
   float scale_log2;  // scale * log2(e)
   float* lse;        // [units * R] natural-log lse or nullptr (non-split variant)
   float* o_part;     // [splits, units, R, D] float32 (split variant)
@@ -368,7 +374,17 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag)) { raise(); ok = false; break; }
           if ((a.debug & 1u) && j == 1 && part == 0) continue;  // timeout test: never load
           const uint32_t dst = sbase + C::kRingOff + s * C::kSlot;
-          if (part == 0) {
+          if (!QUANT && a.block_table != nullptr) {
+            // paged: the tile is one whole block of the pool (an id outside the pool
+            // reads TMA's zero fill, never memory outside it)
+            const int blk = __ldg(a.block_table + (size_t)(u / a.n_kv_heads) * a.bt_stride +
+                                  (jt0 + j));
+            const int hk = u % a.n_kv_heads;
+            const CUtensorMap* m = part == 0 ? &tm_k : &tm_v;
+            mbar_arrive_expect_tx(full_bar(s), part == 0 ? C::kKBytes : C::kVBytes);
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_load_4d(m, dst + bx * 128 * 64 * 2, full_bar(s), bx * 64, 0, hk, blk);
+          } else if (part == 0) {
             mbar_arrive_expect_tx(full_bar(s), C::kKBytes);
             if constexpr (QUANT) {
               tma_load_3d(&tm_k, dst, full_bar(s), 0, kv0, u);

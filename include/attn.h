@@ -33,6 +33,9 @@
  *     (q_len or kv_len 0) may be NULL.  `stream` is a
  *     cudaStream_t passed as void*.  Every call is asynchronous on that stream;
  *     argument errors are reported synchronously, before anything is launched.
+ *   - Keys of a loaded 128-key tile that a row cannot see get a zero weight in P.V;
+ *     they must hold finite values (an Inf or NaN there reaches O).  Key tiles that
+ *     no row of a CTA sees are not loaded at all.
  *   - A context is not safe for concurrent use from several host threads.
  *   - Device-side waits are bounded (about 1.5 s).  A wait that runs out
  *     records an error word in the context; attn_get_error() reports it.
@@ -171,6 +174,27 @@ attn_status attn_forward_host(attn_ctx *c, const void *q_host, const void *k_hos
                               const void *v_host, void *o_host, float *lse_host, void *q_dev,
                               void *k_dev, void *v_dev, void *o_dev, float *lse_dev,
                               const attn_qbufs *qb, int chunks, void *stream);
+
+/* Paged key/value cache (exact mode).
+ * No counterpart on the source pages beyond the decode workload of the qsa2
+ * audit (its 32768-cell KV cache): keys and values live in fixed blocks of 128
+ * positions in a pool shared by all batch entries, as a serving engine keeps
+ * them, and a block table maps each batch entry's positions to blocks.
+ * k_pool, v_pool: [num_blocks, n_kv_heads, 128, head_dim] (the context's dtype,
+ * 16-byte aligned).  block_table: int32 [batch, ceil(kv_len / 128)] (4-byte
+ * aligned, device memory); entry [b][t] is the block that holds positions
+ * 128 t .. 128 t + 127 of batch entry b.  Everything else is as attn_forward
+ * (q, o and lse dense; kv_len is every batch entry's number of positions), and
+ * the result equals attn_forward on K and V gathered through the table.  An
+ * entry outside [0, num_blocks) reads zeros (the copy engine's bounds), never
+ * memory outside the pool.  The positions past kv_len in a batch entry's last
+ * block must hold finite values.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, num_blocks < 1),
+ * ATTN_ERR_UNSUPPORTED (quantised mode), ATTN_ERR_CUDA (tensor-map encode or
+ * launch failure). */
+attn_status attn_forward_paged(attn_ctx *c, const void *q, const void *k_pool,
+                               const void *v_pool, const int32_t *block_table, int num_blocks,
+                               void *o, float *lse, void *stream);
 
 /* Synchronises `stream`, reads and clears the context's device error word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last call,

@@ -10,7 +10,13 @@ against hand-worked examples, brute force, closed forms and library special
 cases.
 """
 
-from .attention import attention_f64, attention_flops, visible_pairs, visible_range  # noqa: F401
+from .attention import (  # noqa: F401
+    attention_f64,
+    attention_flops,
+    gather_paged,
+    visible_pairs,
+    visible_range,
+)
 from .quant import (  # noqa: F401
     E4M3_MAX,
     QK_BLOCK,

@@ -66,6 +66,28 @@ def visible_range(i, *, kv_len, start_pos=0, causal=False, window_lo=0, window_s
     return lo, hi
 
 
+def gather_paged(pool, block_table, kv_len):
+    """Dense keys (or values) ``[B, Hkv, kv_len, D]`` of a paged cache.
+
+    ``pool`` is ``[num_blocks, Hkv, 128, D]`` and ``block_table`` is ``[B, ceil(kv_len / 128)]``:
+    position ``128 t + r`` of batch entry ``b`` is ``pool[block_table[b, t], :, r, :]``.  The
+    pages show no cache layout; this is the block-table reading of the qsa2 audit's
+    32768-cell KV cache ("round 21 track b -- qsa2", section "build and reproduction").
+    """
+    pool = _as_f64(pool)
+    table = np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table,
+                       dtype=np.int64)
+    B, nbt = table.shape
+    _, Hkv, bs, D = pool.shape
+    assert bs == 128 and nbt * 128 >= kv_len
+    out = np.empty((B, Hkv, kv_len, D), dtype=np.float64)
+    for b in range(B):
+        for t in range(nbt):
+            n = min(128, kv_len - 128 * t)
+            out[b, :, 128 * t:128 * t + n, :] = pool[table[b, t], :, :n, :]
+    return out
+
+
 def _as_f64(x):
     """Widen a torch tensor (bf16/fp16/fp32, any device) or array to float64."""
     if hasattr(x, "detach"):
@@ -158,11 +180,11 @@ def attention_flops(B, Hq, Sq, Skv, D, *, causal=False):
     return f / 2.0 if causal else f
 
 
-def visible_pairs(Sq, Skv, *, start_pos=0, causal=False, window_lo=0):
+def visible_pairs(Sq, Skv, *, start_pos=0, causal=False, window_lo=0, window_size=0):
     """Exact number of visible (query, key) pairs of one head."""
     n = 0
     for i in range(Sq):
         lo, hi = visible_range(i, kv_len=Skv, start_pos=start_pos, causal=causal,
-                               window_lo=window_lo)
+                               window_lo=window_lo, window_size=window_size)
         n += max(0, hi - lo + 1)
     return n

@@ -22,7 +22,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import attention_f64, attention_flops, visible_pairs, visible_range
+from oracle import attention_f64, attention_flops, gather_paged, visible_pairs, visible_range
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -306,3 +306,34 @@ def test_keys_outside_the_sliding_window_have_no_influence():
     o3, l3 = attention_f64(q, k, v, causal=True, start_pos=50, window_size=55)
     o4, l4 = attention_f64(q, k, v, causal=True, start_pos=50)
     assert np.array_equal(o3, o4) and np.array_equal(l3, l4)
+
+
+# Paged cache: the block-table gather.
+def test_gather_paged_identity_table_is_a_reshape():
+    rng = np.random.default_rng(41)
+    B, Hkv, n, D = 2, 3, 5, 4
+    dense = rng.standard_normal((B, Hkv, 128 * n, D))
+    # block b * n + t holds positions 128 t .. of batch entry b
+    pool = dense.reshape(B, Hkv, n, 128, D).transpose(0, 2, 1, 3, 4).reshape(B * n, Hkv, 128, D)
+    table = np.arange(B * n).reshape(B, n)
+    assert np.array_equal(gather_paged(pool, table, 128 * n), dense)
+
+
+def test_gather_paged_inverts_a_scatter_through_a_random_table():
+    rng = np.random.default_rng(42)
+    B, Hkv, D, kv_len = 3, 2, 8, 300                 # 3 blocks per entry, the last one partial
+    nbt = -(-kv_len // 128)
+    dense = rng.standard_normal((B, Hkv, kv_len, D))
+    nblocks = B * nbt + 4                             # spare blocks nobody references
+    table = rng.permutation(nblocks)[:B * nbt].reshape(B, nbt)
+    pool = np.full((nblocks, Hkv, 128, D), np.nan)
+    for b in range(B):
+        for t in range(nbt):
+            m = min(128, kv_len - 128 * t)
+            pool[table[b, t], :, :m] = dense[b, :, 128 * t:128 * t + m]
+    got = gather_paged(pool, table, kv_len)
+    assert np.array_equal(got, dense)                 # no NaN from spare blocks or the tail
+    q = rng.standard_normal((B, 4, 5, D))
+    o1, l1 = attention_f64(q, got, got, causal=True, start_pos=295)
+    o2, l2 = attention_f64(q, dense, dense, causal=True, start_pos=295)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
