@@ -69,6 +69,7 @@ def test_null_arguments():
     assert L.attn_forward(None, None, None, None, None, None, None, None) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_quantize_qk(None, None, None, None, None, None) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_forward_host(*([None] * 12), 0, None) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_forward_paged(*([None] * 5), 0, None, None, None) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_get_error(None, None) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_debug_set(None, 0) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_num_splits(None) == 0

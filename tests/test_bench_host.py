@@ -68,3 +68,18 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "--workload", "tiny", "--steps", "1", "--warmup", "1"],
                        capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_work_flops_counts_the_window_visible_pairs():
+    """Without a window the bench uses the headline formula; with one it counts the
+    visible (q, k) pairs: checked against a brute-force double loop."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from attention_forward_flash_b200.inputs import Workload
+    w = Workload("t", 2, 4, 2, 37, 61, 64, causal=True, start_pos=20)
+    assert bench.work_flops(w) == w.flops()
+    for W, lo in ((1, 0), (5, 0), (16, 30), (200, 0)):
+        ww = w.scaled(window_size=W, window_lo=lo)
+        pairs = sum(1 for i in range(ww.q_len) for j in range(ww.kv_len)
+                    if j >= lo and j <= ww.start_pos + i and ww.start_pos + i - j < W)
+        assert bench.work_flops(ww) == 4.0 * ww.batch * ww.n_q_heads * pairs * ww.head_dim
