@@ -23,7 +23,7 @@ The flash method (online softmax over key tiles) reaches exactly this result up
 to rounding order, so the oracle is the definition written out, with a library
 matmul as the only primitive and no tiling.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * layout ``[B, H, S, D]`` contiguous;
 * query head ``hq`` reads key/value head ``hq // (Hq // Hkv)`` (contiguous

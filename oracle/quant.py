@@ -7,10 +7,10 @@ code with the CUDA library.
 The reduced-precision mode is the "SageAttention 2 INT8 QK · FP8 PV" row of the
 table in section "1 · Только ядро" of the page "Ядра attention на домашней RTX
 5080": Q and K are quantised to INT8 per block with FP32 scales, the product
-P·V runs in FP8 E4M3.  The page gives only that description; the granularity
-(one scale per 128-token block per head for Q/K, one scale per head and channel
-for V) comes from the workload statement this build targets.  Everything else
-below is a reading of the plainest kind, listed in the design doc:
+P·V runs in FP8 E4M3.  The page gives only that description.  The granularity
+is one scale per 128-token block per head for Q/K (the block size of the key tile
+the kernels stream) and one scale per head and channel for V.  This and everything
+else below is a reading of the plainest kind:
 
 * Q/K block = 128 consecutive tokens x all D channels of one (b, h); the last
   block of a sequence may be partial.
