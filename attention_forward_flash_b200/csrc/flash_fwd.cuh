@@ -366,19 +366,25 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       for (int s = 0; s < C::kNS; ++s) last_issue[s] = -1;
       int it = 0;
       bool ok = true;
+      // Paged K/V: this unit's row of the block table; each tile's block id is read
+      // one tile ahead, so the read does not delay the tile's copies.
+      const bool paged = !QUANT && a.block_table != nullptr;
+      const int* bt_row =
+          paged ? a.block_table + (size_t)(u / a.n_kv_heads) * a.bt_stride + jt0 : nullptr;
+      int blk_next = (paged && n > 0) ? __ldg(bt_row) : 0;
       for (int j = 0; j < n && ok; ++j) {
         const int kv0 = (jt0 + j) * 128;
+        const int blk = blk_next;
+        if (paged && j + 1 < n) blk_next = __ldg(bt_row + j + 1);
         for (int part = 0; part < 2 && ok; ++part, ++it) {  // 0: K tile, 1: V tile
           const int s = it % C::kNS;
           const uint32_t ph = (it / C::kNS) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag)) { raise(); ok = false; break; }
           if ((a.debug & 1u) && j == 1 && part == 0) continue;  // timeout test: never load
           const uint32_t dst = sbase + C::kRingOff + s * C::kSlot;
-          if (!QUANT && a.block_table != nullptr) {
-            // paged: the tile is one whole block of the pool (an id outside the pool
-            // reads TMA's zero fill, never memory outside it)
-            const int blk = __ldg(a.block_table + (size_t)(u / a.n_kv_heads) * a.bt_stride +
-                                  (jt0 + j));
+          if (paged) {
+            // the tile is one whole block of the pool (an id outside the pool reads
+            // TMA's zero fill, never memory outside it)
             const int hk = u % a.n_kv_heads;
             const CUtensorMap* m = part == 0 ? &tm_k : &tm_v;
             mbar_arrive_expect_tx(full_bar(s), part == 0 ? C::kKBytes : C::kVBytes);
