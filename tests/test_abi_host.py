@@ -90,3 +90,57 @@ def test_qbufs_sizes():
     assert vt == 2 * 2 * 128 * 33 * 128 and vs == 2 * 2 * 128 * 4
     with pytest.raises(afb.AttnError):
         afb.attn_qbufs_sizes(_params(head_dim=80))
+
+
+C_CALLER = r"""
+#include <stddef.h>
+#include <stdint.h>
+#include "attn.h"
+
+/* Every declared function, called with the argument types the header states. */
+int main(void) {
+  attn_params p = {1, 2, 2, 256, 256, 64, 0, 0, 0, 0.0f, ATTN_BF16, ATTN_EXACT, 0, 0};
+  attn_ctx *c = NULL;
+  attn_qbufs qb = {0};
+  size_t sizes[6];
+  unsigned err = 0;
+  int32_t table[2] = {0, 1};
+  if (attn_create(&p, &c) != ATTN_OK) return 1;
+  attn_quantize_qk(c, NULL, NULL, NULL, &qb, NULL);
+  attn_forward(c, NULL, NULL, NULL, NULL, NULL, NULL, NULL);
+  attn_forward_host(c, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0,
+                    NULL);
+  attn_forward_paged(c, NULL, NULL, NULL, table, 1, NULL, NULL, NULL);
+  attn_get_error(c, NULL);
+  attn_qbufs_sizes(&p, sizes);
+  attn_num_splits(c);
+  attn_debug_set(c, 0u);
+  attn_debug_exp2(NULL, NULL, 0, NULL);
+  attn_forward_splitkv_noalloc(&p, NULL, NULL, NULL, NULL, NULL, &err, NULL);
+  (void)attn_status_string(ATTN_OK);
+  attn_destroy(c);
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_against_the_library(tmp_path):
+    """include/attn.h compiles as C99 with warnings as errors, and a C program that
+    calls every declared function links against libattn.so (it is not run: that
+    needs a GPU)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    called = set(re.findall(r"\b(attn_\w+)\s*\(", C_CALLER))
+    assert called >= set(_declared_functions())
+    lib_dir = os.path.dirname(afb.lib_path())
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                        str(tmp_path / "caller"), "-L", lib_dir, "-lattn",
+                        "-Wl,--unresolved-symbols=ignore-in-shared-libs"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
