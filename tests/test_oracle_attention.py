@@ -46,7 +46,8 @@ def test_hand_worked_example():
     scale = math.log(2.0)
     for case in d["cases"]:
         o, lse = attention_f64(q, k, v, scale=scale, causal=case["causal"],
-                               start_pos=case["start_pos"], window_lo=case["window_lo"])
+                               start_pos=case["start_pos"], window_lo=case["window_lo"],
+                               window_size=case.get("window_size", 0))
         want_o = np.array([[_frac(x) for x in row] for row in case["o"]])
         want_lse = np.array([_frac(x) for x in case["lse"]])
         np.testing.assert_allclose(o[0, 0], want_o, rtol=0, atol=1e-15, err_msg=case["name"])
