@@ -36,7 +36,9 @@
  *   - Keys of a loaded 128-key tile that a row cannot see get a zero weight in P.V;
  *     they must hold finite values (an Inf or NaN there reaches O).  Key tiles that
  *     no row of a CTA sees are not loaded at all.
- *   - A context is not safe for concurrent use from several host threads.
+ *   - A context is not safe for concurrent use from several host threads.  Its
+ *     workspace (split-KV partials, V channel maxima) is shared by all of its
+ *     calls: calls on different streams that use it must be ordered by the caller.
  *   - Device-side waits are bounded (about 1.5 s).  A wait that runs out
  *     records an error word in the context; attn_get_error() reports it.
  */
