@@ -1,10 +1,13 @@
 """CUDA path (through the C ABI) against the float64 oracle on the same seeded inputs.
 
 Covers every workload at its full size (all rows where the oracle is quick,
-a seeded subset of 256 query rows per head on the two largest), in both
-precision modes where the workload uses them, plus the boundary matrix of key
-lengths, start positions, windows and query-row counts, empty rows, the
-single-pass and split-KV variants, determinism and masked-key independence.
+a seeded subset of 256 query rows per head on the largest), in both precision
+modes where the workload uses them, plus the boundary matrix of key lengths,
+start positions, windows and query-row counts, empty rows, the single-pass and
+split-KV variants (quantised too), determinism, masked-key independence, the
+bounded-wait error path in both modes, long contexts (131072 keys in one CTA,
+32768-key decodes), per-row sliding windows, and the qsa2 audit's decode matrix
+on a 32768-cell cache.
 """
 
 import math
