@@ -1,6 +1,10 @@
 """Pins of the reference quantisers against things other than themselves.
 
-* hand-worked examples in ``golden/quant_examples.json``;
+* hand-worked examples in ``golden/quant_examples.json``, including scales that
+  are not powers of two, with values whose code changes if the quotient x / s
+  is replaced by a multiplication with a rounded reciprocal or folded factor, or
+  by multiplying first (expected codes derived with exact rationals by
+  ``golden/make_quant_quotient_cases.py``, never by the oracle);
 * the E4M3 encoder against an exhaustive nearest-value search over the finite
   codes decoded from the format definition (ties to the even code), on a dense
   sweep of float32 values;
@@ -39,6 +43,77 @@ def test_e4m3_worked_examples():
     for ex in d["e4m3"]:
         got = int(fp8_e4m3_encode(np.float32(ex["x"])))
         assert got == int(ex["code"], 16), ex
+
+
+def _golden():
+    return json.load(open(os.path.join(GOLDEN, "quant_examples.json")))
+
+
+def _stand_ins(x, amax, qmax):
+    """float32 values of the three stand-ins for the quotient x / RN(amax / qmax)."""
+    f = np.float32
+    x, amax, qmax = f(x), f(amax), f(qmax)
+    s = f(amax / qmax)
+    return {"times_reciprocal": f(x * f(f(1) / s)),
+            "times_folded_factor": f(x * f(qmax / amax)),
+            "multiply_first": f(f(x * qmax) / amax)}
+
+
+def test_int8_quotient_cases():
+    import sys
+    sys.path.insert(0, GOLDEN)
+
+    import make_quant_quotient_cases as mk
+    cases = _golden()["int8_quotient"]
+    assert len(cases) >= 3
+    caught = set()
+    for ex in cases:
+        x = np.array(ex["x"], dtype=np.float32).reshape(1, 1, 1, -1)
+        codes, scales = quantize_qk_int8(x)
+        assert codes.ravel().tolist() == ex["codes"], ex
+        assert scales.ravel().tolist() == [ex["scale"]], ex
+        amax, xv = ex["x"]
+        # the stored code is the exact-rational one, and each listed stand-in gives another
+        assert mk.int8_code(mk.variants(xv, amax, 127)["quotient"]) == ex["codes"][1]
+        alt = _stand_ins(xv, amax, 127)
+        for kind, code in ex["wrong"].items():
+            assert int(np.clip(np.rint(alt[kind]), -127, 127)) == code != ex["codes"][1]
+            caught.add(kind)
+    assert caught == set(mk.KINDS)
+
+
+def test_e4m3_quotient_cases():
+    import sys
+    sys.path.insert(0, GOLDEN)
+
+    import make_quant_quotient_cases as mk
+    cases = _golden()["e4m3_quotient"]
+    assert len(cases) >= 2
+    caught = set()
+    for ex in cases:
+        v = np.array(ex["v"], dtype=np.float32).reshape(1, 1, -1, 1)   # one channel, 2 tokens
+        codes, scales = quantize_v_fp8(v)
+        assert codes[0, 0, 0, :2].tolist() == ex["codes"], ex
+        assert scales.ravel().tolist() == [ex["scale"]], ex
+        amax, vv = ex["v"]
+        assert mk.e4m3_code(mk.variants(vv, amax, 448)["quotient"]) == ex["codes"][1]
+        alt = _stand_ins(vv, amax, 448)
+        for kind, code in ex["wrong"].items():
+            assert int(fp8_e4m3_encode(alt[kind])) == code != ex["codes"][1]
+            caught.add(kind)
+    assert caught == set(mk.KINDS)
+
+
+def test_quotient_cases_catch_a_reciprocal_quantiser():
+    # A quantiser that multiplies by RN(1/s) instead of dividing (a plausible slip)
+    # fails the quotient cases.
+    def int8_by_reciprocal(x):
+        x = np.asarray(x, dtype=np.float32)
+        s = np.float32(np.abs(x).max() / np.float32(127))
+        return np.clip(np.rint(x * np.float32(np.float32(1) / s)), -127, 127).astype(np.int64)
+    missed = [ex for ex in _golden()["int8_quotient"]
+              if int8_by_reciprocal(ex["x"]).tolist() != ex["codes"]]
+    assert missed, "the quotient cases do not tell division from a reciprocal multiply"
 
 
 def _finite_code_table():
