@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "device_once.h"
 #include "flash_fwd.cuh"
 #include "merge.cuh"
 #include "quant.cuh"
@@ -49,6 +50,9 @@ struct attn_ctx {
   unsigned* v_amax;
   unsigned* err;
   unsigned debug;
+  // Recorded on the caller's stream after the work of every call: attn_destroy
+  // waits for it (the context's last call) instead of the whole device.
+  cudaEvent_t done_ev;
   // attn_forward_host's pipeline, created by its first call: stream 0 carries the
   // host-to-device copies, 1 and 2 the kernels of even and odd ranges, 3 the
   // device-to-host copies.
@@ -113,10 +117,19 @@ bool make_pool_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uin
   return r == CUDA_SUCCESS;
 }
 
-template <typename K>
-bool set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-         cudaSuccess;
+// Raises the dynamic shared-memory limit of kernel `Kern` to `bytes` on the
+// current device, once per device: the attribute is per device, so each kernel
+// (one template instance of this function, hence one flag set, per kernel) keeps
+// a flag per device ordinal.
+template <auto Kern>
+bool set_smem(int bytes) {
+  static PerDeviceOnce<> once;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  return once.ensure(dev, [&] {
+    return cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+           cudaSuccess;
+  });
 }
 
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN>
@@ -124,9 +137,8 @@ attn_status launch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorM
                        const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                        cudaStream_t st) {
   using Cfg = FwdCfg<D, NQT, QUANT, SPLIT>;
-  auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN>;
-  static bool attr_ok = set_smem(kern, Cfg::kSmemBytes);
-  if (!attr_ok) return ATTN_ERR_CUDA;
+  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN>;
+  if (!set_smem<kern>(Cfg::kSmemBytes)) return ATTN_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -255,8 +267,7 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
 
 #define ATTN_QUANT_LAUNCH(DD, FF)                                                             \
   do {                                                                                        \
-    static bool qk_attr = set_smem(quant_qk_kernel<DD, FF>, QuantQkCfg<DD>::kSmemBytes);      \
-    if (!qk_attr) return ATTN_ERR_CUDA;                                                       \
+    if (!set_smem<quant_qk_kernel<DD, FF>>(QuantQkCfg<DD>::kSmemBytes)) return ATTN_ERR_CUDA;  \
     const int qk_ctas = QuantQkCfg<DD>::kCtasPerSm * c->num_sms;                              \
     if (nbq > 0) {                                                                            \
       const int tot = nbq * static_cast<int>(BHq);                                            \
@@ -269,8 +280,7 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
           kx, kc, ks, p.kv_len, nbk, tot, c->err, 0u);                                        \
       v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(            \
           vx, vamax, p.kv_len);                                                               \
-      static bool vq_attr = set_smem(v_quant_kernel<DD, FF>, VQuantCfg<DD>::kSmemBytes);      \
-      if (!vq_attr) return ATTN_ERR_CUDA;                                                     \
+      if (!set_smem<v_quant_kernel<DD, FF>>(VQuantCfg<DD>::kSmemBytes)) return ATTN_ERR_CUDA; \
       const int vq_ctas = std::min(tot, VQuantCfg<DD>::kCtasPerSm * c->num_sms);              \
       v_quant_kernel<DD, FF><<<vq_ctas, 256, VQuantCfg<DD>::kSmemBytes, st>>>(                \
           vx, vamax, vt, vs, p.kv_len, S_pad, nbk, tot, c->err);                              \
@@ -472,6 +482,12 @@ size_t d2h_piece_bytes(size_t out_per_unit, size_t in_per_unit) {
   return ratio <= 0.4 ? mib : ratio <= 0.6 ? 2 * mib : ratio <= 0.8 ? 4 * mib : 8 * mib;
 }
 
+// Marks the end of a call's work on `st` (everything it enqueued, errors included).
+attn_status mark_done(attn_ctx* c, attn_status s, cudaStream_t st) {
+  if (cudaEventRecord(c->done_ev, st) != cudaSuccess && s == ATTN_OK) return ATTN_ERR_CUDA;
+  return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -564,8 +580,14 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
     lpart_off = off;
     off += (2 * static_cast<size_t>(c->splits) * rows * 4 + 255) / 256 * 256;
   }
+  if (cudaEventCreateWithFlags(&c->done_ev, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    delete c;
+    return ATTN_ERR_CUDA;
+  }
   if (cudaMalloc(&c->ws, off) != cudaSuccess) {
     cudaGetLastError();
+    cudaEventDestroy(c->done_ev);
     delete c;
     return ATTN_ERR_OOM;
   }
@@ -577,6 +599,7 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   c->lse_part = split ? reinterpret_cast<float*>(base + lpart_off) : nullptr;
   if (cudaMemset(c->err, 0, 256) != cudaSuccess) {
     cudaFree(c->ws);
+    cudaEventDestroy(c->done_ev);
     delete c;
     return ATTN_ERR_CUDA;
   }
@@ -586,8 +609,13 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
 
 void attn_destroy(attn_ctx* c) {
   if (!c) return;
-  cudaDeviceSynchronize();
+  // Wait for the context's own work only: its last call, and the streams of the
+  // host pipeline.  (Other work on the device is not waited for here.)
+  cudaEventSynchronize(c->done_ev);
+  if (c->pipe_ready)
+    for (int i = 0; i < 4; ++i) cudaStreamSynchronize(c->pipe[i]);
   cudaFree(c->ws);
+  cudaEventDestroy(c->done_ev);
   if (c->pipe_ready) {
     for (int i = 0; i < 4; ++i) {
       cudaStreamDestroy(c->pipe[i]);
@@ -638,7 +666,8 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
   const bool need_q = c->p.q_len > 0, need_kv = c->p.kv_len > 0;
   if (bad_ptr(q, need_q) || bad_ptr(k, need_kv) || bad_ptr(v, need_kv) || bad_qbufs(c->p, qb))
     return ATTN_ERR_INVALID_ARG;
-  return quantize_units(c, 0, c->units, q, k, v, qb, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return mark_done(c, quantize_units(c, 0, c->units, q, k, v, qb, st), st);
 }
 
 attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* v,
@@ -646,14 +675,13 @@ attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* 
   if (!c) return ATTN_ERR_INVALID_ARG;
   const attn_status s = check_forward_buffers(c, q, k, v, qb, o, lse);
   if (s != ATTN_OK) return s;
-  return forward_units(c, 0, c->units, q, k, v, qb, o, lse, static_cast<cudaStream_t>(stream),
-                       0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return mark_done(c, forward_units(c, 0, c->units, q, k, v, qb, o, lse, st, 0), st);
 }
 
-attn_status attn_forward_paged(attn_ctx* c, const void* q, const void* k_pool,
-                               const void* v_pool, const int32_t* block_table, int num_blocks,
-                               void* o, float* lse, void* stream) {
-  if (!c) return ATTN_ERR_INVALID_ARG;
+static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_pool,
+                                      const void* v_pool, const int32_t* block_table,
+                                      int num_blocks, void* o, float* lse, void* stream) {
   const attn_params& p = c->p;
   if (p.precision != ATTN_EXACT) return ATTN_ERR_UNSUPPORTED;
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
@@ -719,11 +747,22 @@ attn_status attn_forward_paged(attn_ctx* c, const void* q, const void* k_pool,
   return f16 ? launch_merge<64, true>(c, o, lse, st) : launch_merge<64, false>(c, o, lse, st);
 }
 
-attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_host,
-                              const void* v_host, void* o_host, float* lse_host, void* q_dev,
-                              void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
-                              const attn_qbufs* qb, int chunks, void* stream) {
-  if (!c || chunks < 0 || chunks > kMaxHostChunks) return ATTN_ERR_INVALID_ARG;
+attn_status attn_forward_paged(attn_ctx* c, const void* q, const void* k_pool,
+                               const void* v_pool, const int32_t* block_table, int num_blocks,
+                               void* o, float* lse, void* stream) {
+  if (!c) return ATTN_ERR_INVALID_ARG;
+  return mark_done(c,
+                   forward_paged_impl(c, q, k_pool, v_pool, block_table, num_blocks, o, lse,
+                                      stream),
+                   static_cast<cudaStream_t>(stream));
+}
+
+static attn_status forward_host_impl(attn_ctx* c, const void* q_host, const void* k_host,
+                                     const void* v_host, void* o_host, float* lse_host,
+                                     void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                                     float* lse_dev, const attn_qbufs* qb, int chunks,
+                                     void* stream) {
+  if (chunks < 0 || chunks > kMaxHostChunks) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
   const bool quant = p.precision == ATTN_INT8QK_FP8PV;
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
@@ -808,6 +847,17 @@ attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_hos
   return ok ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_host,
+                              const void* v_host, void* o_host, float* lse_host, void* q_dev,
+                              void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                              const attn_qbufs* qb, int chunks, void* stream) {
+  if (!c) return ATTN_ERR_INVALID_ARG;
+  return mark_done(c,
+                   forward_host_impl(c, q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev,
+                                     v_dev, o_dev, lse_dev, qb, chunks, stream),
+                   static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -854,6 +904,7 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
                                                     float* lse, unsigned* err, void* stream) {
   attn_status st = validate(p);
   if (st != ATTN_OK) return st;
+  if (p->num_splits == 1) return ATTN_ERR_INVALID_ARG;  // always split: 0 or > 1
   if (p->precision != ATTN_EXACT) return ATTN_ERR_UNSUPPORTED;
   const bool need_q = p->q_len > 0, need_kv = p->kv_len > 0;
   auto bad = [](const void* ptr, bool needed) {

@@ -258,6 +258,46 @@ def oracle_sample_time(w: Workload, target_s=12.0, max_rows=None, seed=0):
     return flops, dt, desc, threads
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_single_thread():
+    """Whole calls of the oracle on one host thread: the tiny and decode workloads
+    (small enough to run in full).  Returns {name: {"ms": .., "tflops": ..}}."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attention_f64
+    from attention_forward_flash_b200.inputs import make_qkv
+    out = {}
+    with threadpool_limits(limits=1):
+        for name in ("tiny", "decode"):
+            w = WORKLOADS[name]
+            q, k, v = make_qkv(w)
+            run = lambda: attention_f64(q, k, v, causal=w.causal, start_pos=w.start_pos,  # noqa: E731
+                                        window_lo=w.window_lo, window_size=w.window_size)
+            run()
+            reps, t0 = 0, time.perf_counter()
+            while reps < 3 or time.perf_counter() - t0 < 1.0:
+                run()
+                reps += 1
+            ms = (time.perf_counter() - t0) * 1e3 / reps
+            out[name] = {"ms": ms, "tflops": work_flops(w) / (ms * 1e-3) / 1e12, "calls": reps}
+    return out
+
+
+def host_description(threads):
+    return {"threads_used": threads, "nproc": os.cpu_count(), "cpu_model": cpu_model()}
+
+
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
@@ -292,7 +332,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, args.precision),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "host": host_description(threads)},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -528,7 +568,9 @@ def run_native(args):
                                 "cores": threads, "kind": "oracle", "sample": desc,
                                 "seconds": dt,
                                 # the whole call at the sample's rate (linear in rows)
-                                "extrapolated_full_call_s": flops / (flops_s / dt)}
+                                "extrapolated_full_call_s": flops / (flops_s / dt),
+                                "host": host_description(threads),
+                                "single_thread_full_calls": oracle_single_thread()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -203,7 +203,11 @@ attn_status attn_forward_paged(attn_ctx *c, const void *q, const void *k_pool,
  * ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK. */
 attn_status attn_get_error(attn_ctx *c, void *stream);
 
-/* Frees the context's workspace (after synchronising the device). NULL is ignored. */
+/* Waits for the context's own work (its last call, recorded on that call's
+ * stream, and the streams of attn_forward_host's pipeline), then frees the
+ * workspace.  Work of other contexts or libraries on the device is not waited
+ * for by this call (the CUDA runtime's cudaFree may still synchronise the
+ * device).  NULL is ignored. */
 void attn_destroy(attn_ctx *c);
 
 /* Static string naming a status code. */
@@ -247,7 +251,8 @@ attn_status attn_debug_exp2(const float *x, float *y, size_t n, void *stream);
  * statistics (2 x splits x B x Hq x Sq).
  *
  * Arguments: as attn_forward, with `p` in place of a context; p->precision must
- * be ATTN_EXACT; p->num_splits 0 (library's choice) or > 1 (forced).  `err` is
+ * be ATTN_EXACT; p->num_splits 0 (library's choice) or > 1 (forced); 1 is
+ * rejected with ATTN_ERR_INVALID_ARG (this entry point always splits).  `err` is
  * an optional device word (4-byte aligned) into which a device-side wait that
  * runs out ORs 1; pass NULL to ignore such errors.  The array is shared by
  * every call: calls that overlap on the GPU (several streams, or several host
@@ -256,8 +261,8 @@ attn_status attn_debug_exp2(const float *x, float *y, size_t n, void *stream);
  * clearing between calls.  The first call on each device looks up the array's
  * device address (cudaGetSymbolAddress, with that device current); make that
  * first call before any stream capture.
- * Errors: ATTN_ERR_INVALID_ARG (bad field, NULL or misaligned pointer),
- * ATTN_ERR_UNSUPPORTED (quantised mode, head_dim, or partials larger than the
+ * Errors: ATTN_ERR_INVALID_ARG (bad field, num_splits 1, NULL or misaligned
+ * pointer), ATTN_ERR_UNSUPPORTED (quantised mode, head_dim, or partials larger than the
  * array; use attn_forward then), ATTN_ERR_CUDA (no sm_100 device, lookup,
  * tensor-map encode or launch failure). */
 attn_status attn_forward_splitkv_noalloc(const attn_params *p, const void *q, const void *k,

@@ -144,3 +144,70 @@ def test_header_is_plain_c_and_links_against_the_library(tmp_path):
                         "-Wl,--unresolved-symbols=ignore-in-shared-libs"],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_noalloc_rejects_one_split_before_any_device_call():
+    # The split-free entry always splits: num_splits must be 0 (library's choice) or > 1.
+    L = afb.lib()
+    p = _params(q_len=4, kv_len=4096, num_splits=1)
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: the call returns first
+    status = L.attn_forward_splitkv_noalloc(ctypes.byref(p), fake, fake, fake, fake, None, None,
+                                            None)
+    assert status == _abi.ATTN_ERR_INVALID_ARG
+
+
+DEVICE_ONCE_TEST = r"""
+#include <cstdio>
+#include <initializer_list>
+#include "device_once.h"
+
+int main() {
+  attn::PerDeviceOnce<8> once;
+  int calls[8] = {0};
+  bool fail_next = true;
+  auto setup = [&](int dev) {
+    return [&, dev] {
+      ++calls[dev];
+      if (dev == 3 && fail_next) { fail_next = false; return false; }
+      return true;
+    };
+  };
+  // The first use on each device runs the set-up; later uses on that device do not.
+  for (int rep = 0; rep < 3; ++rep)
+    for (int dev : {0, 1, 0, 2, 1}) if (!once.ensure(dev, setup(dev))) return 10 + dev;
+  if (calls[0] != 1 || calls[1] != 1 || calls[2] != 1) return 2;
+  // A failed set-up is not remembered: the next use on that device runs it again.
+  if (once.ensure(3, setup(3))) return 3;
+  if (once.done(3)) return 4;
+  if (!once.ensure(3, setup(3)) || calls[3] != 2 || !once.done(3)) return 5;
+  // Devices outside the table are refused without running the set-up.
+  int outside = 0;
+  if (once.ensure(8, [&] { ++outside; return true; }) || outside != 0) return 6;
+  if (once.ensure(-1, [&] { ++outside; return true; }) || outside != 0) return 7;
+  std::puts("ok");
+  return 0;
+}
+"""
+
+
+def test_kernel_attributes_are_kept_per_device(tmp_path):
+    """The flag behind every kernel's shared-memory attribute is keyed by device
+    ordinal: set-up runs once per device, failures are retried, and out-of-range
+    devices are refused (host logic, compiled with g++ against the library's header)."""
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no C++ compiler")
+    src = tmp_path / "device_once_test.cc"
+    src.write_text(DEVICE_ONCE_TEST)
+    exe = tmp_path / "device_once_test"
+    csrc = os.path.join(ROOT, "attention_forward_flash_b200", "csrc")
+    r = subprocess.run([gxx, "-std=c++17", "-Wall", "-Werror", "-I", csrc, str(src), "-o",
+                        str(exe), "-pthread"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout)
+    # and the library uses it for every launch that raises the shared-memory limit
+    api = open(os.path.join(csrc, "attn_api.cu")).read()
+    assert "PerDeviceOnce" in api and "static bool" not in api

@@ -373,3 +373,37 @@ def test_decode_qsa2_positions(ntok, pos0, W):
     ro, rl = oracle_for(w, q, k, v)
     check_exact(o, ro, str((ntok, pos0, W)))
     check_lse(lse, rl)
+
+
+# The lazy O correction of the exact mode: O and the row sums are rescaled only
+# when a row maximum grows by more than 8 (base-2 units) over the maximum in use.
+# Keys are built so that every 128-key tile raises each row's maximum by a set
+# amount G: K[j, 0] = g * (j // 128) + N(0, 1) with Q[i, 0] = 4, the other channels
+# small, so scale * log2(e) * 4 * g = G.  G = 7.5 stays under the threshold (the
+# stale maximum is kept and P reaches 2^7.5), G = 8.5 and G = 20 cross it on every
+# tile.  Single-pass kernel (head_dim 64 and 128) and split-KV kernel.
+def _ramp_inputs(D, Sq, Skv, G, seed):
+    g_ = torch.Generator().manual_seed(seed)
+    q = torch.randn(1, 2, Sq, D, generator=g_) * 0.25
+    k = torch.randn(1, 2, Skv, D, generator=g_) * 0.25
+    v = torch.randn(1, 2, Skv, D, generator=g_)
+    q[..., 0] = 4.0
+    step = G / (4.0 * (1.0 / math.sqrt(D)) * math.log2(math.e))
+    tile = torch.div(torch.arange(Skv), 128, rounding_mode="floor").float()
+    k[..., 0] = step * tile + torch.randn(1, 2, Skv, generator=g_)
+    return tuple(t.to(torch.bfloat16) for t in (q, k, v))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [7.5, 8.5, 20.0])
+@pytest.mark.parametrize("split", [False, True])
+def test_exact_rescale_forced(D, G, split):
+    Sq = 8 if split else 300          # few rows take the split-KV kernel
+    Skv = 10 * 128 + 37
+    q, k, v = _ramp_inputs(D, Sq, Skv, G, seed=int(7000 + 10 * G + D))
+    w = Workload("ramp", 1, 2, 2, Sq, Skv, D, "bf16", seed=0)
+    o, lse, att = run_gpu(w, q, k, v, num_splits=3 if split else 1)
+    assert (att.num_splits == 3) == split
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro, f"G={G}")
+    check_lse(lse, rl, f"G={G}")
