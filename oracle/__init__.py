@@ -17,6 +17,13 @@ from .attention import (  # noqa: F401
     visible_pairs,
     visible_range,
 )
+from .rope import (  # noqa: F401
+    apply_rope,
+    apply_rope_f32,
+    rope_frequencies,
+    rope_table,
+    yarn_attention_factor,
+)
 from .quant import (  # noqa: F401
     E4M3_MAX,
     QK_BLOCK,

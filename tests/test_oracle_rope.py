@@ -91,3 +91,98 @@ def test_yarn_ramp_limits():
                                plain, rtol=1e-15)
     assert yarn_attention_factor(1.0) == 1.0
     assert abs(yarn_attention_factor(math.e) - 1.1) < 1e-15
+
+
+# --- the float32 table and rotation (the form the quantised mode reproduces bit for bit)
+from fractions import Fraction  # noqa: E402
+
+from oracle.rope import apply_rope_f32, rope_table  # noqa: E402
+
+
+def _rn32(q):
+    """Exact rational rounded to the nearest float32 (ties to even), as a float."""
+    return float(np.float32(float(q))) if q == 0 else _rn32_exact(q)
+
+
+def _rn32_exact(q):
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (e - 23)
+    r = round(a / quantum) * quantum
+    return float(r if q > 0 else -r)
+
+
+def test_f32_rotation_hand_worked():
+    # exact values: a' = 1*0.5 - 2*0.25 = 0, b' = 1*0.25 + 2*0.5 = 1.25
+    table = np.zeros((4, 2, 1), dtype=np.float32)
+    table[3] = [[0.5], [0.25]]
+    out = apply_rope_f32(np.array([[1.0, 2.0]], np.float32), [3], table)
+    assert out.tolist() == [[0.0, 1.25]]
+    # position 0 with cos 1, sin 0 is the identity, channels past R pass through
+    table = rope_table(2, np.array([1.0, 0.5]))
+    x = np.arange(1, 7, dtype=np.float32)[None]
+    assert np.array_equal(apply_rope_f32(x, [0], table), x)
+
+
+def test_f32_rotation_rounds_each_product_and_the_sum():
+    # a, b, c, s chosen so that rounding each product before the subtraction gives
+    # another float32 than a fused a*c - RN(b*s); the expected value is worked with
+    # exact rationals.
+    rng = np.random.default_rng(4)
+    found = 0
+    for _ in range(20000):
+        a, b, c, s = (np.float32(v) for v in rng.standard_normal(4))
+        A, B, Cc, S = (Fraction(float(v)) for v in (a, b, c, s))
+        want = _rn32(Fraction(_rn32(A * Cc)) - Fraction(_rn32(B * S)))
+        fused = _rn32(A * Cc - Fraction(_rn32(B * S)))
+        if want == fused:
+            continue
+        table = np.array([[[c], [s]]], dtype=np.float32)
+        got = apply_rope_f32(np.array([[a, b]], np.float32), [0], table)[0, 0]
+        assert float(got) == want
+        found += 1
+        if found == 5:
+            break
+    assert found == 5
+
+
+@pytest.mark.parametrize("layout", ["half", "interleaved"])
+@pytest.mark.parametrize("R", [128, 64, 32])
+def test_f32_rotation_within_rounding_of_float64(layout, R):
+    rng = np.random.default_rng(R)
+    D, S = 128, 50
+    theta = rope_frequencies(R, scaling="yarn", factor=4.0, original_len=4096)
+    m = yarn_attention_factor(4.0) if R == D else 1.0
+    x = (rng.standard_normal((2, S, D)) * 3).astype(np.float32)
+    pos = rng.integers(0, 40000, S)
+    table = rope_table(40000, theta, mscale=m)
+    got = apply_rope_f32(x, pos, table, layout=layout).astype(np.float64)
+    ref = apply_rope(x.astype(np.float64), pos, theta, layout=layout, mscale=m)
+    if R < D:   # channels past R are unchanged
+        assert np.array_equal(got[..., R:], x[..., R:])
+    if layout == "half":
+        mag = np.concatenate([np.abs(x[..., :R // 2]) + np.abs(x[..., R // 2:R])] * 2, axis=-1)
+    else:
+        pair = np.abs(x[..., 0:R:2]) + np.abs(x[..., 1:R:2])
+        mag = np.repeat(pair, 2, axis=-1)
+    # table entries, two products and one sum each rounded once: < 4 ulps of |a| + |b|
+    assert np.all(np.abs(got[..., :R] - ref[..., :R]) <= 4 * 2.0 ** -24 * m * mag + 1e-30)
+
+
+def test_rope_table_obeys_the_angle_addition_formulas():
+    theta = rope_frequencies(64, base=10000.0)
+    t = rope_table(3000, theta).astype(np.float64)
+    rng = np.random.default_rng(5)
+    for p, q in rng.integers(0, 1500, (50, 2)):
+        c = t[p, 0] * t[q, 0] - t[p, 1] * t[q, 1]
+        s = t[p, 1] * t[q, 0] + t[p, 0] * t[q, 1]
+        np.testing.assert_allclose(c, t[p + q, 0], atol=2e-6)
+        np.testing.assert_allclose(s, t[p + q, 1], atol=2e-6)
+    np.testing.assert_allclose(t[:, 0] ** 2 + t[:, 1] ** 2, 1.0, atol=1e-6)
+    assert np.all(t[0, 0] == 1.0) and np.all(t[0, 1] == 0.0)
+    m = rope_table(10, theta, mscale=1.5).astype(np.float64)
+    np.testing.assert_allclose(m[:, 0] ** 2 + m[:, 1] ** 2, 2.25, rtol=1e-6)
