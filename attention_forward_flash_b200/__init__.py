@@ -15,6 +15,7 @@ from ._abi import (  # noqa: F401
     AttnError,
     AttnParams,
     AttnQBufs,
+    AttnRopeFreq,
     attn_create,
     attn_debug_set,
     attn_destroy,
@@ -28,4 +29,4 @@ from ._abi import (  # noqa: F401
     lib,
     lib_path,
 )
-from .api import Attention, DeviceStaging, QuantBuffers  # noqa: F401
+from .api import Attention, DeviceStaging, QuantBuffers, rope_table  # noqa: F401

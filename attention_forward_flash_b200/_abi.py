@@ -9,11 +9,12 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_OOM
     ATTN_ERR_TIMEOUT = range(6)
 ATTN_BF16, ATTN_FP16 = 0, 1
 ATTN_EXACT, ATTN_INT8QK_FP8PV = 0, 1
+ATTN_ROPE_PLAIN, ATTN_ROPE_NTK, ATTN_ROPE_YARN = 0, 1, 2
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
             "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host",
-            "attn_forward_paged")
+            "attn_forward_paged", "attn_rope_table", "attn_set_rope_table", "attn_rope_apply")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -27,7 +28,15 @@ class AttnParams(ctypes.Structure):
                 ("q_len", ctypes.c_int), ("kv_len", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("start_pos", ctypes.c_int), ("causal", ctypes.c_int), ("window_lo", ctypes.c_int),
                 ("scale", ctypes.c_float), ("dtype", ctypes.c_int), ("precision", ctypes.c_int),
-                ("num_splits", ctypes.c_int), ("window_size", ctypes.c_int)]
+                ("num_splits", ctypes.c_int), ("window_size", ctypes.c_int),
+                ("rope_dim", ctypes.c_int), ("rope_interleaved", ctypes.c_int),
+                ("rope_keys_rotated", ctypes.c_int)]
+
+
+class AttnRopeFreq(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_float), ("scaling", ctypes.c_int), ("factor", ctypes.c_float),
+                ("original_len", ctypes.c_int), ("beta_fast", ctypes.c_float),
+                ("beta_slow", ctypes.c_float)]
 
 
 class AttnQBufs(ctypes.Structure):
@@ -82,6 +91,12 @@ def lib():
         L.attn_forward_host.restype = c_int
         L.attn_forward_paged.argtypes = [vp, vp, vp, vp, vp, c_int, vp, vp, vp]
         L.attn_forward_paged.restype = c_int
+        L.attn_rope_table.argtypes = [c_int, c_int, ctypes.POINTER(AttnRopeFreq), vp]
+        L.attn_rope_table.restype = c_int
+        L.attn_set_rope_table.argtypes = [vp, vp, c_int]
+        L.attn_set_rope_table.restype = c_int
+        L.attn_rope_apply.argtypes = [vp, vp, vp, c_int, c_int, c_int, vp]
+        L.attn_rope_apply.restype = c_int
         _LIB = L
     return _LIB
 
@@ -152,3 +167,16 @@ def attn_forward_host(ctx, q_host, k_host, v_host, o_host, lse_host, q_dev, k_de
 def attn_forward_paged(ctx, q, k_pool, v_pool, block_table, num_blocks, o, lse, stream):
     _check(lib().attn_forward_paged(ctx, q, k_pool, v_pool, block_table, num_blocks, o, lse,
                                     stream), "attn_forward_paged")
+
+
+def attn_rope_table(rope_dim, n_pos, freq: AttnRopeFreq, table_host_ptr):
+    _check(lib().attn_rope_table(rope_dim, n_pos, ctypes.byref(freq), table_host_ptr),
+           "attn_rope_table")
+
+
+def attn_set_rope_table(ctx, table_dev_ptr, n_pos):
+    _check(lib().attn_set_rope_table(ctx, table_dev_ptr, n_pos), "attn_set_rope_table")
+
+
+def attn_rope_apply(ctx, x, y, n_heads, length, pos0, stream):
+    _check(lib().attn_rope_apply(ctx, x, y, n_heads, length, pos0, stream), "attn_rope_apply")

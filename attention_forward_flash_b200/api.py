@@ -10,7 +10,20 @@ from __future__ import annotations
 import torch
 
 from . import _abi
-from ._abi import (ATTN_BF16, ATTN_EXACT, ATTN_FP16, ATTN_INT8QK_FP8PV, AttnParams, AttnQBufs)
+from ._abi import (ATTN_BF16, ATTN_EXACT, ATTN_FP16, ATTN_INT8QK_FP8PV, ATTN_ROPE_NTK,
+                   ATTN_ROPE_PLAIN, ATTN_ROPE_YARN, AttnParams, AttnQBufs, AttnRopeFreq)
+
+_SCALINGS = {None: ATTN_ROPE_PLAIN, "ntk": ATTN_ROPE_NTK, "yarn": ATTN_ROPE_YARN}
+
+
+def rope_table(rope_dim, n_pos, *, base=10000.0, scaling=None, factor=1.0, original_len=0,
+               beta_fast=32.0, beta_slow=1.0):
+    """The library's cos/sin table (``attn_rope_table``) as a CPU float32 tensor
+    [n_pos, 2, rope_dim / 2]; ``scaling`` is None, "ntk" or "yarn"."""
+    t = torch.empty((n_pos, 2, rope_dim // 2), dtype=torch.float32)
+    f = AttnRopeFreq(base, _SCALINGS[scaling], factor, original_len, beta_fast, beta_slow)
+    _abi.attn_rope_table(rope_dim, n_pos, f, t.data_ptr())
+    return t
 
 _PRECISIONS = {"exact": ATTN_EXACT, "quant": ATTN_INT8QK_FP8PV}
 
@@ -59,7 +72,12 @@ class Attention:
 
     def __init__(self, batch, n_q_heads, n_kv_heads, q_len, kv_len, head_dim, *,
                  dtype=torch.bfloat16, causal=False, start_pos=0, window_lo=0, scale=0.0,
-                 precision="exact", num_splits=0, window_size=0):
+                 precision="exact", num_splits=0, window_size=0, rope_dim=0,
+                 rope_interleaved=False, rope_keys_rotated=False, rope_table=None):
+        """``rope_dim`` > 0 turns on RoPE over the first rope_dim channels; its
+        cos/sin table is ``rope_table`` (a float32 tensor [n_pos, 2, rope_dim / 2],
+        e.g. from ``rope_table()``; copied to the device if it is on the CPU) and
+        can also be given later with ``set_rope_table``."""
         if dtype not in (torch.bfloat16, torch.float16):
             raise ValueError("dtype must be torch.bfloat16 or torch.float16")
         self.dtype = dtype
@@ -67,8 +85,32 @@ class Attention:
         self.params = AttnParams(batch, n_q_heads, n_kv_heads, q_len, kv_len, head_dim, start_pos,
                                  int(bool(causal)), window_lo, float(scale),
                                  ATTN_FP16 if dtype == torch.float16 else ATTN_BF16,
-                                 _PRECISIONS[precision], num_splits, window_size)
+                                 _PRECISIONS[precision], num_splits, window_size, rope_dim,
+                                 int(bool(rope_interleaved)), int(bool(rope_keys_rotated)))
         self.ctx = _abi.attn_create(self.params)
+        self._rope_table = None
+        if rope_table is not None:
+            self.set_rope_table(rope_table)
+
+    def set_rope_table(self, table, device=None):
+        """Gives the context its RoPE table (kept alive by this object)."""
+        if table.dtype != torch.float32 or table.dim() != 3 or table.shape[1] != 2:
+            raise ValueError("rope table: expected float32 [n_pos, 2, rope_dim / 2]")
+        if not table.is_cuda:
+            dev = device if device is not None else torch.device("cuda",
+                                                                 torch.cuda.current_device())
+            table = table.to(dev)
+        table = table.contiguous()
+        _abi.attn_set_rope_table(self.ctx, table.data_ptr(), table.shape[0])
+        self._rope_table = table
+
+    def rope_apply(self, x, out=None, pos0=0, stream=None):
+        """RoPE of x [batch, heads, len, head_dim] (positions pos0 + t) through
+        ``attn_rope_apply``; ``out`` may be x itself."""
+        out = torch.empty_like(x) if out is None else out
+        _abi.attn_rope_apply(self.ctx, x.data_ptr(), out.data_ptr(), x.shape[1], x.shape[2], pos0,
+                             _stream_handle(stream))
+        return out
 
     @property
     def num_splits(self):

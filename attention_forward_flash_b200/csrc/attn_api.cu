@@ -50,6 +50,11 @@ struct attn_ctx {
   unsigned* v_amax;
   unsigned* err;
   unsigned debug;
+  // RoPE: the caller's cos/sin table (attn_set_rope_table) and, in the exact mode
+  // on unrotated keys, a buffer of K's size that receives the rotated keys.
+  const float* rope_table;
+  int rope_npos;
+  void* ws_k;
   // Recorded on the caller's stream after the work of every call: attn_destroy
   // waits for it (the context's last call) instead of the whole device.
   cudaEvent_t done_ev;
@@ -132,38 +137,52 @@ bool set_smem(int bytes) {
   });
 }
 
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN>
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE>
 attn_status launch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                        cudaStream_t st) {
   using Cfg = FwdCfg<D, NQT, QUANT, SPLIT>;
-  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN>;
+  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN, ROPE>;
   if (!set_smem<kern>(Cfg::kSmemBytes)) return ATTN_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool QUANT, bool F16, bool WIN>
+template <int D, bool QUANT, bool F16, bool WIN, bool ROPE>
 attn_status dispatch_win(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                          cudaStream_t st) {
   if (c->split_path)
-    return launch_fwd<D, 1, QUANT, F16, true, true, WIN>(c, tq, tk, tv, to, a, grid, st);
+    return launch_fwd<D, 1, QUANT, F16, true, true, WIN, ROPE>(c, tq, tk, tv, to, a, grid, st);
   // Exact mode keeps a second (float32) row sum only when the caller asks for lse
   // (the quantised mode's only sum is the float32 one).
   if constexpr (!QUANT) {
     if (a.lse != nullptr)
-      return launch_fwd<D, 2, QUANT, F16, false, true, WIN>(c, tq, tk, tv, to, a, grid, st);
+      return launch_fwd<D, 2, QUANT, F16, false, true, WIN, ROPE>(c, tq, tk, tv, to, a, grid, st);
   }
-  return launch_fwd<D, 2, QUANT, F16, false, false, WIN>(c, tq, tk, tv, to, a, grid, st);
+  return launch_fwd<D, 2, QUANT, F16, false, false, WIN, ROPE>(c, tq, tk, tv, to, a, grid, st);
 }
 
+template <int D, bool QUANT, bool F16, bool ROPE>
+attn_status dispatch_rope(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+                          cudaStream_t st) {
+  if (a.window_size > 0)
+    return dispatch_win<D, QUANT, F16, true, ROPE>(c, tq, tk, tv, to, a, grid, st);
+  return dispatch_win<D, QUANT, F16, false, ROPE>(c, tq, tk, tv, to, a, grid, st);
+}
+
+// Exact mode with RoPE: the variant that rotates the staged Q tile (the keys
+// arrive rotated); the quantised mode rotates in its quantiser.
 template <int D, bool QUANT, bool F16>
 attn_status dispatch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
                          cudaStream_t st) {
-  if (a.window_size > 0) return dispatch_win<D, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
-  return dispatch_win<D, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
+  if constexpr (!QUANT) {
+    if (a.rope_table != nullptr)
+      return dispatch_rope<D, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
+  }
+  return dispatch_rope<D, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
 }
 
 // The merge is a programmatic dependent launch of the split kernel: its launch
@@ -204,6 +223,10 @@ attn_status validate(const attn_params* p) {
   if (p->precision != ATTN_EXACT && p->precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
   if (p->num_splits < 0 || p->num_splits > kMergeMaxSplits) return ATTN_ERR_INVALID_ARG;
+  if (p->rope_dim < 0 || p->rope_dim % 16 != 0 || p->rope_dim > p->head_dim ||
+      (p->rope_interleaved != 0 && p->rope_interleaved != 1) ||
+      (p->rope_keys_rotated != 0 && p->rope_keys_rotated != 1))
+    return ATTN_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(p->n_q_heads / p->n_kv_heads) * p->q_len;
   if (rows > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
@@ -239,6 +262,78 @@ attn_status check_forward_buffers(const attn_ctx* c, const void* q, const void* 
   return ATTN_OK;
 }
 
+// y = RoPE(x) over `rows` rows of head_dim channels (row t of a head at position
+// pos0 + t % len), with the context's table and pair layout.
+attn_status launch_rope_apply(const attn_ctx* c, const void* x, void* y, long long rows, int len,
+                              int pos0, cudaStream_t st) {
+  const attn_params& p = c->p;
+  if (rows <= 0) return ATTN_OK;
+  const long long threads = rows * (p.head_dim / 8);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  if (p.dtype == ATTN_FP16)
+    rope_apply_kernel<true><<<blocks, 256, 0, st>>>(
+        static_cast<const uint16_t*>(x), static_cast<uint16_t*>(y), c->rope_table, rows, len,
+        p.head_dim, p.rope_dim, p.rope_interleaved, pos0);
+  else
+    rope_apply_kernel<false><<<blocks, 256, 0, st>>>(
+        static_cast<const uint16_t*>(x), static_cast<uint16_t*>(y), c->rope_table, rows, len,
+        p.head_dim, p.rope_dim, p.rope_interleaved, pos0);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Row tiles per head for the causal heaviest-band-first order of the single-pass
+// kernel (FwdArgs::tph), or 0 where it does not apply.
+int causal_band_tiles(const attn_ctx* c) {
+  const attn_params& p = c->p;
+  if (!p.causal || c->split_path || p.q_len % 256 != 0) return 0;
+  return p.q_len / 256;
+}
+
+// One Q/K quantiser launch over `tot` 128-token blocks (persistent grid).
+template <int D, bool F16, bool ROPE>
+attn_status quant_qk_launch(const attn_ctx* c, const uint16_t* x, int8_t* codes, float* scales,
+                            int S, int nblk, int tot, unsigned debug, const QuantRope& r,
+                            cudaStream_t st) {
+  using Cfg = QuantQkCfg<D, ROPE>;
+  if (!set_smem<quant_qk_kernel<D, F16, ROPE>>(Cfg::kSmemBytes)) return ATTN_ERR_CUDA;
+  const int ctas = std::min(tot, Cfg::kCtasPerSm * c->num_sms);
+  quant_qk_kernel<D, F16, ROPE><<<ctas, 256, Cfg::kSmemBytes, st>>>(x, codes, scales, S, nblk,
+                                                                     tot, c->err, debug, r);
+  return ATTN_OK;
+}
+
+// The quantisers of one range of units: Q and K blocks (rotated first with RoPE),
+// then V's channel maxima and codes.
+template <int D, bool F16>
+attn_status quant_launch(attn_ctx* c, const uint16_t* qx, int8_t* qc, float* qs,
+                         const uint16_t* kx, int8_t* kc, float* ks, const uint16_t* vx,
+                         unsigned* vamax, uint8_t* vt, float* vs, int nbq, int nbk, unsigned BHq,
+                         unsigned BHk, bool rope_q, bool rope_k, const QuantRope& rq,
+                         const QuantRope& rk, cudaStream_t st) {
+  const attn_params& p = c->p;
+  attn_status s = ATTN_OK;
+  if (nbq > 0) {
+    const int tot = nbq * static_cast<int>(BHq);
+    s = rope_q ? quant_qk_launch<D, F16, true>(c, qx, qc, qs, p.q_len, nbq, tot, c->debug, rq, st)
+               : quant_qk_launch<D, F16, false>(c, qx, qc, qs, p.q_len, nbq, tot, c->debug, rq,
+                                                st);
+    if (s != ATTN_OK) return s;
+  }
+  if (nbk > 0) {
+    const int tot = nbk * static_cast<int>(BHk);
+    s = rope_k ? quant_qk_launch<D, F16, true>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st)
+               : quant_qk_launch<D, F16, false>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st);
+    if (s != ATTN_OK) return s;
+    v_amax_kernel<D, F16><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(vx, vamax,
+                                                                               p.kv_len);
+    if (!set_smem<v_quant_kernel<D, F16>>(VQuantCfg<D>::kSmemBytes)) return ATTN_ERR_CUDA;
+    const int vq_ctas = std::min(tot, VQuantCfg<D>::kCtasPerSm * c->num_sms);
+    v_quant_kernel<D, F16><<<vq_ctas, 256, VQuantCfg<D>::kSmemBytes, st>>>(
+        vx, vamax, vt, vs, p.kv_len, nbk * 128, nbk, tot, c->err);
+  }
+  return ATTN_OK;
+}
+
 // Launches the quantisers on `st` for the units [u0, u0 + nu) (unit = one
 // (batch, kv head) pair with its query heads).  Pointers are those of the whole
 // problem, already validated.
@@ -265,39 +360,27 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
   float* vs = nbk > 0 ? qb->v_scale + static_cast<size_t>(u0) * D : nullptr;
   unsigned* vamax = nbk > 0 ? c->v_amax + static_cast<size_t>(u0) * D : nullptr;
 
-#define ATTN_QUANT_LAUNCH(DD, FF)                                                             \
-  do {                                                                                        \
-    if (!set_smem<quant_qk_kernel<DD, FF>>(QuantQkCfg<DD>::kSmemBytes)) return ATTN_ERR_CUDA;  \
-    const int qk_ctas = QuantQkCfg<DD>::kCtasPerSm * c->num_sms;                              \
-    if (nbq > 0) {                                                                            \
-      const int tot = nbq * static_cast<int>(BHq);                                            \
-      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
-          qx, qc, qs, p.q_len, nbq, tot, c->err, c->debug);                                   \
-    }                                                                                         \
-    if (nbk > 0) {                                                                            \
-      const int tot = nbk * static_cast<int>(BHk);                                            \
-      quant_qk_kernel<DD, FF><<<std::min(tot, qk_ctas), 256, QuantQkCfg<DD>::kSmemBytes, st>>>( \
-          kx, kc, ks, p.kv_len, nbk, tot, c->err, 0u);                                        \
-      v_amax_kernel<DD, FF><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(            \
-          vx, vamax, p.kv_len);                                                               \
-      if (!set_smem<v_quant_kernel<DD, FF>>(VQuantCfg<DD>::kSmemBytes)) return ATTN_ERR_CUDA; \
-      const int vq_ctas = std::min(tot, VQuantCfg<DD>::kCtasPerSm * c->num_sms);              \
-      v_quant_kernel<DD, FF><<<vq_ctas, 256, VQuantCfg<DD>::kSmemBytes, st>>>(                \
-          vx, vamax, vt, vs, p.kv_len, S_pad, nbk, tot, c->err);                              \
-    }                                                                                         \
-  } while (0)
-
   if (nbk > 0 &&
       cudaMemsetAsync(vamax, 0, static_cast<size_t>(nu) * D * 4, st) != cudaSuccess)
     return ATTN_ERR_CUDA;
+  // RoPE: Q rows at start_pos + token, K rows at token (unless already rotated)
+  const bool rope = p.rope_dim > 0;
+  const QuantRope rq{c->rope_table, p.rope_dim, p.rope_interleaved, p.start_pos};
+  const QuantRope rk{c->rope_table, p.rope_dim, p.rope_interleaved, 0};
+  const bool rope_k = rope && !p.rope_keys_rotated;
+  attn_status s = ATTN_OK;
   if (D == 128) {
-    if (f16) ATTN_QUANT_LAUNCH(128, true);
-    else ATTN_QUANT_LAUNCH(128, false);
+    s = f16 ? quant_launch<128, true>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
+                                      BHq, BHk, rope, rope_k, rq, rk, st)
+            : quant_launch<128, false>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
+                                       BHq, BHk, rope, rope_k, rq, rk, st);
   } else {
-    if (f16) ATTN_QUANT_LAUNCH(64, true);
-    else ATTN_QUANT_LAUNCH(64, false);
+    s = f16 ? quant_launch<64, true>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
+                                     BHq, BHk, rope, rope_k, rq, rk, st)
+            : quant_launch<64, false>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
+                                      BHq, BHk, rope, rope_k, rq, rk, st);
   }
-#undef ATTN_QUANT_LAUNCH
+  if (s != ATTN_OK) return s;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -339,6 +422,14 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
     q = static_cast<const uint16_t*>(q) + qe;
     k = static_cast<const uint16_t*>(k) + ke;
     v = static_cast<const uint16_t*>(v) + ke;
+    if (p.rope_dim > 0 && !p.rope_keys_rotated) {
+      // the range's keys, rotated once into the workspace (positions 0 .. kv_len-1)
+      uint16_t* kr = static_cast<uint16_t*>(c->ws_k) + ke;
+      const attn_status rs = launch_rope_apply(c, k, kr, static_cast<long long>(nu) * p.kv_len,
+                                               p.kv_len, 0, st);
+      if (rs != ATTN_OK) return rs;
+      k = kr;
+    }
   }
 
   // Tensor maps.  Q, O: [units][R][D]; K, V: [units][Skv][D]; V^T: [units][D][S_pad].
@@ -404,6 +495,12 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
   a.nblk_k = ceil_div(p.kv_len, 128);
   a.err = c->err;
   a.debug = c->debug;
+  if (!quant && p.rope_dim > 0) {
+    a.rope_table = c->rope_table;
+    a.rope_R = p.rope_dim;
+    a.rope_inter = p.rope_interleaved;
+  }
+  a.tph = causal_band_tiles(c);
   const int grid = nu * c->row_tiles * (c->split_path ? c->splits : 1);
 
   attn_status s;
@@ -487,6 +584,9 @@ attn_status mark_done(attn_ctx* c, attn_status s, cudaStream_t st) {
   if (cudaEventRecord(c->done_ev, st) != cudaSuccess && s == ATTN_OK) return ATTN_ERR_CUDA;
   return s;
 }
+
+// With RoPE the context needs its table before anything is launched.
+bool rope_ready(const attn_ctx* c) { return c->p.rope_dim == 0 || c->rope_table != nullptr; }
 
 }  // namespace
 
@@ -592,6 +692,16 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
     return ATTN_ERR_OOM;
   }
   c->ws_bytes = off;
+  if (p->rope_dim > 0 && !p->rope_keys_rotated && p->precision == ATTN_EXACT) {
+    const size_t kbytes = static_cast<size_t>(c->units) * p->kv_len * p->head_dim * 2;
+    if (kbytes > 0 && cudaMalloc(&c->ws_k, kbytes) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(c->ws);
+      cudaEventDestroy(c->done_ev);
+      delete c;
+      return ATTN_ERR_OOM;
+    }
+  }
   uint8_t* base = static_cast<uint8_t*>(c->ws);
   c->err = reinterpret_cast<unsigned*>(base);
   c->v_amax = vamax_off ? reinterpret_cast<unsigned*>(base + vamax_off) : nullptr;
@@ -599,6 +709,7 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   c->lse_part = split ? reinterpret_cast<float*>(base + lpart_off) : nullptr;
   if (cudaMemset(c->err, 0, 256) != cudaSuccess) {
     cudaFree(c->ws);
+    if (c->ws_k) cudaFree(c->ws_k);
     cudaEventDestroy(c->done_ev);
     delete c;
     return ATTN_ERR_CUDA;
@@ -615,6 +726,7 @@ void attn_destroy(attn_ctx* c) {
   if (c->pipe_ready)
     for (int i = 0; i < 4; ++i) cudaStreamSynchronize(c->pipe[i]);
   cudaFree(c->ws);
+  if (c->ws_k) cudaFree(c->ws_k);
   cudaEventDestroy(c->done_ev);
   if (c->pipe_ready) {
     for (int i = 0; i < 4; ++i) {
@@ -662,7 +774,7 @@ attn_status attn_get_error(attn_ctx* c, void* stream) {
 attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const void* v,
                              const attn_qbufs* qb, void* stream) {
   if (!c || !qb) return ATTN_ERR_INVALID_ARG;
-  if (c->p.precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
+  if (c->p.precision != ATTN_INT8QK_FP8PV || !rope_ready(c)) return ATTN_ERR_INVALID_ARG;
   const bool need_q = c->p.q_len > 0, need_kv = c->p.kv_len > 0;
   if (bad_ptr(q, need_q) || bad_ptr(k, need_kv) || bad_ptr(v, need_kv) || bad_qbufs(c->p, qb))
     return ATTN_ERR_INVALID_ARG;
@@ -672,7 +784,7 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
 
 attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* v,
                          const attn_qbufs* qb, void* o, float* lse, void* stream) {
-  if (!c) return ATTN_ERR_INVALID_ARG;
+  if (!c || !rope_ready(c)) return ATTN_ERR_INVALID_ARG;
   const attn_status s = check_forward_buffers(c, q, k, v, qb, o, lse);
   if (s != ATTN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -684,6 +796,8 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
                                       int num_blocks, void* o, float* lse, void* stream) {
   const attn_params& p = c->p;
   if (p.precision != ATTN_EXACT) return ATTN_ERR_UNSUPPORTED;
+  if (p.rope_dim > 0 && !p.rope_keys_rotated) return ATTN_ERR_UNSUPPORTED;  // pool keys rotated
+  if (!rope_ready(c)) return ATTN_ERR_INVALID_ARG;
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
   if (bad_ptr(q, need_q) || bad_ptr(o, need_q) || (lse && !aligned16(lse)) ||
       bad_ptr(k_pool, need_kv) || bad_ptr(v_pool, need_kv) ||
@@ -724,6 +838,12 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
   a.window_size = p.window_size;
   a.block_table = block_table;
   a.bt_stride = ceil_div(p.kv_len, 128);
+  a.tph = causal_band_tiles(c);
+  if (p.rope_dim > 0) {
+    a.rope_table = c->rope_table;
+    a.rope_R = p.rope_dim;
+    a.rope_inter = p.rope_interleaved;
+  }
   a.n_kv_heads = p.n_kv_heads;
   a.scale_log2 = c->scale * 1.4426950408889634f;
   a.lse = lse;
@@ -762,7 +882,7 @@ static attn_status forward_host_impl(attn_ctx* c, const void* q_host, const void
                                      void* q_dev, void* k_dev, void* v_dev, void* o_dev,
                                      float* lse_dev, const attn_qbufs* qb, int chunks,
                                      void* stream) {
-  if (chunks < 0 || chunks > kMaxHostChunks) return ATTN_ERR_INVALID_ARG;
+  if (chunks < 0 || chunks > kMaxHostChunks || !rope_ready(c)) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
   const bool quant = p.precision == ATTN_INT8QK_FP8PV;
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
@@ -847,6 +967,59 @@ static attn_status forward_host_impl(attn_ctx* c, const void* q_host, const void
   return ok ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+attn_status attn_rope_table(int rope_dim, int n_pos, const attn_rope_freq* f, float* table) {
+  if (!f || !table || rope_dim < 2 || rope_dim % 2 != 0 || n_pos < 1) return ATTN_ERR_INVALID_ARG;
+  if (!(f->base > 0.0f) || !(f->factor >= 1.0f)) return ATTN_ERR_INVALID_ARG;
+  if (f->scaling != ATTN_ROPE_PLAIN && f->scaling != ATTN_ROPE_NTK && f->scaling != ATTN_ROPE_YARN)
+    return ATTN_ERR_INVALID_ARG;
+  if (f->scaling == ATTN_ROPE_YARN && (f->original_len < 1 || !(f->beta_fast > f->beta_slow)))
+    return ATTN_ERR_INVALID_ARG;
+  const int half = rope_dim / 2;
+  const double R = rope_dim, s = f->factor;
+  double base = f->base;
+  if (f->scaling == ATTN_ROPE_NTK) base *= std::pow(s, R / (R - 2.0));
+  double m = 1.0;
+  if (f->scaling == ATTN_ROPE_YARN && s > 1.0) m = 0.1 * std::log(s) + 1.0;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int i = 0; i < half; ++i) {
+    double th = std::pow(base, -2.0 * i / R);
+    if (f->scaling == ATTN_ROPE_YARN) {
+      const double r = f->original_len * th / two_pi;
+      double g = (r - f->beta_slow) / (static_cast<double>(f->beta_fast) - f->beta_slow);
+      g = g < 0.0 ? 0.0 : (g > 1.0 ? 1.0 : g);
+      th = (1.0 - g) * th / s + g * th;
+    }
+    for (int p = 0; p < n_pos; ++p) {
+      const double ang = p * th;
+      table[static_cast<size_t>(p) * rope_dim + i] = static_cast<float>(std::cos(ang) * m);
+      table[static_cast<size_t>(p) * rope_dim + half + i] = static_cast<float>(std::sin(ang) * m);
+    }
+  }
+  return ATTN_OK;
+}
+
+attn_status attn_set_rope_table(attn_ctx* c, const float* table, int n_pos) {
+  if (!c || !table || !aligned16(table) || c->p.rope_dim == 0) return ATTN_ERR_INVALID_ARG;
+  const long long need = std::max<long long>(static_cast<long long>(c->p.start_pos) + c->p.q_len,
+                                             c->p.kv_len);
+  if (n_pos < 1 || n_pos < need) return ATTN_ERR_INVALID_ARG;
+  c->rope_table = table;
+  c->rope_npos = n_pos;
+  return ATTN_OK;
+}
+
+attn_status attn_rope_apply(attn_ctx* c, const void* x, void* y, int n_heads, int len, int pos0,
+                            void* stream) {
+  if (!c || c->p.rope_dim == 0 || !c->rope_table || n_heads < 1 || len < 0 || pos0 < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(pos0) + len > c->rope_npos) return ATTN_ERR_INVALID_ARG;
+  const bool any = len > 0;
+  if (bad_ptr(x, any) || bad_ptr(y, any)) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long rows = static_cast<long long>(c->p.batch) * n_heads * len;
+  return mark_done(c, launch_rope_apply(c, x, y, rows, len, pos0, st), st);
+}
+
 attn_status attn_forward_host(attn_ctx* c, const void* q_host, const void* k_host,
                               const void* v_host, void* o_host, float* lse_host, void* q_dev,
                               void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
@@ -905,7 +1078,7 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   attn_status st = validate(p);
   if (st != ATTN_OK) return st;
   if (p->num_splits == 1) return ATTN_ERR_INVALID_ARG;  // always split: 0 or > 1
-  if (p->precision != ATTN_EXACT) return ATTN_ERR_UNSUPPORTED;
+  if (p->precision != ATTN_EXACT || p->rope_dim != 0) return ATTN_ERR_UNSUPPORTED;
   const bool need_q = p->q_len > 0, need_kv = p->kv_len > 0;
   auto bad = [](const void* ptr, bool needed) {
     return needed ? (ptr == nullptr || !aligned16(ptr)) : (ptr != nullptr && !aligned16(ptr));

@@ -33,6 +33,7 @@
 #include <cuda_fp16.h>
 
 #include "ptx.cuh"
+#include "rope.cuh"
 
 namespace attn {
 
@@ -55,6 +56,11 @@ struct FwdArgs {
   const int* block_table;
   int bt_stride;
   int n_kv_heads;
+  // Causal, single-pass kernel, whole row tiles per head (q_len a multiple of 256):
+  // row tiles per head.  The grid then runs all row tiles of one position band
+  // (the band nearest the end of the sequence first) before the next band, across
+  // every unit and head, so the heaviest CTAs start first.  0: unit-major order.
+  int tph;
   float scale_log2;  // scale * log2(e)
   float* lse;        // [units * R] natural-log lse or nullptr (non-split variant)
   float* o_part;     // [splits, units, R, D] float32 (split variant)
@@ -67,6 +73,11 @@ struct FwdArgs {
   int nblk_k;
   unsigned* err;     // device error word
   unsigned debug;    // bit 0: skip the second key tile (timeout test)
+  // RoPE (exact mode, ROPE variant): the staged Q tile is rotated in shared
+  // memory before the first Q K^T; row r of a unit at position start_pos + r % Sq.
+  const float* rope_table;  // [n_pos][2][rope_R/2] float32
+  int rope_R;               // rotated channels (multiple of 16)
+  int rope_inter;           // interleaved pairs
 };
 
 constexpr int kErrTimeout = 1;
@@ -95,8 +106,8 @@ struct FwdCfg {
   static constexpr int kRingOff = kFixed;
   static constexpr int kBarOff = kRingOff + kNS * kSlot;
   // barriers: q_full, full[NS], empty[NS], s_ready[NQT], p_ready[NQT][2] (one per
-  // 64-key half of P), o_final
-  static constexpr int kNumBars = 1 + 2 * kNS + 3 * NQT + 1;
+  // 64-key half of P), o_final, q_rot (RoPE: the staged Q has been rotated)
+  static constexpr int kNumBars = 1 + 2 * kNS + 3 * NQT + 2;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;      // tmem base, abort flag
   static constexpr int kSvOff = kMiscOff + 16;                  // v scales (quant)
   static constexpr int kSmemBytes = kSvOff + (QUANT ? D * 4 : 0) + 1024;  // + alignment slack
@@ -229,11 +240,52 @@ __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 c
   }
 }
 
+// Rotates one row of a staged 16-bit Q tile in shared memory (RoPE): the tile is
+// 128 rows in boxes of 64 channels, 128-byte rows with 16-byte chunk k of row r
+// at chunk position k ^ (r & 7) (the TMA 128-byte swizzle).  Each chunk of the
+// first R channels is rotated with its partner chunk (rope.cuh); the half layout
+// handles both chunks of a pair at once.
+template <bool F16>
+__device__ __forceinline__ void rope_q_row(uint32_t tile, int row, const float* table, int R,
+                                           bool inter, int pos) {
+  auto addr = [&](int cj) {  // chunk cj (channels 8 cj .. 8 cj + 7) of this row
+    return tile + (cj >> 3) * (128 * 128) + row * 128 + (((cj & 7) ^ (row & 7)) << 4);
+  };
+  auto ld = [](uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+  };
+  auto st = [](uint32_t a, const uint4& v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+  };
+  const int n = inter ? R / 8 : R / 16;
+#pragma unroll 1
+  for (int cj = 0; cj < n; ++cj) {
+    const int pj = rope_partner(cj, R, inter);
+    const uint4 a = ld(addr(cj));
+    const uint4 b = inter ? a : ld(addr(pj));
+    float fa[8];
+    rope_chunk<F16>(a, b, cj, table, R, inter, pos, fa);
+    if (!inter) {
+      float fb[8];
+      rope_chunk<F16>(b, a, pj, table, R, false, pos, fb);
+      st(addr(pj), rope_pack8<F16>(fb));
+    }
+    st(addr(cj), rope_pack8<F16>(fa));
+  }
+}
+
 // LF: the kernel also keeps the float32 row sum for the log-sum-exp (exact mode;
 // needed by the split variant and when the caller asks for lse).  WIN: the
 // per-row sliding window (window_size) is applied; the kernels without it keep
-// the bounds they need in fewer registers.
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN>
+// the bounds they need in fewer registers.  ROPE (exact mode): the softmax
+// warpgroups rotate the staged Q tile before the first Q K^T (the keys arrive
+// rotated).
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE>
 __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
                                   FwdCfg<D, NQT, QUANT, SPLIT>::kCtasPerSm)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -242,6 +294,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
                      const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
   using C = FwdCfg<D, NQT, QUANT, SPLIT>;
   static_assert(!SPLIT || LF, "the split variant always needs the float32 row sum");
+  static_assert(!(ROPE && QUANT), "the quantised mode rotates Q and K in its quantiser");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -257,9 +310,17 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       split = lin % a.splits;
       lin /= a.splits;
     }
-    u = lin / a.row_tiles;
-    t = lin % a.row_tiles;
-    if (!SPLIT && a.causal) t = a.row_tiles - 1 - t;  // heaviest tiles of a unit first
+    if (!SPLIT && a.causal && a.tph > 0) {
+      const int per_band = a.units * a.G;  // row tiles of one position band
+      const int band = lin / per_band, rem = lin % per_band;
+      const int g = rem % a.G;             // heads of a unit adjacent: they share K/V
+      u = rem / a.G;
+      t = g * a.tph + (a.tph - 1 - band);
+    } else {
+      u = lin / a.row_tiles;
+      t = lin % a.row_tiles;
+      if (!SPLIT && a.causal) t = a.row_tiles - 1 - t;  // heaviest tiles of a unit first
+    }
   }
   const int BM = NQT * 128;
   const int r0 = t * BM;
@@ -299,6 +360,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
   auto s_ready = [&](int q) { return bar(1 + 2 * C::kNS + q); };
   auto p_ready = [&](int q, int h) { return bar(1 + 2 * C::kNS + NQT + 2 * q + h); };
   const uint32_t o_final = bar(1 + 2 * C::kNS + 3 * NQT);
+  const uint32_t q_rot = bar(2 + 2 * C::kNS + 3 * NQT);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   float* sv_smem = reinterpret_cast<float*>(smem + C::kSvOff);
@@ -315,6 +377,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       mbar_init(p_ready(q, 1), 4);
     }
     mbar_init(o_final, 1);
+    mbar_init(q_rot, 4 * NQT);  // one arrive per softmax warp
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -432,7 +495,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
           QUANT ? instr_desc(2, 1, 1, 0, 0, 128, 128) : instr_desc(1, fmt, fmt, 0, 0, 128, 128);
       constexpr uint32_t idesc_pv =
           QUANT ? instr_desc(1, 0, 0, 0, 0, 128, D) : instr_desc(1, fmt, fmt, 0, 1, 128, D);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+      bool ok = mbar_wait(ROPE ? q_rot : q_full, 0, abort_flag);
       if (!ok) raise();
       int it = 0;
 
@@ -569,6 +632,22 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     if constexpr (QUANT)
       if (n > 0) ksc_next = ld_global_f32(ksrc);
     constexpr int kPoly = QUANT ? kPolyEveryQ : kPolyEvery;
+    if constexpr (ROPE) {
+      // Rotate this thread's row of the staged Q tile, then hand the tile to the
+      // MMA warp (generic-proxy writes made visible to the tensor core first).
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
+      if (!ok) {
+        if (lane == 0) raise();
+      } else if (rvalid) {
+        constexpr int kQBox = 128 * 64 * 2;
+        static_assert(C::kQTile == (D / 64) * kQBox, "16-bit Q tile in 64-channel boxes");
+        rope_q_row<F16>(sbase + C::kQOff + q * C::kQTile, row, a.rope_table, a.rope_R,
+                        a.rope_inter != 0, pos);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_rot);
+    }
     // Quantised scores arrive as int32 s; adding 0x4B400000 to the bits gives the
     // float F = 1.5 * 2^23 + s exactly (|s| < 2^22).  The offset is removed in the
     // maximum and folded into the exponent's FMA: 2^(F * c - K) with
@@ -587,7 +666,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       __syncwarp();
       if (lane == 0) mbar_arrive(p_ready(q, h));
     };
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < n && ok; ++j) {
       const float ksc = ksc_next;
       if constexpr (QUANT)
         if (j + 1 < n) ksc_next = ld_global_f32(ksrc + j + 1);

@@ -17,6 +17,7 @@
 #include <cuda_fp16.h>
 
 #include "ptx.cuh"
+#include "rope.cuh"
 
 namespace attn {
 
@@ -83,20 +84,32 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 // shared memory; two buffers let the next block stream in while this one is
 // reduced and quantised, keeping HBM busy.  Waits are bounded: on a timeout the
 // CTA records kErrTimeout in `err` and stops.
-template <int D>
+//
+// With ROPE the block is rotated first (rope.cuh: float32 operations on the
+// table, token t of block b at position pos0 + 128 b + t): each thread rotates
+// its chunks (reading the partner chunk of the pairs from shared memory), keeps
+// the rotated floats in registers, and the maximum and the codes are those of
+// the rotated values.  The extra registers leave room for fewer CTAs per SM.
+template <int D, bool ROPE = false>
 struct QuantQkCfg {
   static constexpr int kBlockBytes = 128 * D * 2;
   static constexpr int kSmemBytes = 2 * kBlockBytes + 64 + 128;  // buffers, barriers, reduction
-  static constexpr int kCtasPerSm = D == 128 ? 3 : 6;
+  static constexpr int kCtasPerSm = D == 128 ? (ROPE ? 2 : 3) : (ROPE ? 3 : 6);
 };
 
-template <int D, bool F16>
-__global__ void __launch_bounds__(256, QuantQkCfg<D>::kCtasPerSm) quant_qk_kernel(const uint16_t* __restrict__ x,
-                                                       int8_t* __restrict__ codes,
-                                                       float* __restrict__ scales, int S,
-                                                       int nblk, int total, unsigned* err,
-                                                       unsigned debug) {
-  using C = QuantQkCfg<D>;
+// RoPE arguments of the quantiser (unused without ROPE).
+struct QuantRope {
+  const float* table;  // [n_pos][2][R/2] float32
+  int R;               // rotated channels
+  int inter;           // interleaved pairs
+  int pos0;            // position of token 0
+};
+
+template <int D, bool F16, bool ROPE = false>
+__global__ void __launch_bounds__(256, QuantQkCfg<D, ROPE>::kCtasPerSm) quant_qk_kernel(
+    const uint16_t* __restrict__ x, int8_t* __restrict__ codes, float* __restrict__ scales, int S,
+    int nblk, int total, unsigned* err, unsigned debug, QuantRope rope) {
+  using C = QuantQkCfg<D, ROPE>;
   constexpr int kChunks = 128 * D / 8;  // 16-byte chunks of a full block
   constexpr int kPer = kChunks / 256;
   extern __shared__ __align__(128) uint8_t qsm[];
@@ -145,16 +158,28 @@ __global__ void __launch_bounds__(256, QuantQkCfg<D>::kCtasPerSm) quant_qk_kerne
     const int nelem = min(128, S - t * 128) * D;
     const uint4* src = reinterpret_cast<const uint4*>(qsm + stage * C::kBlockBytes);
     uint4 w[kPer];
+    float rv[ROPE ? kPer : 1][8];  // rotated values (ROPE)
     float amax = 0.0f;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int c = threadIdx.x + k * 256;
       if (c * 8 < nelem) {
         w[k] = src[c];
-        float f[8];
-        unpack8<F16>(w[k], f);
+        if constexpr (ROPE) {
+          constexpr int kCpr = D / 8;  // chunks per token
+          const int tok = c / kCpr, cj = c % kCpr;
+          const int pj = rope_partner(cj, rope.R, rope.inter != 0);
+          const uint4 pw = src[tok * kCpr + pj];
+          rope_chunk<F16>(w[k], pw, cj, rope.table, rope.R, rope.inter != 0,
+                          rope.pos0 + t * 128 + tok, rv[k]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(rv[k][e]));
+        } else {
+          float f[8];
+          unpack8<F16>(w[k], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+        }
       } else {
         w[k] = make_uint4(0, 0, 0, 0);
       }
@@ -187,7 +212,12 @@ __global__ void __launch_bounds__(256, QuantQkCfg<D>::kCtasPerSm) quant_qk_kerne
       const int c = threadIdx.x + k * 256;
       if (c * 8 < nelem) {
         float f[8];
-        unpack8<F16>(w[k], f);
+        if constexpr (ROPE) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = rv[k][e];
+        } else {
+          unpack8<F16>(w[k], f);
+        }
         uint32_t bits[8];
         if (fast) {
 #pragma unroll

@@ -19,6 +19,9 @@ Shapes mirror the pages' workloads:
 * ``llm``: a causal GQA prefill with 1% of K entries scaled by 20.
 * ``llm_window``: the same shape with a per-row sliding window of 1024 positions
   (each query row sees the last 1024 keys up to its own).
+* ``video_rope`` / ``llm_rope``: the video and causal GQA prefill shapes with
+  rotary position embedding on all head_dim channels (the RoPE "inside the
+  kernel" planned in section "Планы · Rigsy Kernel" of the RTX 5080 page).
 * ``tiny``: a small exact case the oracle finishes in well under a second.
 
 Recipe: a CPU ``torch.Generator`` seeded with the workload's seed draws float32
@@ -54,6 +57,7 @@ class Workload:
     k_outlier_frac: float = 0.0         # fraction of K entries multiplied by k_outlier_mult
     k_outlier_mult: float = 1.0
     oracle_rows: int = 0                 # 0: every row; else a seeded subset per head
+    rope_dim: int = 0                    # rotary channels (0: no RoPE)
 
     @property
     def torch_dtype(self):
@@ -89,6 +93,11 @@ WORKLOADS = {
     "llm_window": Workload("llm_window", 4, 32, 8, 8192, 8192, 128, "bf16", causal=True,
                            window_size=1024, modes=("exact", "quant"), seed=1005,
                            oracle_rows=256),
+    # rotary position embedding on every channel (plain frequencies, base 10000)
+    "video_rope": Workload("video_rope", 1, 40, 40, 32760, 32760, 128, "bf16",
+                           modes=("exact", "quant"), seed=1006, oracle_rows=256, rope_dim=128),
+    "llm_rope": Workload("llm_rope", 4, 32, 8, 8192, 8192, 128, "bf16", causal=True,
+                         modes=("exact", "quant"), seed=1007, oracle_rows=256, rope_dim=128),
 }
 
 

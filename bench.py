@@ -175,16 +175,22 @@ class ClockSampler:
 
 
 def make_attention(w: Workload, precision):
-    from attention_forward_flash_b200 import Attention
+    from attention_forward_flash_b200 import Attention, rope_table
+    table = None
+    if w.rope_dim > 0:
+        table = rope_table(w.rope_dim, max(w.start_pos + w.q_len, w.kv_len))
     return Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
                      dtype=w.torch_dtype, causal=w.causal, start_pos=w.start_pos,
-                     window_lo=w.window_lo, precision=precision, window_size=w.window_size)
+                     window_lo=w.window_lo, precision=precision, window_size=w.window_size,
+                     rope_dim=w.rope_dim, rope_table=table)
 
 
 def launches_per_step(att, precision):
     n = 1 + (1 if att.num_splits > 1 else 0)
     if precision == "quant":
         n += 4  # Q and K block quantisers, V channel maxima, V quantiser
+    elif att.params.rope_dim > 0 and not att.params.rope_keys_rotated:
+        n += 1  # the keys' rotation pass
     return n
 
 
@@ -362,7 +368,8 @@ def workload_config(w: Workload, precision):
     return {"workload": w.name, "batch": w.batch, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "q_len": w.q_len, "kv_len": w.kv_len,
             "head_dim": w.head_dim, "causal": w.causal, "start_pos": w.start_pos,
-            "window_lo": w.window_lo, "window_size": w.window_size, "precision": precision,
+            "window_lo": w.window_lo, "window_size": w.window_size, "rope_dim": w.rope_dim,
+            "precision": precision,
             "input_dtype": w.dtype,
             "l2": (f"inputs {in_bytes / 1e9:.2f} GB > 126 MB L2" if in_bytes > L2_BYTES
                    else "L2 flushed before every timed call (256 MB written, then 256 MB read)"),
@@ -536,7 +543,8 @@ def run_native(args):
         for name, prec in (("video", "quant" if precision == "exact" else "exact"),
                            ("llm", "exact"), ("llm", "quant"), ("image", "exact"),
                            ("image", "quant"), ("decode", "exact"), ("decode_window", "exact"),
-                           ("llm_window", "exact")):
+                           ("llm_window", "exact"), ("video_rope", "exact"),
+                           ("video_rope", "quant"), ("llm_rope", "exact")):
             if name == w.name and prec == precision:
                 continue
             wx = WORKLOADS[name]

@@ -84,7 +84,35 @@ typedef struct {
   int num_splits;  /* key/value splits: 0 = chosen by the library, 1 = none, >1 = forced */
   int window_size; /* sliding window W >= 0: row i sees keys j >= start_pos + i - W + 1
                       (0: none); combined with window_lo, the larger bound applies */
+  /* Rotary position embedding (RoPE), applied to Q and K before Q K^T.  Planned
+   * "with NTK / YaRN scaling" inside the kernel instead of a separate pass on the
+   * page "Ядра attention на домашней RTX 5080", section "Планы · Rigsy Kernel".
+   * Query row i rotates by position start_pos + i, key j by position j, with the
+   * cos/sin table given by attn_set_rope_table (built by attn_rope_table). */
+  int rope_dim;          /* rotated channels R: 0 (no RoPE) or a multiple of 16 <= head_dim;
+                            channels R .. head_dim-1 are not rotated */
+  int rope_interleaved;  /* 0: channel i pairs with i + R/2; 1: channel 2i pairs with 2i + 1 */
+  int rope_keys_rotated; /* 1: k already holds rotated keys (a key cache written through
+                            attn_rope_apply); only q is rotated.  0: both are rotated */
 } attn_params;
+
+/* Frequencies of the rotary table: theta_i = base^(-2i/R), i < R/2.
+ *   ATTN_ROPE_PLAIN: as is.
+ *   ATTN_ROPE_NTK:   base becomes base * factor^(R / (R - 2)) (NTK-aware scaling).
+ *   ATTN_ROPE_YARN:  with r_i = original_len * theta_i / (2 pi) and the ramp
+ *                    g_i = clamp((r_i - beta_slow) / (beta_fast - beta_slow), 0, 1),
+ *                    theta_i becomes (1 - g_i) theta_i / factor + g_i theta_i, and
+ *                    cos and sin are multiplied by 0.1 ln(factor) + 1 (factor > 1). */
+typedef enum { ATTN_ROPE_PLAIN = 0, ATTN_ROPE_NTK = 1, ATTN_ROPE_YARN = 2 } attn_rope_scaling;
+
+typedef struct {
+  float base;        /* > 0, e.g. 10000 */
+  int scaling;       /* attn_rope_scaling */
+  float factor;      /* NTK / YaRN context-extension factor (>= 1; 1 = none) */
+  int original_len;  /* YaRN: the original context length */
+  float beta_fast;   /* YaRN ramp bounds (e.g. 32 and 1), beta_fast > beta_slow */
+  float beta_slow;
+} attn_rope_freq;
 
 /* Caller-owned device buffers of the quantised mode (all 16-byte aligned):
  *   q       int8   [B, Hq,  Sq,  D]          q_scale float [B, Hq,  ceil(Sq/128)]
@@ -104,8 +132,9 @@ typedef struct attn_ctx attn_ctx;
 
 /* Validates `p`, picks the kernel variant and the key/value split for the
  * current CUDA device, and allocates the context's workspace (split partial
- * results, the V channel maxima, the device error word).  On success *out
- * owns that workspace until attn_destroy().  Launches nothing.
+ * results, the V channel maxima, the device error word, and in the exact mode
+ * with RoPE on unrotated keys a buffer of K's size for the rotated keys).  On
+ * success *out owns that workspace until attn_destroy().  Launches nothing.
  * Errors: ATTN_ERR_INVALID_ARG (bad field or NULL), ATTN_ERR_UNSUPPORTED
  * (head_dim not 64/128), ATTN_ERR_CUDA (no device), ATTN_ERR_OOM. */
 attn_status attn_create(const attn_params *p, attn_ctx **out);
@@ -115,9 +144,11 @@ attn_status attn_create(const attn_params *p, attn_ctx **out);
  * block) s = max|x| / 127 and code = clamp(round_half_even(x / s), +-127), s = 0
  * for an all-zero block.  V: per (b, hkv, channel) s = max|v| / 448 and code =
  * E4M3(v / s) rounded to nearest-even and saturated.  Each step is one
- * correctly rounded float32 operation, so the bytes are reproducible.
+ * correctly rounded float32 operation, so the bytes are reproducible.  With
+ * RoPE, Q and K (K unless rope_keys_rotated) are rotated in float32 first and
+ * the codes are those of the rotated values.
  * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, context not in the
- * quantised mode), ATTN_ERR_CUDA (launch failure). */
+ * quantised mode, RoPE without a table), ATTN_ERR_CUDA (launch failure). */
 attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const void *v,
                              const attn_qbufs *qb, void *stream);
 
@@ -127,8 +158,10 @@ attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const vo
  * lse is not NULL, the natural-log sum of exp(scale * q.k) over each row's
  * visible keys.  Few-row (decode-shaped) problems are split along the keys and
  * merged by a second kernel into the same outputs.
+ * With RoPE (rope_dim > 0) the table must have been set (attn_set_rope_table).
  * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, qb presence not
- * matching the mode), ATTN_ERR_CUDA (tensor-map encode or launch failure). */
+ * matching the mode, RoPE without a table), ATTN_ERR_CUDA (tensor-map encode or
+ * launch failure). */
 attn_status attn_forward(attn_ctx *c, const void *q, const void *k, const void *v,
                          const attn_qbufs *qb, void *o, float *lse, void *stream);
 
@@ -198,6 +231,45 @@ attn_status attn_forward_paged(attn_ctx *c, const void *q, const void *k_pool,
                                const void *v_pool, const int32_t *block_table, int num_blocks,
                                void *o, float *lse, void *stream);
 
+/* Host-side RoPE table: table_host[p][0][i] = cos(p theta_i) * m and
+ * table_host[p][1][i] = sin(p theta_i) * m for p < n_pos, i < rope_dim / 2
+ * (float32, n_pos * rope_dim floats), with theta_i and the factor m from `f`
+ * (m = 1 except for YaRN).  Each entry is computed in double precision and
+ * rounded once.  Pure host arithmetic; copy the table to device memory and pass
+ * it to attn_set_rope_table.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL pointer, rope_dim not a positive even
+ * number, n_pos < 1, base <= 0, factor < 1, YaRN with beta_fast <= beta_slow or
+ * original_len < 1, unknown scaling). */
+attn_status attn_rope_table(int rope_dim, int n_pos, const attn_rope_freq *f, float *table_host);
+
+/* Gives a context with rope_dim > 0 its cos/sin table: a DEVICE pointer (16-byte
+ * aligned, caller-owned, valid while the context uses it) to float32
+ * [n_pos][2][rope_dim / 2] as attn_rope_table writes it.  n_pos must cover every
+ * position the context rotates: max(start_pos + q_len, kv_len) (and the
+ * positions passed to attn_rope_apply).  Launches nothing.
+ * How the rotation runs: in the quantised mode the Q/K quantiser rotates each
+ * block in float32 before taking its maximum (no extra pass: the codes are those
+ * of the rotated values, reproducible bit for bit).  In the exact mode the
+ * attention kernel rotates its staged Q tile in shared memory, and K (unless
+ * rope_keys_rotated) is rotated by a pass into the context's workspace before
+ * the kernel.  Rotated 16-bit values are rounded to nearest-even.  The rotation
+ * of a pair (a, b) with table entries (c, s) is a' = RN(RN(a c) - RN(b s)),
+ * b' = RN(RN(a s) + RN(b c)) in float32.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL context or table, misaligned table, the
+ * context has rope_dim 0, n_pos too small). */
+attn_status attn_set_rope_table(attn_ctx *c, const float *table_dev, int n_pos);
+
+/* Rotates x [batch, n_heads, len, head_dim] (the context's dtype, batch and
+ * head_dim; device memory) into y (same shape; y may equal x) with the
+ * context's table and pair layout; row t of every head sits at position
+ * pos0 + t.  For writing keys into a cache once, so that later forwards can run
+ * with rope_keys_rotated = 1.  Asynchronous on `stream`.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, n_heads < 1,
+ * len < 0, pos0 < 0, no table set, positions past the table),
+ * ATTN_ERR_CUDA (launch failure). */
+attn_status attn_rope_apply(attn_ctx *c, const void *x, void *y, int n_heads, int len, int pos0,
+                            void *stream);
+
 /* Synchronises `stream`, reads and clears the context's device error word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last call,
  * ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK. */
@@ -262,7 +334,7 @@ attn_status attn_debug_exp2(const float *x, float *y, size_t n, void *stream);
  * device address (cudaGetSymbolAddress, with that device current); make that
  * first call before any stream capture.
  * Errors: ATTN_ERR_INVALID_ARG (bad field, num_splits 1, NULL or misaligned
- * pointer), ATTN_ERR_UNSUPPORTED (quantised mode, head_dim, or partials larger than the
+ * pointer), ATTN_ERR_UNSUPPORTED (quantised mode, RoPE, head_dim, or partials larger than the
  * array; use attn_forward then), ATTN_ERR_CUDA (no sm_100 device, lookup,
  * tensor-map encode or launch failure). */
 attn_status attn_forward_splitkv_noalloc(const attn_params *p, const void *q, const void *k,

@@ -99,7 +99,7 @@ C_CALLER = r"""
 
 /* Every declared function, called with the argument types the header states. */
 int main(void) {
-  attn_params p = {1, 2, 2, 256, 256, 64, 0, 0, 0, 0.0f, ATTN_BF16, ATTN_EXACT, 0, 0};
+  attn_params p = {1, 2, 2, 256, 256, 64, 0, 0, 0, 0.0f, ATTN_BF16, ATTN_EXACT, 0, 0, 0, 0, 0};
   attn_ctx *c = NULL;
   attn_qbufs qb = {0};
   size_t sizes[6];
@@ -117,6 +117,11 @@ int main(void) {
   attn_debug_set(c, 0u);
   attn_debug_exp2(NULL, NULL, 0, NULL);
   attn_forward_splitkv_noalloc(&p, NULL, NULL, NULL, NULL, NULL, &err, NULL);
+  attn_rope_freq f = {10000.0f, ATTN_ROPE_YARN, 4.0f, 4096, 32.0f, 1.0f};
+  float rope[2 * 64];
+  attn_rope_table(64, 2, &f, rope);
+  attn_set_rope_table(c, NULL, 0);
+  attn_rope_apply(c, NULL, NULL, 1, 0, 0, NULL);
   (void)attn_status_string(ATTN_OK);
   attn_destroy(c);
   return 0;
