@@ -8,7 +8,7 @@ import os
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_OOM, \
     ATTN_ERR_TIMEOUT = range(6)
 ATTN_BF16, ATTN_FP16 = 0, 1
-ATTN_EXACT, ATTN_INT8QK_FP8PV = 0, 1
+ATTN_EXACT, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG = 0, 1, 2
 ATTN_ROPE_PLAIN, ATTN_ROPE_NTK, ATTN_ROPE_YARN = 0, 1, 2
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",

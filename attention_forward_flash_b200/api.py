@@ -10,7 +10,8 @@ from __future__ import annotations
 import torch
 
 from . import _abi
-from ._abi import (ATTN_BF16, ATTN_EXACT, ATTN_FP16, ATTN_INT8QK_FP8PV, ATTN_ROPE_NTK,
+from ._abi import (ATTN_BF16, ATTN_EXACT, ATTN_FP16, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG,
+                   ATTN_ROPE_NTK,
                    ATTN_ROPE_PLAIN, ATTN_ROPE_YARN, AttnParams, AttnQBufs, AttnRopeFreq)
 
 _SCALINGS = {None: ATTN_ROPE_PLAIN, "ntk": ATTN_ROPE_NTK, "yarn": ATTN_ROPE_YARN}
@@ -25,7 +26,8 @@ def rope_table(rope_dim, n_pos, *, base=10000.0, scaling=None, factor=1.0, origi
     _abi.attn_rope_table(rope_dim, n_pos, f, t.data_ptr())
     return t
 
-_PRECISIONS = {"exact": ATTN_EXACT, "quant": ATTN_INT8QK_FP8PV}
+# "mixed": the quantised mode with 16-bit Q K^T on the causal diagonal band tiles
+_PRECISIONS = {"exact": ATTN_EXACT, "quant": ATTN_INT8QK_FP8PV, "mixed": ATTN_MIXED_DIAG}
 
 
 def _stream_handle(stream):
@@ -128,8 +130,8 @@ class Attention:
                                  f"{shape}, got {t.dtype} {tuple(t.shape)} on {t.device}")
 
     def quantize(self, q, k, v, qbufs=None, stream=None):
-        if self.precision != "quant":
-            raise ValueError("quantize() needs precision='quant'")
+        if self.precision not in ("quant", "mixed"):
+            raise ValueError("quantize() needs precision='quant' or 'mixed'")
         self._check_inputs(q, k, v)
         qbufs = qbufs if qbufs is not None else QuantBuffers(self.params, q.device)
         _abi.attn_quantize_qk(self.ctx, q.data_ptr(), k.data_ptr(), v.data_ptr(), qbufs.struct(),
@@ -151,6 +153,12 @@ class Attention:
             if qbufs is None:
                 qbufs = self.quantize(q, k, v, stream=stream)
             _abi.attn_forward(self.ctx, None, None, None, qbufs.struct(), out.data_ptr(), lse_ptr, st)
+        elif self.precision == "mixed":   # the band tiles read the 16-bit q and k
+            self._check_inputs(q, k, v)
+            if qbufs is None:
+                qbufs = self.quantize(q, k, v, stream=stream)
+            _abi.attn_forward(self.ctx, q.data_ptr(), k.data_ptr(), None, qbufs.struct(),
+                              out.data_ptr(), lse_ptr, st)
         else:
             self._check_inputs(q, k, v)
             _abi.attn_forward(self.ctx, q.data_ptr(), k.data_ptr(), v.data_ptr(), None,
@@ -212,7 +220,7 @@ class Attention:
             if cached is None or (want_lse and cached.lse is None):
                 dev = (device if device is not None
                        else torch.device("cuda", torch.cuda.current_device()))
-                cached = DeviceStaging(p, self.dtype, dev, self.precision == "quant", want_lse)
+                cached = DeviceStaging(p, self.dtype, dev, self.precision != "exact", want_lse)
                 self._staging = cached
             staging = cached
         if out is None:

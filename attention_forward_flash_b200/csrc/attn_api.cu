@@ -23,11 +23,17 @@ constexpr int kMaxHostChunks = 64;  // ranges of units of one attn_forward_host 
 
 // Tensor maps of one launch, kept with the base pointers and unit count they were
 // encoded for: a later launch on the same buffers reuses them.
+// The tensor maps of one attention launch: Q, K, V (or their INT8 / E4M3 codes),
+// O, and in the diagonal band mode the 16-bit Q and K (else unused copies).
+struct FwdMaps {
+  CUtensorMap q, k, v, o, q16, k16;
+};
+
 struct MapCache {
   bool valid;
-  const void* key[4];  // Q, K, V (or their INT8/E4M3 codes) and O of the launch
+  const void* key[6];  // the base pointers the maps were encoded for
   int nu;
-  CUtensorMap tq, tk, tv, to;
+  FwdMaps m;
 };
 }  // namespace
 
@@ -137,52 +143,54 @@ bool set_smem(int bytes) {
   });
 }
 
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE>
-attn_status launch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
-                       const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
+          bool DIAG = false>
+attn_status launch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
                        cudaStream_t st) {
-  using Cfg = FwdCfg<D, NQT, QUANT, SPLIT>;
-  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN, ROPE>;
+  using Cfg = FwdCfg<D, NQT, QUANT, SPLIT, DIAG>;
+  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN, ROPE, DIAG>;
   if (!set_smem<kern>(Cfg::kSmemBytes)) return ATTN_ERR_CUDA;
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(m.q, m.k, m.v, m.o, m.q16, m.k16, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, bool QUANT, bool F16, bool WIN, bool ROPE>
-attn_status dispatch_win(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
-                         const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+attn_status dispatch_win(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
                          cudaStream_t st) {
+  // the diagonal band mode: single-pass quantised kernel with 16-bit band tiles
+  if constexpr (QUANT) {
+    if (c->p.precision == ATTN_MIXED_DIAG)
+      return launch_fwd<D, 2, true, F16, false, false, WIN, false, true>(c, m, a, grid, st);
+  }
   if (c->split_path)
-    return launch_fwd<D, 1, QUANT, F16, true, true, WIN, ROPE>(c, tq, tk, tv, to, a, grid, st);
+    return launch_fwd<D, 1, QUANT, F16, true, true, WIN, ROPE>(c, m, a, grid, st);
   // Exact mode keeps a second (float32) row sum only when the caller asks for lse
   // (the quantised mode's only sum is the float32 one).
   if constexpr (!QUANT) {
     if (a.lse != nullptr)
-      return launch_fwd<D, 2, QUANT, F16, false, true, WIN, ROPE>(c, tq, tk, tv, to, a, grid, st);
+      return launch_fwd<D, 2, QUANT, F16, false, true, WIN, ROPE>(c, m, a, grid, st);
   }
-  return launch_fwd<D, 2, QUANT, F16, false, false, WIN, ROPE>(c, tq, tk, tv, to, a, grid, st);
+  return launch_fwd<D, 2, QUANT, F16, false, false, WIN, ROPE>(c, m, a, grid, st);
 }
 
 template <int D, bool QUANT, bool F16, bool ROPE>
-attn_status dispatch_rope(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
-                          const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+attn_status dispatch_rope(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
                           cudaStream_t st) {
   if (a.window_size > 0)
-    return dispatch_win<D, QUANT, F16, true, ROPE>(c, tq, tk, tv, to, a, grid, st);
-  return dispatch_win<D, QUANT, F16, false, ROPE>(c, tq, tk, tv, to, a, grid, st);
+    return dispatch_win<D, QUANT, F16, true, ROPE>(c, m, a, grid, st);
+  return dispatch_win<D, QUANT, F16, false, ROPE>(c, m, a, grid, st);
 }
 
 // Exact mode with RoPE: the variant that rotates the staged Q tile (the keys
 // arrive rotated); the quantised mode rotates in its quantiser.
 template <int D, bool QUANT, bool F16>
-attn_status dispatch_fwd(const attn_ctx* c, const CUtensorMap& tq, const CUtensorMap& tk,
-                         const CUtensorMap& tv, const CUtensorMap& to, const FwdArgs& a, int grid,
+attn_status dispatch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
                          cudaStream_t st) {
   if constexpr (!QUANT) {
     if (a.rope_table != nullptr)
-      return dispatch_rope<D, QUANT, F16, true>(c, tq, tk, tv, to, a, grid, st);
+      return dispatch_rope<D, QUANT, F16, true>(c, m, a, grid, st);
   }
-  return dispatch_rope<D, QUANT, F16, false>(c, tq, tk, tv, to, a, grid, st);
+  return dispatch_rope<D, QUANT, F16, false>(c, m, a, grid, st);
 }
 
 // The merge is a programmatic dependent launch of the split kernel: its launch
@@ -220,7 +228,12 @@ attn_status validate(const attn_params* p) {
     return ATTN_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_INVALID_ARG;
-  if (p->precision != ATTN_EXACT && p->precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_INVALID_ARG;
+  if (p->precision != ATTN_EXACT && p->precision != ATTN_INT8QK_FP8PV &&
+      p->precision != ATTN_MIXED_DIAG)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->precision == ATTN_MIXED_DIAG && p->num_splits > 1) return ATTN_ERR_INVALID_ARG;
+  // the band tiles read the caller's 16-bit Q and K, which the quantiser's RoPE never sees
+  if (p->precision == ATTN_MIXED_DIAG && p->rope_dim > 0) return ATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
   if (p->num_splits < 0 || p->num_splits > kMergeMaxSplits) return ATTN_ERR_INVALID_ARG;
   if (p->rope_dim < 0 || p->rope_dim % 16 != 0 || p->rope_dim > p->head_dim ||
@@ -252,7 +265,9 @@ attn_status check_forward_buffers(const attn_ctx* c, const void* q, const void* 
   const attn_params& p = c->p;
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
   if (bad_ptr(o, need_q) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
-  if (p.precision == ATTN_INT8QK_FP8PV) {
+  if (p.precision == ATTN_MIXED_DIAG) {  // codes and the 16-bit Q and K
+    if (bad_qbufs(p, qb) || bad_ptr(q, need_q) || bad_ptr(k, need_kv)) return ATTN_ERR_INVALID_ARG;
+  } else if (p.precision == ATTN_INT8QK_FP8PV) {
     if (bad_qbufs(p, qb)) return ATTN_ERR_INVALID_ARG;
   } else {
     if (qb) return ATTN_ERR_INVALID_ARG;
@@ -392,7 +407,8 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
                           cudaStream_t st, int slot) {
   if (c->split_path && (u0 != 0 || nu != c->units)) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
-  const bool quant = p.precision == ATTN_INT8QK_FP8PV;
+  const bool quant = p.precision != ATTN_EXACT;        // INT8/FP8 codes (both quantised modes)
+  const bool diag = p.precision == ATTN_MIXED_DIAG;    // plus 16-bit Q, K for the band tiles
   const int D = p.head_dim;
   const bool f16 = p.dtype == ATTN_FP16;
   const size_t rows = static_cast<size_t>(nu) * c->R;
@@ -418,11 +434,12 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
     qo.v_t = qb->v_t + static_cast<size_t>(u0) * D * (static_cast<size_t>(nbk) * 128);
     qo.v_scale = qb->v_scale + static_cast<size_t>(u0) * D;
     qb = &qo;
-  } else {
+  }
+  if (!quant || diag) {
     q = static_cast<const uint16_t*>(q) + qe;
     k = static_cast<const uint16_t*>(k) + ke;
-    v = static_cast<const uint16_t*>(v) + ke;
-    if (p.rope_dim > 0 && !p.rope_keys_rotated) {
+    if (!quant) v = static_cast<const uint16_t*>(v) + ke;
+    if (!quant && p.rope_dim > 0 && !p.rope_keys_rotated) {
       // the range's keys, rotated once into the workspace (positions 0 .. kv_len-1)
       uint16_t* kr = static_cast<uint16_t*>(c->ws_k) + ke;
       const attn_status rs = launch_rope_apply(c, k, kr, static_cast<long long>(nu) * p.kv_len,
@@ -437,35 +454,44 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
       f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t R = c->R, Sk = p.kv_len, U = nu;
   MapCache& mc = c->maps[slot];
-  const void* key[4] = {quant ? static_cast<const void*>(qb->q) : q,
+  const void* key[6] = {quant ? static_cast<const void*>(qb->q) : q,
                         quant ? static_cast<const void*>(qb->k) : k,
-                        quant ? static_cast<const void*>(qb->v_t) : v, o};
-  const bool hit = mc.valid && mc.nu == nu && mc.key[0] == key[0] && mc.key[1] == key[1] &&
-                   mc.key[2] == key[2] && mc.key[3] == key[3];
-  CUtensorMap& tq = mc.tq;
-  CUtensorMap& tk = mc.tk;
-  CUtensorMap& tv = mc.tv;
-  CUtensorMap& to = mc.to;
+                        quant ? static_cast<const void*>(qb->v_t) : v, o,
+                        diag ? q : nullptr, diag ? k : nullptr};
+  bool hit = mc.valid && mc.nu == nu;
+  for (int i = 0; i < 6; ++i) hit = hit && mc.key[i] == key[i];
+  FwdMaps& m = mc.m;
   bool ok = true;
   if (hit) {
   } else if (quant) {
     const CUtensorMapSwizzle sw8 =
         D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const uint64_t S_pad = static_cast<uint64_t>(ceil_div(p.kv_len, 128)) * 128;
-    ok &= make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, D, R, U, D, R * D, D, 128, sw8);
-    ok &= make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, D, Sk, U, D, Sk * D, D, 128, sw8);
-    ok &= make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->v_t, S_pad, D, U, S_pad, S_pad * D, 128,
-                   D, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, D, R, U, D, R * D, D, 128, sw8);
+    ok &= make_map(&m.k, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, D, Sk, U, D, Sk * D, D, 128, sw8);
+    ok &= make_map(&m.v, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->v_t, S_pad, D, U, S_pad, S_pad * D,
+                   128, D, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (diag) {
+      ok &= make_map(&m.q16, t16, q, D, R, U, D * 2, R * D * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&m.k16, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+      m.q16 = m.q;
+      m.k16 = m.k;
+    }
   } else {
-    ok &= make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&m.q, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&m.k, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&m.v, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    m.q16 = m.q;
+    m.k16 = m.k;
   }
   if (!hit) {
-    ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map(&m.o, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     mc.valid = ok;
     mc.nu = nu;
-    for (int i = 0; i < 4; ++i) mc.key[i] = key[i];
+    for (int i = 0; i < 6; ++i) mc.key[i] = key[i];
   }
   if (!ok) return ATTN_ERR_CUDA;
 
@@ -505,15 +531,15 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
 
   attn_status s;
   if (D == 128) {
-    if (quant) s = f16 ? dispatch_fwd<128, true, true>(c, tq, tk, tv, to, a, grid, st)
-                       : dispatch_fwd<128, true, false>(c, tq, tk, tv, to, a, grid, st);
-    else s = f16 ? dispatch_fwd<128, false, true>(c, tq, tk, tv, to, a, grid, st)
-                 : dispatch_fwd<128, false, false>(c, tq, tk, tv, to, a, grid, st);
+    if (quant) s = f16 ? dispatch_fwd<128, true, true>(c, m, a, grid, st)
+                       : dispatch_fwd<128, true, false>(c, m, a, grid, st);
+    else s = f16 ? dispatch_fwd<128, false, true>(c, m, a, grid, st)
+                 : dispatch_fwd<128, false, false>(c, m, a, grid, st);
   } else {
-    if (quant) s = f16 ? dispatch_fwd<64, true, true>(c, tq, tk, tv, to, a, grid, st)
-                       : dispatch_fwd<64, true, false>(c, tq, tk, tv, to, a, grid, st);
-    else s = f16 ? dispatch_fwd<64, false, true>(c, tq, tk, tv, to, a, grid, st)
-                 : dispatch_fwd<64, false, false>(c, tq, tk, tv, to, a, grid, st);
+    if (quant) s = f16 ? dispatch_fwd<64, true, true>(c, m, a, grid, st)
+                       : dispatch_fwd<64, true, false>(c, m, a, grid, st);
+    else s = f16 ? dispatch_fwd<64, false, true>(c, m, a, grid, st)
+                 : dispatch_fwd<64, false, false>(c, m, a, grid, st);
   }
   if (s != ATTN_OK) return s;
   if (c->split_path) {
@@ -649,7 +675,9 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   const int big_ctas = c->units * ceil_div(c->R, 256);
   bool split = false;
   int splits = 1;
-  if (p->num_splits > 1) {
+  if (p->precision == ATTN_MIXED_DIAG) {
+    // single-pass kernel only (the band mode has no split-KV variant)
+  } else if (p->num_splits > 1) {
     split = true;
     splits = p->num_splits;
   } else if (p->num_splits == 0) {
@@ -669,7 +697,7 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   // workspace: error word | V channel maxima | split partials
   size_t off = 256;
   size_t vamax_off = 0, opart_off = 0, lpart_off = 0;
-  if (p->precision == ATTN_INT8QK_FP8PV) {
+  if (p->precision != ATTN_EXACT) {
     vamax_off = off;
     off += (static_cast<size_t>(c->units) * p->head_dim * 4 + 255) / 256 * 256;
   }
@@ -774,7 +802,7 @@ attn_status attn_get_error(attn_ctx* c, void* stream) {
 attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const void* v,
                              const attn_qbufs* qb, void* stream) {
   if (!c || !qb) return ATTN_ERR_INVALID_ARG;
-  if (c->p.precision != ATTN_INT8QK_FP8PV || !rope_ready(c)) return ATTN_ERR_INVALID_ARG;
+  if (c->p.precision == ATTN_EXACT || !rope_ready(c)) return ATTN_ERR_INVALID_ARG;
   const bool need_q = c->p.q_len > 0, need_kv = c->p.kv_len > 0;
   if (bad_ptr(q, need_q) || bad_ptr(k, need_kv) || bad_ptr(v, need_kv) || bad_qbufs(c->p, qb))
     return ATTN_ERR_INVALID_ARG;
@@ -817,11 +845,13 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
   const CUtensorMapDataType t16 =
       f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t R = c->R, U = c->units;
-  CUtensorMap tq, tk, tv, to;
-  bool ok = make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_pool_map(&tk, t16, k_pool, D, p.n_kv_heads, num_blocks);
-  ok &= make_pool_map(&tv, t16, v_pool, D, p.n_kv_heads, num_blocks);
-  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  FwdMaps m;
+  bool ok = make_map(&m.q, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_pool_map(&m.k, t16, k_pool, D, p.n_kv_heads, num_blocks);
+  ok &= make_pool_map(&m.v, t16, v_pool, D, p.n_kv_heads, num_blocks);
+  ok &= make_map(&m.o, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  m.q16 = m.q;
+  m.k16 = m.k;
   if (!ok) return ATTN_ERR_CUDA;
   FwdArgs a{};
   a.R = c->R;
@@ -856,11 +886,11 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
   const int grid = c->units * c->row_tiles * (c->split_path ? c->splits : 1);
   attn_status s;
   if (D == 128)
-    s = f16 ? dispatch_fwd<128, false, true>(c, tq, tk, tv, to, a, grid, st)
-            : dispatch_fwd<128, false, false>(c, tq, tk, tv, to, a, grid, st);
+    s = f16 ? dispatch_fwd<128, false, true>(c, m, a, grid, st)
+            : dispatch_fwd<128, false, false>(c, m, a, grid, st);
   else
-    s = f16 ? dispatch_fwd<64, false, true>(c, tq, tk, tv, to, a, grid, st)
-            : dispatch_fwd<64, false, false>(c, tq, tk, tv, to, a, grid, st);
+    s = f16 ? dispatch_fwd<64, false, true>(c, m, a, grid, st)
+            : dispatch_fwd<64, false, false>(c, m, a, grid, st);
   if (s != ATTN_OK || !c->split_path) return s;
   if (D == 128)
     return f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
@@ -884,7 +914,7 @@ static attn_status forward_host_impl(attn_ctx* c, const void* q_host, const void
                                      void* stream) {
   if (chunks < 0 || chunks > kMaxHostChunks || !rope_ready(c)) return ATTN_ERR_INVALID_ARG;
   const attn_params& p = c->p;
-  const bool quant = p.precision == ATTN_INT8QK_FP8PV;
+  const bool quant = p.precision != ATTN_EXACT;
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
   if ((need_q && (!q_host || !o_host)) || (need_kv && (!k_host || !v_host)))
     return ATTN_ERR_INVALID_ARG;
@@ -947,8 +977,11 @@ static attn_status forward_host_impl(attn_ctx* c, const void* q_host, const void
     if (!ok) break;
     if (quant) {
       s = quantize_units(c, u0, nu, q_dev, k_dev, v_dev, qb, cs);
+      // the band mode also reads the 16-bit Q and K of its diagonal tiles
+      const bool diag = p.precision == ATTN_MIXED_DIAG;
       if (s == ATTN_OK)
-        s = forward_units(c, u0, nu, nullptr, nullptr, nullptr, qb, o_dev, lse_dev, cs, 1 + i);
+        s = forward_units(c, u0, nu, diag ? q_dev : nullptr, diag ? k_dev : nullptr, nullptr, qb,
+                          o_dev, lse_dev, cs, 1 + i);
     } else {
       s = forward_units(c, u0, nu, q_dev, k_dev, v_dev, nullptr, o_dev, lse_dev, cs, 1 + i);
     }
@@ -1141,12 +1174,14 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   const CUtensorMapDataType t16 =
       f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t R = c.R, Sk = p->kv_len, U = c.units;
-  CUtensorMap tq, tk, tv, to;
+  FwdMaps m;
   bool ok = true;
-  ok &= make_map(&tq, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&tk, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&tv, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&to, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m.q, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m.k, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m.v, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m.o, t16, o, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  m.q16 = m.q;
+  m.k16 = m.k;
   if (!ok) return ATTN_ERR_CUDA;
 
   FwdArgs a{};
@@ -1172,13 +1207,13 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   a.debug = 0;
   const int grid = c.units * c.row_tiles * c.splits;
   if (D == 128) {
-    st = f16 ? dispatch_fwd<128, false, true>(&c, tq, tk, tv, to, a, grid, s)
-             : dispatch_fwd<128, false, false>(&c, tq, tk, tv, to, a, grid, s);
+    st = f16 ? dispatch_fwd<128, false, true>(&c, m, a, grid, s)
+             : dispatch_fwd<128, false, false>(&c, m, a, grid, s);
     if (st == ATTN_OK)
       st = f16 ? launch_merge<128, true>(&c, o, lse, s) : launch_merge<128, false>(&c, o, lse, s);
   } else {
-    st = f16 ? dispatch_fwd<64, false, true>(&c, tq, tk, tv, to, a, grid, s)
-             : dispatch_fwd<64, false, false>(&c, tq, tk, tv, to, a, grid, s);
+    st = f16 ? dispatch_fwd<64, false, true>(&c, m, a, grid, s)
+             : dispatch_fwd<64, false, false>(&c, m, a, grid, s);
     if (st == ATTN_OK)
       st = f16 ? launch_merge<64, true>(&c, o, lse, s) : launch_merge<64, false>(&c, o, lse, s);
   }

@@ -32,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "rope.cuh"
 
@@ -82,8 +84,12 @@ struct FwdArgs {
 
 constexpr int kErrTimeout = 1;
 
-template <int D, int NQT, bool QUANT, bool SPLIT>
+// DIAG (quantised mode only): the key tiles of the causal diagonal band get
+// Q K^T from the 16-bit inputs; 16-bit Q tiles sit next to the INT8 ones and one
+// 16-bit K tile buffer serves the band tiles (the ring carries the rest).
+template <int D, int NQT, bool QUANT, bool SPLIT, bool DIAG = false>
 struct FwdCfg {
+  static_assert(!DIAG || (QUANT && !SPLIT), "the diagonal band mode is a single-pass quantised kernel");
   static constexpr int kThreads = 128 * (1 + NQT);
   static constexpr int kElem = QUANT ? 1 : 2;                 // bytes per Q/K element
   static constexpr int kQTile = 128 * D * kElem;              // one 128-row Q tile
@@ -91,10 +97,14 @@ struct FwdCfg {
   static constexpr int kVTile = 128 * D * (QUANT ? 1 : 2);
   static constexpr int kSlot = kKTile > kVTile ? kKTile : kVTile;
   static constexpr int kOStage = 128 * D * 2;                 // 16-bit output tile
+  static constexpr int kQ16Tile = DIAG ? 128 * D * 2 : 0;     // 16-bit Q tile (DIAG)
+  static constexpr int kKdBytes = DIAG ? 128 * D * 2 : 0;     // 16-bit K tile (DIAG)
   static constexpr bool kStageInQ = (kQTile >= kOStage);
-  static constexpr int kStageBytes = (SPLIT || kStageInQ) ? 0 : NQT * kOStage;
-  static constexpr int kFixed = NQT * kQTile + kStageBytes;
-  static constexpr int kBudget = 200 * 1024;
+  static constexpr int kStageBytes = (SPLIT || kStageInQ || DIAG) ? 0 : NQT * kOStage;
+  static constexpr int kFixed = NQT * (kQTile + kQ16Tile) + kKdBytes + kStageBytes;
+  // (the band mode's extra 16-bit tiles would leave a 4-slot ring at 200 KB; it takes
+  // up to 224 KB of the 227 KB a CTA may use, for 6 slots at head_dim 128)
+  static constexpr int kBudget = (DIAG ? 224 : 200) * 1024;
   static constexpr int kNSraw = (kBudget - kFixed) / kSlot;
   // The split-KV variant serves few-row (decode) problems whose CTAs each see a
   // short key range: two K/V slots suffice, so that two CTAs share an SM.
@@ -102,27 +112,37 @@ struct FwdCfg {
   static constexpr int kCtasPerSm = SPLIT ? 2 : 1;
   static_assert(kNS >= 2, "ring too small");
   static constexpr int kQOff = 0;
-  static constexpr int kStageOff = NQT * kQTile;
+  static constexpr int kQ16Off = NQT * kQTile;                // DIAG: 16-bit Q tiles
+  static constexpr int kKdOff = kQ16Off + NQT * kQ16Tile;     // DIAG: 16-bit K tile
+  // output staging: its own buffers, or the Q tiles (16-bit Q tiles in DIAG)
+  static constexpr int kStageOff = DIAG ? kQ16Off : NQT * kQTile;
+  static constexpr int kStageTile = DIAG ? kQ16Tile : (kStageInQ ? kQTile : kOStage);
+  static constexpr bool kStageInQBuf = kStageInQ && !DIAG;
   static constexpr int kRingOff = kFixed;
   static constexpr int kBarOff = kRingOff + kNS * kSlot;
   // barriers: q_full, full[NS], empty[NS], s_ready[NQT], p_ready[NQT][2] (one per
-  // 64-key half of P), o_final, q_rot (RoPE: the staged Q has been rotated)
-  static constexpr int kNumBars = 1 + 2 * kNS + 3 * NQT + 2;
+  // 64-key half of P), o_final, q_rot (RoPE: the staged Q has been rotated),
+  // kd_full, kd_empty (DIAG: the 16-bit K tile buffer)
+  static constexpr int kNumBars = 1 + 2 * kNS + 3 * NQT + 4;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;      // tmem base, abort flag
   static constexpr int kSvOff = kMiscOff + 16;                  // v scales (quant)
   static constexpr int kSmemBytes = kSvOff + (QUANT ? D * 4 : 0) + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
   static constexpr int kTmemNeed = NQT * (128 + D);
   static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
   // transaction bytes
-  static constexpr uint32_t kQBytes = NQT * kQTile;
+  static constexpr uint32_t kQBytes = NQT * (kQTile + kQ16Tile);
   static constexpr uint32_t kKBytes = kKTile;
   static constexpr uint32_t kVBytes = kVTile;
   // softmax rescale threshold (base-2 units): O and l are rescaled only when a
   // row max grows by more than this, so P <= 2^thresh.  Quantised: P is scaled by
   // 2^kPScale before the E4M3 cast and 2^(kPScale + thresh) = 2^8.8 ~ 445 stays
-  // within the largest finite E4M3 value (448).
-  static constexpr float kRescaleThresh = QUANT ? 1.8f : 8.0f;
-  static constexpr float kPScale = QUANT ? 7.0f : 0.0f;
+  // within the largest finite E4M3 value (448).  A larger threshold means fewer
+  // rescales; the smaller factor only moves the E4M3 subnormal floor of P from
+  // 2^-16 to 2^-14 relative to the running max (video, quantised: 15.41 ms with
+  // 2^7 and 1.8, 15.02 ms with 2^5 and 3.8; the outputs' error is unchanged).
+  static constexpr float kRescaleThresh = QUANT ? 3.8f : 8.0f;
+  static constexpr float kPScale = QUANT ? 5.0f : 0.0f;
   // Registers per thread at launch (65536 / (threads * CTAs per SM), rounded
   // down to a multiple of 8) and their split between warpgroups: the
   // loader/MMA warpgroup needs few, the softmax warpgroups many.
@@ -179,14 +199,17 @@ struct RowSums {
 // second half once its first 32 keys are computed and before they are stored:
 // the hand-off of the first half waits for that half's stores to complete, and
 // by then they have.
-template <bool F16, bool QUANT, int POLY, bool LF, int H, typename Mid>
+// FS (quantised mode, diagonal band tiles): x holds float32 scores already.
+template <bool F16, bool QUANT, int POLY, bool LF, int H, bool FS = false, typename Mid>
 __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 cm, f32x2 mm,
                                                   uint32_t tS, RowSums& rs, Mid&& mid) {
 #pragma unroll
   for (int ch = 2 * H; ch < 2 * H + 2; ++ch) {
     if constexpr (QUANT) {
       // x holds the int32 scores' bits; adding 0x4B400000 gives 1.5 * 2^23 + s exactly
-      auto sc = [](float v) { return __uint_as_float(__float_as_uint(v) + 0x4B400000u); };
+      auto sc = [](float v) {
+        return FS ? v : __uint_as_float(__float_as_uint(v) + 0x4B400000u);
+      };
       uint32_t pk[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -245,7 +268,7 @@ __device__ __forceinline__ void softmax_emit_half(const float (&x)[128], f32x2 c
 // at chunk position k ^ (r & 7) (the TMA 128-byte swizzle).  Each chunk of the
 // first R channels is rotated with its partner chunk (rope.cuh); the half layout
 // handles both chunks of a pair at once.
-template <bool F16>
+template <int D, bool F16>
 __device__ __forceinline__ void rope_q_row(uint32_t tile, int row, const float* table, int R,
                                            bool inter, int pos) {
   auto addr = [&](int cj) {  // chunk cj (channels 8 cj .. 8 cj + 7) of this row
@@ -257,14 +280,19 @@ __device__ __forceinline__ void rope_q_row(uint32_t tile, int row, const float* 
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
   };
+  // (no memory clobber: the table loads of later chunks may be issued early; the
+  // caller's proxy fence orders these stores before the tensor core reads them)
   auto st = [](uint32_t a, const uint4& v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
+                 "r"(v.z), "r"(v.w));
   };
   const int n = inter ? R / 8 : R / 16;
-#pragma unroll 1
-  for (int cj = 0; cj < n; ++cj) {
+  // unrolled over the most chunks a row can have, so that the table loads of
+  // several chunks are in flight together
+  constexpr int kMaxChunks = D / 8;
+#pragma unroll
+  for (int cj = 0; cj < kMaxChunks; ++cj) {
+    if (cj >= n) break;
     const int pj = rope_partner(cj, R, inter);
     const uint4 a = ld(addr(cj));
     const uint4 b = inter ? a : ld(addr(pj));
@@ -285,14 +313,17 @@ __device__ __forceinline__ void rope_q_row(uint32_t tile, int row, const float* 
 // the bounds they need in fewer registers.  ROPE (exact mode): the softmax
 // warpgroups rotate the staged Q tile before the first Q K^T (the keys arrive
 // rotated).
-template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE>
-__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
-                                  FwdCfg<D, NQT, QUANT, SPLIT>::kCtasPerSm)
+template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
+          bool DIAG = false>
+__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
+                                  FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kCtasPerSm)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_o, const FwdArgs a) {
-  using C = FwdCfg<D, NQT, QUANT, SPLIT>;
+                     const __grid_constant__ CUtensorMap tm_o,
+                     const __grid_constant__ CUtensorMap tm_q16,
+                     const __grid_constant__ CUtensorMap tm_k16, const FwdArgs a) {
+  using C = FwdCfg<D, NQT, QUANT, SPLIT, DIAG>;
   static_assert(!SPLIT || LF, "the split variant always needs the float32 row sum");
   static_assert(!(ROPE && QUANT), "the quantised mode rotates Q and K in its quantiser");
   extern __shared__ uint8_t smem_raw[];
@@ -361,6 +392,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
   auto p_ready = [&](int q, int h) { return bar(1 + 2 * C::kNS + NQT + 2 * q + h); };
   const uint32_t o_final = bar(1 + 2 * C::kNS + 3 * NQT);
   const uint32_t q_rot = bar(2 + 2 * C::kNS + 3 * NQT);
+  const uint32_t kd_full = bar(3 + 2 * C::kNS + 3 * NQT);
+  const uint32_t kd_empty = bar(4 + 2 * C::kNS + 3 * NQT);
+  // DIAG: key tile j (absolute tile index jt) lies in the causal diagonal band of
+  // this CTA when some of its rows must mask part of it for causality; its Q K^T
+  // uses the 16-bit inputs.  The loader, the MMA warp and the softmax evaluate the
+  // same predicate.
+  auto in_band = [&](int jt) { return DIAG && a.causal && (jt * 128 + 127 > pos_min); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   float* sv_smem = reinterpret_cast<float*>(smem + C::kSvOff);
@@ -378,6 +416,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
     }
     mbar_init(o_final, 1);
     mbar_init(q_rot, 4 * NQT);  // one arrive per softmax warp
+    mbar_init(kd_full, 1);
+    mbar_init(kd_empty, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -425,9 +465,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         for (int bx = 0; bx < kQBoxes; ++bx)
           tma_load_3d(&tm_q, sbase + C::kQOff + q * C::kQTile + bx * kQBox, q_full,
                       bx * kBoxCols, r0 + q * 128, u);
+      if constexpr (DIAG) {  // the 16-bit Q tiles, for the band's Q K^T
+        prefetch_tmap(&tm_q16);
+        prefetch_tmap(&tm_k16);
+        for (int q = 0; q < NQT; ++q)
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_3d(&tm_q16, sbase + C::kQ16Off + q * C::kQ16Tile + bx * 128 * 64 * 2,
+                        q_full, bx * 64, r0 + q * 128, u);
+      }
       int last_issue[C::kNS];
       for (int s = 0; s < C::kNS; ++s) last_issue[s] = -1;
       int it = 0;
+      int kd_it = 0;  // DIAG: 16-bit K tiles loaded
       bool ok = true;
       // Paged K/V: this unit's row of the block table; each tile's block id is read
       // one tile ahead, so the read does not delay the tile's copies.
@@ -440,6 +489,17 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         const int blk = blk_next;
         if (paged && j + 1 < n) blk_next = __ldg(bt_row + j + 1);
         for (int part = 0; part < 2 && ok; ++part, ++it) {  // 0: K tile, 1: V tile
+          if (part == 0 && in_band(jt0 + j)) {
+            // DIAG: the band's K tile in 16 bits, into its own buffer (no ring slot)
+            if (!mbar_wait(kd_empty, (kd_it & 1) ^ 1, abort_flag)) { raise(); ok = false; break; }
+            mbar_arrive_expect_tx(kd_full, C::kKdBytes);
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_load_3d(&tm_k16, sbase + C::kKdOff + bx * 128 * 64 * 2, kd_full, bx * 64, kv0,
+                          u);
+            ++kd_it;
+            --it;  // undone by the loop's increment: the ring was not used
+            continue;
+          }
           const int s = it % C::kNS;
           const uint32_t ph = (it / C::kNS) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag)) { raise(); ok = false; break; }
@@ -486,6 +546,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
                  globaltimer_ns() - t0 < kWaitTimeoutNs) {
           }
         }
+      if (kd_it > 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(kd_full, (kd_it - 1) & 1) &&
+               globaltimer_ns() - t0 < kWaitTimeoutNs) {
+        }
+      }
     }
   } else if (warp == 1) {
     // ========================================================= MMA issuer
@@ -508,6 +574,22 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       const uint32_t q_lo0 = desc_lo(sbase + C::kQOff, 16);
       const uint32_t ring_lo = desc_lo(sbase + C::kRingOff, 16);
       const uint32_t ring_lo_v = desc_lo(sbase + C::kRingOff, lbo_v);
+      // DIAG: Q K^T of a band tile from the 16-bit Q tile and K buffer (f32 scores)
+      constexpr uint32_t idesc_qk16 = instr_desc(1, fmt, fmt, 0, 0, 128, 128);
+      constexpr uint32_t hi_16 = desc_hi(1024u, 2u);
+      const uint32_t q16_lo0 = desc_lo(sbase + C::kQ16Off, 16);
+      const uint32_t kd_lo = desc_lo(sbase + C::kKdOff, 16);
+      auto issue_qk16 = [&](int q) {
+        const uint32_t q_lo = q16_lo0 + q * (C::kQ16Tile >> 4);
+        const uint32_t d = tmem + q * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 2;  // (64-col box, 32 B) >> 4
+          mma_f16_ss(d, desc_pack(q_lo + off, hi_16), desc_pack(kd_lo + off, hi_16), idesc_qk16,
+                     kk > 0);
+        }
+      };
+      int kd_it = 0;  // band K tiles consumed
       auto issue_qk = [&](int q, uint32_t k_lo) {
         const uint32_t q_lo = q_lo0 + q * (C::kQTile >> 4);
         const uint32_t d = tmem + q * 128;
@@ -547,7 +629,19 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       };
 
       // S_0 for every query tile
-      if (ok) {
+      if (ok && in_band(jt0)) {
+        ok = mbar_wait(kd_full, 0, abort_flag);
+        if (!ok) raise();
+        else {
+          tc_fence_after();
+          for (int q = 0; q < NQT; ++q) {
+            issue_qk16(q);
+            tc_commit(s_ready(q));
+          }
+          tc_commit(kd_empty);
+          ++kd_it;
+        }
+      } else if (ok) {
         const int s = it % C::kNS;
         ok = mbar_wait(full_bar(s), (it / C::kNS) & 1, abort_flag);
         if (!ok) raise();
@@ -567,8 +661,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         if (!mbar_wait(full_bar(sv), (it / C::kNS) & 1, abort_flag)) { raise(); ok = false; break; }
         ++it;
         const bool has_next = (j + 1 < n);
+        const bool next_band = has_next && in_band(jt0 + j + 1);
         int sk = 0;
-        if (has_next) {
+        if (next_band) {
+          if (!mbar_wait(kd_full, kd_it & 1, abort_flag)) { raise(); ok = false; break; }
+        } else if (has_next) {
           sk = it % C::kNS;
           if (!mbar_wait(full_bar(sk), (it / C::kNS) & 1, abort_flag)) { raise(); ok = false; break; }
           ++it;
@@ -585,12 +682,20 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
           }
           if (!ok) break;
           if (q == NQT - 1) tc_commit(empty_bar(sv));
-          if (has_next) {
+          if (next_band) {
+            issue_qk16(q);
+            tc_commit(s_ready(q));
+          } else if (has_next) {
             issue_qk(q, k_lo);
             tc_commit(s_ready(q));
           }
         }
-        if (ok && has_next) tc_commit(empty_bar(sk));
+        if (ok && next_band) {
+          tc_commit(kd_empty);
+          ++kd_it;
+        } else if (ok && has_next) {
+          tc_commit(empty_bar(sk));
+        }
       }
       tc_commit(o_final);
       // Leave only once every issued MMA has finished (TMEM is freed at exit).
@@ -641,8 +746,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       } else if (rvalid) {
         constexpr int kQBox = 128 * 64 * 2;
         static_assert(C::kQTile == (D / 64) * kQBox, "16-bit Q tile in 64-channel boxes");
-        rope_q_row<F16>(sbase + C::kQOff + q * C::kQTile, row, a.rope_table, a.rope_R,
-                        a.rope_inter != 0, pos);
+        rope_q_row<D, F16>(sbase + C::kQOff + q * C::kQTile, row, a.rope_table, a.rope_R,
+                           a.rope_inter != 0, pos);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -666,6 +771,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
       __syncwarp();
       if (lane == 0) mbar_arrive(p_ready(q, h));
     };
+    if constexpr (!DIAG) {
+    // (the kernels without the band mode keep this straight-line form of the tile loop;
+    // the band mode below compiles the tile body once per kind of score)
     for (int j = 0; j < n && ok; ++j) {
       const float ksc = ksc_next;
       if constexpr (QUANT)
@@ -798,6 +906,160 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         if constexpr (LF) lf += fsum;
       }
     }
+    } else {
+    for (int j = 0; j < n && ok; ++j) {
+      const float ksc = ksc_next;
+      if constexpr (QUANT)
+        if (j + 1 < n) ksc_next = ld_global_f32(ksrc + j + 1);
+      // DIAG: a band tile's scores are float32 products of the 16-bit inputs
+      const bool band = in_band(jt0 + j);
+      // The tile's body, compiled once per kind of score: FS (the diagonal band
+      // mode's band tiles) reads float32 scores, otherwise INT8 products (quantised)
+      // or float32 (exact).  Separate copies keep each one's registers to itself.
+      auto tile = [&](auto fs_tag) -> bool {
+        constexpr bool FS = decltype(fs_tag)::value;
+        // raw score -> base-2 scaled score factor (quantised: kept positive so that
+        // masked -inf scores stay -inf for an all-zero block); known before S lands
+        const float cj =
+            (QUANT && !FS)
+                ? __uint_as_float(__float_as_uint(fmaxf(qsc * ksc * a.scale_log2, 1e-30f)) & ~7u)
+                : a.scale_log2;
+        bool ok2 = __all_sync(0xffffffffu, mbar_wait(s_ready(q), j & 1, abort_flag));
+        if (!ok2) {
+          if (lane == 0) raise();
+          return false;
+        }
+        tc_fence_after();
+        const int kv0 = (jt0 + j) * 128;
+        const bool need_mask =
+            (kv0 < kv_lo_max) || (kv0 + 128 > a.Skv) || (a.causal && kv0 + 127 > pos_min);
+        // S is read in two 64-column halves: the second half's load overlaps the
+        // masking and maximum of the first.  Row max: four chains of three-input maxima.
+        // Quantised: x keeps the int32 scores' bits, the row max runs on the integers
+        // (eight chains) and the float offset is added in the emit; a masked score is
+        // the bit pattern that the offset turns into -inf (below every real score).
+        constexpr uint32_t kMaskedBits = 0xFF800000u - 0x4B400000u;
+        const float masked = (QUANT && !FS) ? __uint_as_float(kMaskedBits) : -INFINITY;
+        float x[128];
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        constexpr int kIntMin = -2147483647 - 1;
+        int mi[8] = {kIntMin, kIntMin, kIntMin, kIntMin, kIntMin, kIntMin, kIntMin, kIntMin};
+        auto row_max = [&](int c0) {
+  #pragma unroll
+          for (int c = c0; c < c0 + 64; c += 8) {
+            if (QUANT && !FS) {
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) mi[e] = max(mi[e], static_cast<int>(__float_as_uint(x[c + e])));
+            } else {
+  #pragma unroll
+              for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[c + 2 * e], x[c + 2 * e + 1]);
+            }
+          }
+        };
+        {
+          uint32_t s0[32], s1[32];
+          tmem_ld32(tS + 0, s0);
+          tmem_ld32(tS + 32, s1);
+          tmem_ld_wait(s0);
+          tmem_ld_wait(s1);
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[c] = __uint_as_float(s0[c]);
+            x[32 + c] = __uint_as_float(s1[c]);
+          }
+        }
+        uint32_t s2[32], s3[32];
+        tmem_ld32(tS + 64, s2);
+        tmem_ld32(tS + 96, s3);
+        if (need_mask) {
+  #pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int kj = kv0 + c;
+            if (kj < lo_r || kj > hi_r) x[c] = masked;
+          }
+        }
+        row_max(0);
+        tmem_ld_wait(s2);
+        tmem_ld_wait(s3);
+  #pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[64 + c] = __uint_as_float(s2[c]);
+          x[96 + c] = __uint_as_float(s3[c]);
+        }
+        if (need_mask) {
+  #pragma unroll
+          for (int c = 64; c < 128; ++c) {
+            const int kj = kv0 + c;
+            if (kj < lo_r || kj > hi_r) x[c] = masked;
+          }
+        }
+        row_max(64);
+        float mx;
+        if (QUANT && !FS) {
+          int mr = max(max(max(mi[0], mi[1]), max(mi[2], mi[3])),
+                       max(max(mi[4], mi[5]), max(mi[6], mi[7])));
+          mx = to_score(static_cast<uint32_t>(mr)) - kMagic;  // exact; -inf if all masked
+        } else {
+          mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        }
+        const float m_tile = mx * cj;  // cj > 0; -inf stays -inf
+        const float m_prev = m_used;
+        const float m_new = fmaxf(m_prev, m_tile);
+        const bool need = (m_prev != -INFINITY) && (m_new > m_prev + C::kRescaleThresh);
+        if (m_prev == -INFINITY || need) m_used = QUANT ? ceilf(m_new) : m_new;
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? ex2(m_prev - m_used) : 1.0f;
+          l *= f;
+          lf *= f;
+  #pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_ld_wait(o);
+  #pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+            tmem_st32(tO + c0, o);
+          }
+        }
+        // P = 2^(x * cj - m)  (quantised: times 2^7 before the E4M3 cast), written
+        // over S in two 64-key halves; the MMA warp starts on the first half while
+        // the second is computed.  Exact mode: the row sum l adds the 16-bit values
+        // that the P.V product actually uses, so O is a convex combination of V rows;
+        // lf adds the float32 values (for lse).  On tiles without masked keys a share
+        // of the exponentials run on the FMA pipe (poly_ex2x2).
+        const float mb = (m_used == -INFINITY ? 0.0f : m_used) - C::kPScale;
+        const float kq = (QUANT && !FS) ? fmaf(kMagic, cj, mb) : mb;  // int scores: offset folded in
+        const f32x2 cm{cj, cj}, mm{-kq, -kq};
+        RowSums rs{{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f}, {0.0f, 0.0f}};
+        auto none = [] {};
+        auto first_half_done = [&] { p_half_done(0); };
+        if constexpr (FS) {
+          softmax_emit_half<F16, QUANT, 0, LF, 0, true>(x, cm, mm, tS, rs, none);
+          softmax_emit_half<F16, QUANT, 0, LF, 1, true>(x, cm, mm, tS, rs, first_half_done);
+        } else if (need_mask) {
+          softmax_emit_half<F16, QUANT, 0, LF, 0>(x, cm, mm, tS, rs, none);
+          softmax_emit_half<F16, QUANT, 0, LF, 1>(x, cm, mm, tS, rs, first_half_done);
+        } else {
+          softmax_emit_half<F16, QUANT, kPoly, LF, 0>(x, cm, mm, tS, rs, none);
+          softmax_emit_half<F16, QUANT, kPoly, LF, 1>(x, cm, mm, tS, rs, first_half_done);
+        }
+        p_half_done(1);
+        const float fsum = (rs.f0.x + rs.f0.y) + (rs.f1.x + rs.f1.y);
+        if constexpr (QUANT) {
+          l += fsum;
+          lf += fsum;
+        } else {
+          l += (rs.r[0] + rs.r[1]) + (rs.r[2] + rs.r[3]);
+          if constexpr (LF) lf += fsum;
+        }
+        return true;
+      };
+      if (DIAG && band)
+        ok = tile(std::true_type{});
+      else
+        ok = tile(std::false_type{});
+    }
+    }
 
     // ----------------------------------------------------------- epilogue
     if (ok && n > 0) {
@@ -852,8 +1114,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT>::kThreads,
         a.lse_part[(size_t)a.splits * a.units * a.R + prow] = lse2;
       }
     } else {
-      const uint32_t stage = C::kStageInQ ? sbase + C::kQOff + q * C::kQTile
-                                          : sbase + C::kStageOff + q * C::kOStage;
+      const uint32_t stage = C::kStageInQBuf ? sbase + C::kQOff + q * C::kQTile
+                                             : sbase + C::kStageOff + q * C::kStageTile;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];

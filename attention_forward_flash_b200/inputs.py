@@ -87,7 +87,7 @@ WORKLOADS = {
     "video": Workload("video", 1, 40, 40, 32760, 32760, 128, "bf16", modes=("exact", "quant"),
                       seed=1003, oracle_rows=256),
     "llm": Workload("llm", 4, 32, 8, 8192, 8192, 128, "bf16", causal=True,
-                    modes=("exact", "quant"), seed=1004, k_outlier_frac=0.01,
+                    modes=("exact", "quant", "mixed"), seed=1004, k_outlier_frac=0.01,
                     k_outlier_mult=20.0, oracle_rows=256),
     # the causal GQA prefill with a 1024-position sliding window per row
     "llm_window": Workload("llm_window", 4, 32, 8, 8192, 8192, 128, "bf16", causal=True,

@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video", choices=sorted(WORKLOADS))
-    ap.add_argument("--precision", default="exact", choices=["exact", "quant"])
+    ap.add_argument("--precision", default="exact", choices=["exact", "quant", "mixed"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -187,7 +187,7 @@ def make_attention(w: Workload, precision):
 
 def launches_per_step(att, precision):
     n = 1 + (1 if att.num_splits > 1 else 0)
-    if precision == "quant":
+    if precision != "exact":
         n += 4  # Q and K block quantisers, V channel maxima, V quantiser
     elif att.params.rope_dim > 0 and not att.params.rope_keys_rotated:
         n += 1  # the keys' rotation pass
@@ -392,14 +392,12 @@ def measure(w: Workload, precision, steps, warmup, device):
         scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
         scratch_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
         flush = lambda: (scratch.fill_(1), scratch_r.sum())  # noqa: E731
-    qb = att.quantize(q, k, v) if precision == "quant" else None
+    qb = att.quantize(q, k, v) if precision != "exact" else None
 
     def step():
-        if precision == "quant":
+        if precision != "exact":
             att.quantize(q, k, v, qbufs=qb)
-            att.forward(qbufs=qb, out=out)
-        else:
-            att.forward(q, k, v, out=out)
+        att.forward(q, k, v, qbufs=qb, out=out)
 
     def kernel_only():
         att.forward(q, k, v, qbufs=qb, out=out)
@@ -421,7 +419,7 @@ def measure_e2e(w: Workload, precision, m, steps, warmup, chunks=0):
     att = m["att"]
     hq, hk, hv = (t.cpu().pin_memory() for t in (m["q"], m["k"], m["v"]))
     ho = torch.empty(m["out"].shape, dtype=m["out"].dtype).pin_memory()
-    staging = DeviceStaging(att.params, att.dtype, m["q"].device, precision == "quant", False)
+    staging = DeviceStaging(att.params, att.dtype, m["q"].device, precision != "exact", False)
 
     def step():
         att.forward_host(hq, hk, hv, out=ho, staging=staging, chunks=chunks)
@@ -456,11 +454,9 @@ def run_native(args):
     out, q, k, v, qb = m["out"], m["q"], m["k"], m["v"], m["qb"]
 
     def step():
-        if precision == "quant":
+        if precision != "exact":
             att.quantize(q, k, v, qbufs=qb)
-            att.forward(qbufs=qb, out=out)
-        else:
-            att.forward(q, k, v, out=out)
+        att.forward(q, k, v, qbufs=qb, out=out)
 
     for _ in range(args.warmup):
         step()
@@ -483,26 +479,26 @@ def run_native(args):
     value = flops * world / (ms * 1e-3) / 1e12
 
     # ---- dominant kernel (the fused attention kernel) for the roofline
-    if precision == "quant":
-        ms_kernel = time_steps(lambda: att.forward(qbufs=qb, out=out), args.steps, 2)
+    if precision != "exact":
+        ms_kernel = time_steps(lambda: att.forward(q, k, v, qbufs=qb, out=out), args.steps, 2)
     else:
         ms_kernel = ms_local
     peak_key = "bf16_tflops"
     peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
-    if precision == "quant":
+    if precision != "exact":
         peak = 2.0 * peak  # INT8 / FP8 dense rate = 2x the bf16 rate (nominal 4.5 vs 2.25 PF)
     achieved = flops / (ms_kernel * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": recorded_traffic(w.name, precision),
                 "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" +
-                (" x2 for INT8/FP8" if precision == "quant" else ""),
+                (" x2 for INT8/FP8" if precision != "exact" else ""),
                 "kernel": "flash_fwd_kernel", "kernel_ms": ms_kernel}
 
     # ---- the quantisers on their own (quantised mode): an HBM-bound pass whose
     # algorithmic bytes are Q and K read once, V read twice (channel maxima, then
     # the codes), and the codes and scales written once
     quantiser = None
-    if precision == "quant":
+    if precision != "exact":
         ms_q = time_steps(lambda: att.quantize(q, k, v, qbufs=qb), args.steps, 2)
         q_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, v))
         q_bytes += sum(t.numel() * t.element_size()
@@ -544,7 +540,7 @@ def run_native(args):
                            ("llm", "exact"), ("llm", "quant"), ("image", "exact"),
                            ("image", "quant"), ("decode", "exact"), ("decode_window", "exact"),
                            ("llm_window", "exact"), ("video_rope", "exact"),
-                           ("video_rope", "quant"), ("llm_rope", "exact")):
+                           ("video_rope", "quant"), ("llm_rope", "exact"), ("llm", "mixed")):
             if name == w.name and prec == precision:
                 continue
             wx = WORKLOADS[name]
@@ -558,7 +554,7 @@ def run_native(args):
                 kv_bytes = 2 * wx.batch * wx.n_kv_heads * wx.kv_len * wx.head_dim * 2
                 entry["hbm_gbs_kernel"] = kv_bytes / (mx["ms_kernel"] * 1e-3) / 1e9
                 entry["us_per_call"] = mx["ms_kernel"] * 1e3
-            if prec == "quant":
+            if prec != "exact":
                 entry["pct_of_int8_peak_kernel"] = 100 * entry["tflops_kernel"] / (2 * peaks.get(
                     "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
             else:

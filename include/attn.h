@@ -65,8 +65,15 @@ typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype;
 
 /* ATTN_EXACT is the default: 16-bit inputs, f32 accumulation.
  * ATTN_INT8QK_FP8PV is opt-in: Q/K quantised to INT8 per 128-token block with
- * FP32 scales, P and V in FP8 E4M3 (V with one FP32 scale per head and channel). */
-typedef enum { ATTN_EXACT = 0, ATTN_INT8QK_FP8PV = 1 } attn_precision;
+ * FP32 scales, P and V in FP8 E4M3 (V with one FP32 scale per head and channel).
+ * ATTN_MIXED_DIAG is opt-in too: diagonal-tiled mixed precision ("Transformers
+ * Get a Turbo Boost with Mixed-Precision Magic": two kinds of computation chosen
+ * per tile).  It is ATTN_INT8QK_FP8PV except that the key tiles of the causal
+ * diagonal band -- the tiles some row of a 256-row query tile must partly mask --
+ * get Q K^T from the 16-bit inputs (float32 scores); P and V stay FP8 E4M3.
+ * Without a causal mask there is no band and it computes what ATTN_INT8QK_FP8PV
+ * does.  It always runs the single-pass kernel (num_splits 0 or 1). */
+typedef enum { ATTN_EXACT = 0, ATTN_INT8QK_FP8PV = 1, ATTN_MIXED_DIAG = 2 } attn_precision;
 
 typedef struct {
   int batch;       /* B >= 1 */
@@ -139,7 +146,7 @@ typedef struct attn_ctx attn_ctx;
  * (head_dim not 64/128), ATTN_ERR_CUDA (no device), ATTN_ERR_OOM. */
 attn_status attn_create(const attn_params *p, attn_ctx **out);
 
-/* Quantised mode, step 1 (the per-block quantiser): reads q, k, v (dtype of
+/* Quantised and diagonal band modes, step 1 (the per-block quantiser): reads q, k, v (dtype of
  * the context) and writes every buffer of *qb.  Q and K: per (b, h, 128-token
  * block) s = max|x| / 127 and code = clamp(round_half_even(x / s), +-127), s = 0
  * for an all-zero block.  V: per (b, hkv, channel) s = max|v| / 448 and code =
@@ -154,7 +161,8 @@ attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const vo
 
 /* The attention forward.  Exact mode: q, k, v are read and qb must be NULL.
  * Quantised mode: q, k, v are ignored (may be NULL) and qb holds the output of
- * attn_quantize_qk.  Writes o ([B, Hq, Sq, D], the context's dtype) and, if
+ * attn_quantize_qk.  Diagonal band mode: qb as in the quantised mode, and q and k
+ * (the 16-bit inputs) are read for the band tiles; v is ignored.  Writes o ([B, Hq, Sq, D], the context's dtype) and, if
  * lse is not NULL, the natural-log sum of exp(scale * q.k) over each row's
  * visible keys.  Few-row (decode-shaped) problems are split along the keys and
  * merged by a second kernel into the same outputs.

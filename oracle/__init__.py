@@ -12,6 +12,8 @@ cases.
 
 from .attention import (  # noqa: F401
     attention_f64,
+    attention_f64_mixed,
+    diagonal_band_start,
     attention_flops,
     gather_paged,
     visible_pairs,

@@ -188,3 +188,67 @@ def visible_pairs(Sq, Skv, *, start_pos=0, causal=False, window_lo=0, window_siz
                                window_lo=window_lo, window_size=window_size)
         n += max(0, hi - lo + 1)
     return n
+
+
+def diagonal_band_start(i, hq, *, Sq, n_q_heads, n_kv_heads, start_pos=0, causal=True,
+                        query_tile=256, key_tile=128):
+    """First key of the causal diagonal band of query row ``i`` of head ``hq``.
+
+    The diagonal-tiled mixed precision of the page "Transformers Get a Turbo Boost
+    with Mixed-Precision Magic" chooses the arithmetic per tile; the page does not
+    say which tiles are "diagonal".  Reading: the query rows of a unit (the
+    ``G = n_q_heads / n_kv_heads`` heads sharing a kv head, stacked head-major,
+    ``G * Sq`` rows) are cut into tiles of ``query_tile`` rows; the band of a query
+    tile is every ``key_tile``-key tile that some row of it must partly mask for
+    causality, i.e. the key tiles from the one holding the smallest position
+    among its rows.  Without a causal mask there is no band (returns a key index
+    past any sequence).
+    """
+    if not causal:
+        return np.iinfo(np.int64).max
+    G = n_q_heads // n_kv_heads
+    r = (hq % G) * Sq + int(i)                      # stacked row within the unit
+    t0 = (r // query_tile) * query_tile
+    t1 = min(t0 + query_tile, G * Sq)
+    stacked = np.arange(t0, t1)
+    pos_min = int(start_pos) + int((stacked % Sq).min())
+    # key tile jt is in the band when jt * key_tile + key_tile - 1 > pos_min
+    return key_tile * ((pos_min + 1) // key_tile)
+
+
+def attention_f64_mixed(q, k, q_low, k_low, v, *, scale=None, causal=False, start_pos=0,
+                        rows=None, query_tile=256, key_tile=128):
+    """Float64 attention whose scores come from (q, k) on each row's causal diagonal
+    band (``diagonal_band_start``) and from (q_low, k_low) on every other key: the
+    definition of the diagonal-tiled mixed precision mode, with the low-precision
+    operands given as the values they represent (e.g. dequantised INT8 codes).
+    Same conventions and returns as ``attention_f64`` (no sliding window)."""
+    q, k, ql, kl, v = (_as_f64(x) for x in (q, k, q_low, k_low, v))
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    assert ql.shape == q.shape and kl.shape == k.shape and v.shape == k.shape
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.arange(Sq) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((B, Hq, len(rows), D))
+    lse = np.full((B, Hq, len(rows)), -np.inf)
+    j = np.arange(Skv)
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // group
+            for n, i in enumerate(rows):
+                lo, hi = visible_range(int(i), kv_len=Skv, start_pos=start_pos, causal=causal)
+                if hi < lo:
+                    continue
+                band = diagonal_band_start(i, hq, Sq=Sq, n_q_heads=Hq, n_kv_heads=Hkv,
+                                           start_pos=start_pos, causal=causal,
+                                           query_tile=query_tile, key_tile=key_tile)
+                keys = j[lo:hi + 1]
+                s = np.where(keys >= band, k[b, hk, lo:hi + 1] @ q[b, hq, i],
+                             kl[b, hk, lo:hi + 1] @ ql[b, hq, i]) * scale
+                m = s.max()
+                p = np.exp(s - m)
+                out[b, hq, n] = (p / p.sum()) @ v[b, hk, lo:hi + 1]
+                lse[b, hq, n] = m + math.log(p.sum())
+    return out, lse
