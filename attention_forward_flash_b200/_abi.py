@@ -8,13 +8,14 @@ import os
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_OOM, \
     ATTN_ERR_TIMEOUT = range(6)
 ATTN_BF16, ATTN_FP16 = 0, 1
-ATTN_EXACT, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG = 0, 1, 2
+ATTN_EXACT, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG, ATTN_MXFP4QK_FP8PV = 0, 1, 2, 3
 ATTN_ROPE_PLAIN, ATTN_ROPE_NTK, ATTN_ROPE_YARN = 0, 1, 2
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
             "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host",
-            "attn_forward_paged", "attn_rope_table", "attn_set_rope_table", "attn_rope_apply")
+            "attn_forward_paged", "attn_rope_table", "attn_set_rope_table", "attn_rope_apply",
+            "attn_qbufs_sf_sizes")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -42,7 +43,8 @@ class AttnRopeFreq(ctypes.Structure):
 class AttnQBufs(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
                 ("k_scale", ctypes.c_void_p), ("v_t", ctypes.c_void_p),
-                ("v_scale", ctypes.c_void_p)]
+                ("v_scale", ctypes.c_void_p), ("q_sf", ctypes.c_void_p),
+                ("k_sf", ctypes.c_void_p)]
 
 
 class AttnError(RuntimeError):
@@ -78,6 +80,9 @@ def lib():
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_qbufs_sizes.argtypes = [ctypes.POINTER(AttnParams), ctypes.POINTER(ctypes.c_size_t)]
         L.attn_qbufs_sizes.restype = c_int
+        L.attn_qbufs_sf_sizes.argtypes = [ctypes.POINTER(AttnParams),
+                                          ctypes.POINTER(ctypes.c_size_t)]
+        L.attn_qbufs_sf_sizes.restype = c_int
         L.attn_num_splits.argtypes = [vp]
         L.attn_num_splits.restype = c_int
         L.attn_debug_set.argtypes = [vp, ctypes.c_uint]
@@ -136,6 +141,12 @@ def attn_destroy(ctx):
 def attn_qbufs_sizes(params: AttnParams):
     sizes = (ctypes.c_size_t * 6)()
     _check(lib().attn_qbufs_sizes(ctypes.byref(params), sizes), "attn_qbufs_sizes")
+    return list(sizes)
+
+
+def attn_qbufs_sf_sizes(params: AttnParams):
+    sizes = (ctypes.c_size_t * 2)()
+    _check(lib().attn_qbufs_sf_sizes(ctypes.byref(params), sizes), "attn_qbufs_sf_sizes")
     return list(sizes)
 
 

@@ -11,7 +11,7 @@ import torch
 
 from . import _abi
 from ._abi import (ATTN_BF16, ATTN_EXACT, ATTN_FP16, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG,
-                   ATTN_ROPE_NTK,
+                   ATTN_MXFP4QK_FP8PV, ATTN_ROPE_NTK,
                    ATTN_ROPE_PLAIN, ATTN_ROPE_YARN, AttnParams, AttnQBufs, AttnRopeFreq)
 
 _SCALINGS = {None: ATTN_ROPE_PLAIN, "ntk": ATTN_ROPE_NTK, "yarn": ATTN_ROPE_YARN}
@@ -26,8 +26,10 @@ def rope_table(rope_dim, n_pos, *, base=10000.0, scaling=None, factor=1.0, origi
     _abi.attn_rope_table(rope_dim, n_pos, f, t.data_ptr())
     return t
 
-# "mixed": the quantised mode with 16-bit Q K^T on the causal diagonal band tiles
-_PRECISIONS = {"exact": ATTN_EXACT, "quant": ATTN_INT8QK_FP8PV, "mixed": ATTN_MIXED_DIAG}
+# "mixed": the quantised mode with 16-bit Q K^T on the causal diagonal band tiles;
+# "fp4": MXFP4 Q K^T (block-scaled MMA) with FP8 P V, head_dim 64
+_PRECISIONS = {"exact": ATTN_EXACT, "quant": ATTN_INT8QK_FP8PV, "mixed": ATTN_MIXED_DIAG,
+               "fp4": ATTN_MXFP4QK_FP8PV}
 
 
 def _stream_handle(stream):
@@ -36,22 +38,38 @@ def _stream_handle(stream):
 
 
 class QuantBuffers:
-    """Device buffers of the quantised mode (see ``attn_qbufs`` in include/attn.h)."""
+    """Device buffers of the quantised modes (see ``attn_qbufs`` in include/attn.h).
+
+    FP4 mode: ``q``/``k`` hold packed E2M1 codes ([..., D/2] bytes), ``q_sf``/``k_sf``
+    the E8M0 scale chunks, and there are no FP32 Q/K scales."""
 
     def __init__(self, params: AttnParams, device):
         B, Hq, Hk = params.batch, params.n_q_heads, params.n_kv_heads
         Sq, Sk, D = params.q_len, params.kv_len, params.head_dim
         nbq, nbk = (Sq + 127) // 128, (Sk + 127) // 128
-        self.q = torch.empty((B, Hq, Sq, D), dtype=torch.int8, device=device)
-        self.k = torch.empty((B, Hk, Sk, D), dtype=torch.int8, device=device)
-        self.q_scale = torch.empty((B, Hq, nbq), dtype=torch.float32, device=device)
-        self.k_scale = torch.empty((B, Hk, nbk), dtype=torch.float32, device=device)
+        fp4 = params.precision == ATTN_MXFP4QK_FP8PV
+        w = D // 2 if fp4 else D
+        self.q = torch.empty((B, Hq, Sq, w), dtype=torch.uint8 if fp4 else torch.int8,
+                             device=device)
+        self.k = torch.empty((B, Hk, Sk, w), dtype=torch.uint8 if fp4 else torch.int8,
+                             device=device)
+        self.q_scale = None if fp4 else torch.empty((B, Hq, nbq), dtype=torch.float32,
+                                                    device=device)
+        self.k_scale = None if fp4 else torch.empty((B, Hk, nbk), dtype=torch.float32,
+                                                    device=device)
         self.v_t = torch.empty((B, Hk, D, nbk * 128), dtype=torch.uint8, device=device)
         self.v_scale = torch.empty((B, Hk, D), dtype=torch.float32, device=device)
+        self.q_sf = self.k_sf = None
+        if fp4:
+            nq, nk = _abi.attn_qbufs_sf_sizes(params)
+            self.q_sf = torch.empty(max(nq, 16), dtype=torch.uint8, device=device)
+            self.k_sf = torch.empty(max(nk, 16), dtype=torch.uint8, device=device)
 
     def struct(self):
-        return AttnQBufs(self.q.data_ptr(), self.k.data_ptr(), self.q_scale.data_ptr(),
-                         self.k_scale.data_ptr(), self.v_t.data_ptr(), self.v_scale.data_ptr())
+        ptr = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
+        return AttnQBufs(self.q.data_ptr(), self.k.data_ptr(), ptr(self.q_scale),
+                         ptr(self.k_scale), self.v_t.data_ptr(), self.v_scale.data_ptr(),
+                         ptr(self.q_sf), ptr(self.k_sf))
 
 
 class DeviceStaging:
@@ -130,8 +148,8 @@ class Attention:
                                  f"{shape}, got {t.dtype} {tuple(t.shape)} on {t.device}")
 
     def quantize(self, q, k, v, qbufs=None, stream=None):
-        if self.precision not in ("quant", "mixed"):
-            raise ValueError("quantize() needs precision='quant' or 'mixed'")
+        if self.precision == "exact":
+            raise ValueError("quantize() needs a quantised precision ('quant', 'mixed', 'fp4')")
         self._check_inputs(q, k, v)
         qbufs = qbufs if qbufs is not None else QuantBuffers(self.params, q.device)
         _abi.attn_quantize_qk(self.ctx, q.data_ptr(), k.data_ptr(), v.data_ptr(), qbufs.struct(),
@@ -149,7 +167,7 @@ class Attention:
             lse = torch.empty((p.batch, p.n_q_heads, p.q_len), dtype=torch.float32, device=device)
         st = _stream_handle(stream)
         lse_ptr = lse.data_ptr() if lse is not None else None
-        if self.precision == "quant":
+        if self.precision in ("quant", "fp4"):
             if qbufs is None:
                 qbufs = self.quantize(q, k, v, stream=stream)
             _abi.attn_forward(self.ctx, None, None, None, qbufs.struct(), out.data_ptr(), lse_ptr, st)

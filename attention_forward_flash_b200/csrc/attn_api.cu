@@ -144,11 +144,11 @@ bool set_smem(int bytes) {
 }
 
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
-          bool DIAG = false>
+          bool DIAG = false, bool FP4 = false>
 attn_status launch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
                        cudaStream_t st) {
-  using Cfg = FwdCfg<D, NQT, QUANT, SPLIT, DIAG>;
-  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN, ROPE, DIAG>;
+  using Cfg = FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>;
+  constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN, ROPE, DIAG, FP4>;
   if (!set_smem<kern>(Cfg::kSmemBytes)) return ATTN_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(m.q, m.k, m.v, m.o, m.q16, m.k16, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -161,6 +161,12 @@ attn_status dispatch_win(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, 
   if constexpr (QUANT) {
     if (c->p.precision == ATTN_MIXED_DIAG)
       return launch_fwd<D, 2, true, F16, false, false, WIN, false, true>(c, m, a, grid, st);
+  }
+  // the FP4 mode (head_dim 64): single-pass kernel with block-scaled MXFP4 Q K^T
+  if constexpr (QUANT && D == 64) {
+    if (c->p.precision == ATTN_MXFP4QK_FP8PV)
+      return launch_fwd<D, 2, true, F16, false, false, WIN, false, false, true>(c, m, a, grid,
+                                                                                st);
   }
   if (c->split_path)
     return launch_fwd<D, 1, QUANT, F16, true, true, WIN, ROPE>(c, m, a, grid, st);
@@ -229,9 +235,14 @@ attn_status validate(const attn_params* p) {
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_INVALID_ARG;
   if (p->precision != ATTN_EXACT && p->precision != ATTN_INT8QK_FP8PV &&
-      p->precision != ATTN_MIXED_DIAG)
+      p->precision != ATTN_MIXED_DIAG && p->precision != ATTN_MXFP4QK_FP8PV)
     return ATTN_ERR_INVALID_ARG;
-  if (p->precision == ATTN_MIXED_DIAG && p->num_splits > 1) return ATTN_ERR_INVALID_ARG;
+  const bool single_pass_mode =
+      p->precision == ATTN_MIXED_DIAG || p->precision == ATTN_MXFP4QK_FP8PV;
+  if (single_pass_mode && p->num_splits > 1) return ATTN_ERR_INVALID_ARG;
+  // FP4: the scale factors fit tensor memory beside head_dim-64 scores and outputs only
+  if (p->precision == ATTN_MXFP4QK_FP8PV && (p->head_dim != 64 || p->rope_dim > 0))
+    return ATTN_ERR_UNSUPPORTED;
   // the band tiles read the caller's 16-bit Q and K, which the quantiser's RoPE never sees
   if (p->precision == ATTN_MIXED_DIAG && p->rope_dim > 0) return ATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
@@ -255,9 +266,21 @@ bool bad_ptr(const void* ptr, bool needed) {
 
 bool bad_qbufs(const attn_params& p, const attn_qbufs* qb) {
   const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
-  return !qb || bad_ptr(qb->q, need_q) || bad_ptr(qb->q_scale, need_q) ||
+  if (!qb) return true;
+  if (p.precision == ATTN_MXFP4QK_FP8PV)  // packed codes and scale chunks; no FP32 scales
+    return bad_ptr(qb->q, need_q) || bad_ptr(qb->q_sf, need_q) || bad_ptr(qb->k, need_kv) ||
+           bad_ptr(qb->k_sf, need_kv) || bad_ptr(qb->v_t, need_kv) ||
+           bad_ptr(qb->v_scale, need_kv);
+  return bad_ptr(qb->q, need_q) || bad_ptr(qb->q_scale, need_q) ||
          bad_ptr(qb->k, need_kv) || bad_ptr(qb->k_scale, need_kv) || bad_ptr(qb->v_t, need_kv) ||
          bad_ptr(qb->v_scale, need_kv);
+}
+
+// FP4 mode: 128-row scale chunks per unit of Q (an even count: the two-tile CTAs
+// always read two) and of K.
+int fp4_q_tiles(const attn_params& p) {
+  const long long R = static_cast<long long>(p.n_q_heads / p.n_kv_heads) * p.q_len;
+  return 2 * static_cast<int>((R + 255) / 256);
 }
 
 attn_status check_forward_buffers(const attn_ctx* c, const void* q, const void* k, const void* v,
@@ -267,7 +290,7 @@ attn_status check_forward_buffers(const attn_ctx* c, const void* q, const void* 
   if (bad_ptr(o, need_q) || (lse && !aligned16(lse))) return ATTN_ERR_INVALID_ARG;
   if (p.precision == ATTN_MIXED_DIAG) {  // codes and the 16-bit Q and K
     if (bad_qbufs(p, qb) || bad_ptr(q, need_q) || bad_ptr(k, need_kv)) return ATTN_ERR_INVALID_ARG;
-  } else if (p.precision == ATTN_INT8QK_FP8PV) {
+  } else if (p.precision != ATTN_EXACT) {  // the quantised and FP4 modes read the codes only
     if (bad_qbufs(p, qb)) return ATTN_ERR_INVALID_ARG;
   } else {
     if (qb) return ATTN_ERR_INVALID_ARG;
@@ -317,6 +340,21 @@ attn_status quant_qk_launch(const attn_ctx* c, const uint16_t* x, int8_t* codes,
   return ATTN_OK;
 }
 
+// V's channel maxima, then its transposed E4M3 codes (both quantised modes).
+template <int D, bool F16>
+attn_status v_launch(attn_ctx* c, const uint16_t* vx, unsigned* vamax, uint8_t* vt, float* vs,
+                     int nbk, unsigned BHk, cudaStream_t st) {
+  const attn_params& p = c->p;
+  const int tot = nbk * static_cast<int>(BHk);
+  v_amax_kernel<D, F16><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(vx, vamax,
+                                                                             p.kv_len);
+  if (!set_smem<v_quant_kernel<D, F16>>(VQuantCfg<D>::kSmemBytes)) return ATTN_ERR_CUDA;
+  const int vq_ctas = std::min(tot, VQuantCfg<D>::kCtasPerSm * c->num_sms);
+  v_quant_kernel<D, F16><<<vq_ctas, 256, VQuantCfg<D>::kSmemBytes, st>>>(
+      vx, vamax, vt, vs, p.kv_len, nbk * 128, nbk, tot, c->err);
+  return ATTN_OK;
+}
+
 // The quantisers of one range of units: Q and K blocks (rotated first with RoPE),
 // then V's channel maxima and codes.
 template <int D, bool F16>
@@ -339,12 +377,7 @@ attn_status quant_launch(attn_ctx* c, const uint16_t* qx, int8_t* qc, float* qs,
     s = rope_k ? quant_qk_launch<D, F16, true>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st)
                : quant_qk_launch<D, F16, false>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st);
     if (s != ATTN_OK) return s;
-    v_amax_kernel<D, F16><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(vx, vamax,
-                                                                               p.kv_len);
-    if (!set_smem<v_quant_kernel<D, F16>>(VQuantCfg<D>::kSmemBytes)) return ATTN_ERR_CUDA;
-    const int vq_ctas = std::min(tot, VQuantCfg<D>::kCtasPerSm * c->num_sms);
-    v_quant_kernel<D, F16><<<vq_ctas, 256, VQuantCfg<D>::kSmemBytes, st>>>(
-        vx, vamax, vt, vs, p.kv_len, nbk * 128, nbk, tot, c->err);
+    return v_launch<D, F16>(c, vx, vamax, vt, vs, nbk, BHk, st);
   }
   return ATTN_OK;
 }
@@ -368,9 +401,10 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
   const uint16_t* kx = static_cast<const uint16_t*>(k) + (nbk > 0 ? ke : 0);
   const uint16_t* vx = static_cast<const uint16_t*>(v) + (nbk > 0 ? ke : 0);
   int8_t* qc = nbq > 0 ? qb->q + qe : nullptr;
-  float* qs = nbq > 0 ? qb->q_scale + static_cast<size_t>(u0) * c->G * nbq : nullptr;
+  float* qs = (nbq > 0 && qb->q_scale) ? qb->q_scale + static_cast<size_t>(u0) * c->G * nbq
+                                       : nullptr;
   int8_t* kc = nbk > 0 ? qb->k + ke : nullptr;
-  float* ks = nbk > 0 ? qb->k_scale + static_cast<size_t>(u0) * nbk : nullptr;
+  float* ks = (nbk > 0 && qb->k_scale) ? qb->k_scale + static_cast<size_t>(u0) * nbk : nullptr;
   uint8_t* vt = nbk > 0 ? qb->v_t + static_cast<size_t>(u0) * D * S_pad : nullptr;
   float* vs = nbk > 0 ? qb->v_scale + static_cast<size_t>(u0) * D : nullptr;
   unsigned* vamax = nbk > 0 ? c->v_amax + static_cast<size_t>(u0) * D : nullptr;
@@ -378,6 +412,28 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
   if (nbk > 0 &&
       cudaMemsetAsync(vamax, 0, static_cast<size_t>(nu) * D * 4, st) != cudaSuccess)
     return ATTN_ERR_CUDA;
+  if (p.precision == ATTN_MXFP4QK_FP8PV) {
+    // Q and K to MXFP4 (packed E2M1 codes and E8M0 scale chunks; head_dim 64), V as in
+    // the quantised mode.  Q's rows are each unit's stacked query rows.
+    const int qt = fp4_q_tiles(p);
+    uint8_t* qcodes = reinterpret_cast<uint8_t*>(qb->q) + static_cast<size_t>(u0) * c->R * (D / 2);
+    uint8_t* kcodes =
+        reinterpret_cast<uint8_t*>(qb->k) + static_cast<size_t>(u0) * p.kv_len * (D / 2);
+    uint8_t* qsf = qb->q_sf + static_cast<size_t>(u0) * qt * 512;
+    uint8_t* ksf = qb->k_sf + static_cast<size_t>(u0) * nbk * 512;
+    if (nbq > 0) {
+      if (f16) mxfp4_qk_kernel<true><<<dim3(qt, nu), 256, 0, st>>>(qx, qcodes, qsf, c->R, qt);
+      else mxfp4_qk_kernel<false><<<dim3(qt, nu), 256, 0, st>>>(qx, qcodes, qsf, c->R, qt);
+    }
+    if (nbk > 0) {
+      if (f16) mxfp4_qk_kernel<true><<<dim3(nbk, nu), 256, 0, st>>>(kx, kcodes, ksf, p.kv_len, nbk);
+      else mxfp4_qk_kernel<false><<<dim3(nbk, nu), 256, 0, st>>>(kx, kcodes, ksf, p.kv_len, nbk);
+      const attn_status vs_st = f16 ? v_launch<64, true>(c, vx, vamax, vt, vs, nbk, BHk, st)
+                                    : v_launch<64, false>(c, vx, vamax, vt, vs, nbk, BHk, st);
+      if (vs_st != ATTN_OK) return vs_st;
+    }
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
   // RoPE: Q rows at start_pos + token, K rows at token (unless already rotated)
   const bool rope = p.rope_dim > 0;
   const QuantRope rq{c->rope_table, p.rope_dim, p.rope_interleaved, p.start_pos};
@@ -425,12 +481,19 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
   }
   attn_qbufs qo{};
+  const bool fp4 = p.precision == ATTN_MXFP4QK_FP8PV;
   if (quant) {
     const int nbq = ceil_div(p.q_len, 128), nbk = ceil_div(p.kv_len, 128);
-    qo.q = qb->q + qe;
-    qo.k = qb->k + ke;
-    qo.q_scale = qb->q_scale + static_cast<size_t>(u0) * c->G * nbq;
-    qo.k_scale = qb->k_scale + static_cast<size_t>(u0) * nbk;
+    const size_t half = fp4 ? 2 : 1;  // FP4: two codes per byte
+    qo.q = qb->q + qe / half;
+    qo.k = qb->k + ke / half;
+    if (fp4) {
+      qo.q_sf = qb->q_sf + static_cast<size_t>(u0) * fp4_q_tiles(p) * 512;
+      qo.k_sf = qb->k_sf + static_cast<size_t>(u0) * nbk * 512;
+    } else {
+      qo.q_scale = qb->q_scale + static_cast<size_t>(u0) * c->G * nbq;
+      qo.k_scale = qb->k_scale + static_cast<size_t>(u0) * nbk;
+    }
     qo.v_t = qb->v_t + static_cast<size_t>(u0) * D * (static_cast<size_t>(nbk) * 128);
     qo.v_scale = qb->v_scale + static_cast<size_t>(u0) * D;
     qb = &qo;
@@ -465,10 +528,12 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
   if (hit) {
   } else if (quant) {
     const CUtensorMapSwizzle sw8 =
-        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+        fp4 ? CU_TENSOR_MAP_SWIZZLE_32B
+            : (D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
     const uint64_t S_pad = static_cast<uint64_t>(ceil_div(p.kv_len, 128)) * 128;
-    ok &= make_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, D, R, U, D, R * D, D, 128, sw8);
-    ok &= make_map(&m.k, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, D, Sk, U, D, Sk * D, D, 128, sw8);
+    const uint64_t W = fp4 ? D / 2 : D;  // bytes per row of the Q/K codes
+    ok &= make_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->q, W, R, U, W, R * W, W, 128, sw8);
+    ok &= make_map(&m.k, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->k, W, Sk, U, W, Sk * W, W, 128, sw8);
     ok &= make_map(&m.v, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb->v_t, S_pad, D, U, S_pad, S_pad * D,
                    128, D, CU_TENSOR_MAP_SWIZZLE_128B);
     if (diag) {
@@ -525,6 +590,11 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
     a.rope_table = c->rope_table;
     a.rope_R = p.rope_dim;
     a.rope_inter = p.rope_interleaved;
+  }
+  if (fp4) {
+    a.q_sf = qb->q_sf;
+    a.k_sf = qb->k_sf;
+    a.q_tiles = fp4_q_tiles(p);
   }
   a.tph = causal_band_tiles(c);
   const int grid = nu * c->row_tiles * (c->split_path ? c->splits : 1);
@@ -643,6 +713,24 @@ attn_status attn_qbufs_sizes(const attn_params* p, size_t sizes[6]) {
   sizes[3] = B * Hk * nbk * 4;
   sizes[4] = B * Hk * D * nbk * 128;
   sizes[5] = B * Hk * D * 4;
+  if (p->precision == ATTN_MXFP4QK_FP8PV) {  // packed E2M1 codes; no FP32 Q/K scales
+    sizes[0] /= 2;
+    sizes[1] /= 2;
+    sizes[2] = sizes[3] = 0;
+  }
+  return ATTN_OK;
+}
+
+attn_status attn_qbufs_sf_sizes(const attn_params* p, size_t sizes[2]) {
+  if (!sizes) return ATTN_ERR_INVALID_ARG;
+  attn_status v = validate(p);
+  if (v != ATTN_OK) return v;
+  sizes[0] = sizes[1] = 0;
+  if (p->precision == ATTN_MXFP4QK_FP8PV) {
+    const size_t units = static_cast<size_t>(p->batch) * p->n_kv_heads;
+    sizes[0] = units * fp4_q_tiles(*p) * 512;
+    sizes[1] = units * ((static_cast<size_t>(p->kv_len) + 127) / 128) * 512;
+  }
   return ATTN_OK;
 }
 
@@ -675,8 +763,8 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   const int big_ctas = c->units * ceil_div(c->R, 256);
   bool split = false;
   int splits = 1;
-  if (p->precision == ATTN_MIXED_DIAG) {
-    // single-pass kernel only (the band mode has no split-KV variant)
+  if (p->precision == ATTN_MIXED_DIAG || p->precision == ATTN_MXFP4QK_FP8PV) {
+    // single-pass kernel only (the band and FP4 modes have no split-KV variant)
   } else if (p->num_splits > 1) {
     split = true;
     splits = p->num_splits;

@@ -80,6 +80,11 @@ struct FwdArgs {
   const float* rope_table;  // [n_pos][2][rope_R/2] float32
   int rope_R;               // rotated channels (multiple of 16)
   int rope_inter;           // interleaved pairs
+  // FP4 mode: E8M0 scale chunks (512 bytes per 128-row tile) of Q, per unit
+  // [units][q_tiles], and of K, per unit [units][nblk_k]
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  int q_tiles;
 };
 
 constexpr int kErrTimeout = 1;
@@ -87,21 +92,28 @@ constexpr int kErrTimeout = 1;
 // DIAG (quantised mode only): the key tiles of the causal diagonal band get
 // Q K^T from the 16-bit inputs; 16-bit Q tiles sit next to the INT8 ones and one
 // 16-bit K tile buffer serves the band tiles (the ring carries the rest).
-template <int D, int NQT, bool QUANT, bool SPLIT, bool DIAG = false>
+// FP4 (quantised mode, head_dim 64): Q and K are packed E2M1 (half a byte per
+// element) with E8M0 scale chunks (512 bytes per 128-row tile) that the MMA warp
+// copies into tensor memory; a K slot holds the tile and, after it, its chunk.
+template <int D, int NQT, bool QUANT, bool SPLIT, bool DIAG = false, bool FP4 = false>
 struct FwdCfg {
   static_assert(!DIAG || (QUANT && !SPLIT), "the diagonal band mode is a single-pass quantised kernel");
+  static_assert(!FP4 || (QUANT && !SPLIT && !DIAG && D == 64), "the FP4 mode: single pass, head_dim 64");
   static constexpr int kThreads = 128 * (1 + NQT);
   static constexpr int kElem = QUANT ? 1 : 2;                 // bytes per Q/K element
-  static constexpr int kQTile = 128 * D * kElem;              // one 128-row Q tile
-  static constexpr int kKTile = 128 * D * kElem;
+  static constexpr int kQTile = FP4 ? 128 * D / 2 : 128 * D * kElem;  // one 128-row Q tile
+  static constexpr int kKTile = FP4 ? 128 * D / 2 : 128 * D * kElem;
+  static constexpr int kSfChunk = 512;                        // FP4: scales of a 128-row tile
+  static constexpr int kKSlotBytes = kKTile + (FP4 ? kSfChunk : 0);
   static constexpr int kVTile = 128 * D * (QUANT ? 1 : 2);
-  static constexpr int kSlot = kKTile > kVTile ? kKTile : kVTile;
+  static constexpr int kSlot = kKSlotBytes > kVTile ? kKSlotBytes : kVTile;
   static constexpr int kOStage = 128 * D * 2;                 // 16-bit output tile
   static constexpr int kQ16Tile = DIAG ? 128 * D * 2 : 0;     // 16-bit Q tile (DIAG)
   static constexpr int kKdBytes = DIAG ? 128 * D * 2 : 0;     // 16-bit K tile (DIAG)
   static constexpr bool kStageInQ = (kQTile >= kOStage);
   static constexpr int kStageBytes = (SPLIT || kStageInQ || DIAG) ? 0 : NQT * kOStage;
-  static constexpr int kFixed = NQT * (kQTile + kQ16Tile) + kKdBytes + kStageBytes;
+  static constexpr int kSfaBytes = FP4 ? NQT * kSfChunk : 0;  // FP4: Q tiles' scale chunks
+  static constexpr int kFixed = NQT * (kQTile + kQ16Tile) + kKdBytes + kStageBytes + kSfaBytes;
   // (the band mode's extra 16-bit tiles would leave a 4-slot ring at 200 KB; it takes
   // up to 224 KB of the 227 KB a CTA may use, for 6 slots at head_dim 128)
   static constexpr int kBudget = (DIAG ? 224 : 200) * 1024;
@@ -116,6 +128,7 @@ struct FwdCfg {
   static constexpr int kKdOff = kQ16Off + NQT * kQ16Tile;     // DIAG: 16-bit K tile
   // output staging: its own buffers, or the Q tiles (16-bit Q tiles in DIAG)
   static constexpr int kStageOff = DIAG ? kQ16Off : NQT * kQTile;
+  static constexpr int kSfaOff = kStageOff + kStageBytes;     // FP4 (after the staging)
   static constexpr int kStageTile = DIAG ? kQ16Tile : (kStageInQ ? kQTile : kOStage);
   static constexpr bool kStageInQBuf = kStageInQ && !DIAG;
   static constexpr int kRingOff = kFixed;
@@ -128,11 +141,13 @@ struct FwdCfg {
   static constexpr int kSvOff = kMiscOff + 16;                  // v scales (quant)
   static constexpr int kSmemBytes = kSvOff + (QUANT ? D * 4 : 0) + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
-  static constexpr int kTmemNeed = NQT * (128 + D);
+  // FP4: 4 scale-factor columns per Q tile and two K buffers after S and O
+  static constexpr int kSfCols = FP4 ? 4 * NQT + 8 : 0;
+  static constexpr int kTmemNeed = NQT * (128 + D) + kSfCols;
   static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
   // transaction bytes
-  static constexpr uint32_t kQBytes = NQT * (kQTile + kQ16Tile);
-  static constexpr uint32_t kKBytes = kKTile;
+  static constexpr uint32_t kQBytes = NQT * (kQTile + kQ16Tile) + kSfaBytes;
+  static constexpr uint32_t kKBytes = kKSlotBytes;
   static constexpr uint32_t kVBytes = kVTile;
   // softmax rescale threshold (base-2 units): O and l are rescaled only when a
   // row max grows by more than this, so P <= 2^thresh.  Quantised: P is scaled by
@@ -314,16 +329,16 @@ __device__ __forceinline__ void rope_q_row(uint32_t tile, int row, const float* 
 // warpgroups rotate the staged Q tile before the first Q K^T (the keys arrive
 // rotated).
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
-          bool DIAG = false>
-__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
-                                  FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kCtasPerSm)
+          bool DIAG = false, bool FP4 = false>
+__global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>::kThreads,
+                                  FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>::kCtasPerSm)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_o,
                      const __grid_constant__ CUtensorMap tm_q16,
                      const __grid_constant__ CUtensorMap tm_k16, const FwdArgs a) {
-  using C = FwdCfg<D, NQT, QUANT, SPLIT, DIAG>;
+  using C = FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>;
   static_assert(!SPLIT || LF, "the split variant always needs the float32 row sum");
   static_assert(!(ROPE && QUANT), "the quantised mode rotates Q and K in its quantiser");
   extern __shared__ uint8_t smem_raw[];
@@ -457,14 +472,20 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      constexpr int kBoxCols = QUANT ? D : 64;         // elements per box row
+      constexpr int kBoxCols = FP4 ? D / 2 : (QUANT ? D : 64);  // box row (elements, FP4 bytes)
       constexpr int kQBoxes = QUANT ? 1 : D / 64;
-      constexpr int kQBox = 128 * kBoxCols * C::kElem;
+      constexpr int kQBox = FP4 ? C::kQTile : 128 * kBoxCols * C::kElem;
       mbar_arrive_expect_tx(q_full, C::kQBytes);
       for (int q = 0; q < NQT; ++q)
         for (int bx = 0; bx < kQBoxes; ++bx)
           tma_load_3d(&tm_q, sbase + C::kQOff + q * C::kQTile + bx * kQBox, q_full,
                       bx * kBoxCols, r0 + q * 128, u);
+      if constexpr (FP4) {  // the Q tiles' scale chunks (every unit has an even count)
+        for (int q = 0; q < NQT; ++q)
+          bulk_load(sbase + C::kSfaOff + q * C::kSfChunk,
+                    a.q_sf + ((size_t)u * a.q_tiles + r0 / 128 + q) * C::kSfChunk, C::kSfChunk,
+                    q_full);
+      }
       if constexpr (DIAG) {  // the 16-bit Q tiles, for the band's Q K^T
         prefetch_tmap(&tm_q16);
         prefetch_tmap(&tm_k16);
@@ -515,7 +536,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
               tma_load_4d(m, dst + bx * 128 * 64 * 2, full_bar(s), bx * 64, 0, hk, blk);
           } else if (part == 0) {
             mbar_arrive_expect_tx(full_bar(s), C::kKBytes);
-            if constexpr (QUANT) {
+            if constexpr (FP4) {  // the packed tile, then its scale chunk after it
+              tma_load_3d(&tm_k, dst, full_bar(s), 0, kv0, u);
+              bulk_load(dst + C::kKTile, a.k_sf + ((size_t)u * a.nblk_k + jt0 + j) * C::kSfChunk,
+                        C::kSfChunk, full_bar(s));
+            } else if constexpr (QUANT) {
               tma_load_3d(&tm_k, dst, full_bar(s), 0, kv0, u);
             } else {
               for (int bx = 0; bx < D / 64; ++bx)
@@ -564,6 +589,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
       bool ok = mbar_wait(ROPE ? q_rot : q_full, 0, abort_flag);
       if (!ok) raise();
       int it = 0;
+      if constexpr (FP4) {  // the Q tiles' scale factors, once
+        if (ok) {
+          tc_fence_after();
+          for (int q = 0; q < NQT; ++q)
+            tmem_cp_32x128b_x4(tmem + NQT * (128 + D) + 4 * q,
+                               desc_pack(desc_lo(sbase + C::kSfaOff + q * C::kSfChunk, 16),
+                                         desc_hi(128u, 0u)));
+        }
+      }
 
       // Descriptor words: the high word is fixed per operand kind; the low word
       // is the start address (>> 4) plus a compile-time offset per K step.
@@ -590,10 +624,25 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
         }
       };
       int kd_it = 0;  // band K tiles consumed
+      // FP4: block-scaled MXFP4 Q K^T (K = 64 = the whole row of 32 bytes, 32-byte
+      // swizzle, SBO 256).  Scale factors in tensor memory after S and O: the Q tiles'
+      // (copied once) and two K buffers (copied per tile, alternating).
+      constexpr uint32_t idesc_qk4 = instr_desc_mx(1, 1, 128, 128);
+      constexpr uint32_t hi_4 = desc_hi(256u, 6u);
+      const uint32_t sf_col = tmem + NQT * (128 + D);
+      int k_sf_it = 0;
+      auto copy_k_sf = [&](int slot) {  // the K tile's chunk, behind the tile in its slot
+        const uint32_t src = sbase + C::kRingOff + slot * C::kSlot + C::kKTile;
+        tmem_cp_32x128b_x4(sf_col + 4 * NQT + 4 * (k_sf_it & 1),
+                           desc_pack(desc_lo(src, 16), desc_hi(128u, 0u)));
+      };
       auto issue_qk = [&](int q, uint32_t k_lo) {
         const uint32_t q_lo = q_lo0 + q * (C::kQTile >> 4);
         const uint32_t d = tmem + q * 128;
-        if constexpr (QUANT) {
+        if constexpr (FP4) {
+          mma_mxf4_ss(d, desc_pack(q_lo, hi_4), desc_pack(k_lo, hi_4), idesc_qk4, sf_col + 4 * q,
+                      sf_col + 4 * NQT + 4 * (k_sf_it & 1), 0u);
+        } else if constexpr (QUANT) {
           // int8, K = D bytes per row: one swizzle atom column (128 B, or 64 B at D = 64)
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
@@ -648,12 +697,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
         else {
           tc_fence_after();
           const uint32_t k_lo = ring_lo + s * (C::kSlot >> 4);
+          if constexpr (FP4) copy_k_sf(s);
           for (int q = 0; q < NQT; ++q) {
             issue_qk(q, k_lo);
             tc_commit(s_ready(q));
           }
           tc_commit(empty_bar(s));
           ++it;
+          ++k_sf_it;
         }
       }
       for (int j = 0; j < n && ok; ++j) {
@@ -673,6 +724,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
         tc_fence_after();
         const uint32_t v_lo = ring_lo_v + sv * (C::kSlot >> 4);
         const uint32_t k_lo = ring_lo + sk * (C::kSlot >> 4);
+        if constexpr (FP4) {
+          if (has_next && !next_band) copy_k_sf(sk);
+        }
         for (int q = 0; q < NQT && ok; ++q) {
           // The first half of P.V runs while the softmax still writes the second.
           for (int h = 0; h < 2; ++h) {
@@ -695,6 +749,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
           ++kd_it;
         } else if (ok && has_next) {
           tc_commit(empty_bar(sk));
+          ++k_sf_it;
         }
       }
       tc_commit(o_final);
@@ -721,7 +776,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
     const uint32_t tS = tmem + lane_off + q * 128;
     const uint32_t tO = tmem + lane_off + NQT * 128 + q * D;
     float qsc = 1.0f;
-    if constexpr (QUANT) {
+    if constexpr (QUANT && !FP4) {  // (FP4: the scales are applied inside the MMA)
       const int g = ri / a.Sq;
       qsc = a.q_scale[((size_t)u * a.G + g) * a.nblk_q + i / 128];
     }
@@ -732,9 +787,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
     bool ok = true;
     // Quantised: the K block scale of tile j is loaded one tile ahead (a pinned
     // load, so that its latency hides behind the previous tile's softmax).
-    const float* ksrc = QUANT ? a.k_scale + (size_t)u * a.nblk_k + jt0 : nullptr;
+    const float* ksrc = (QUANT && !FP4) ? a.k_scale + (size_t)u * a.nblk_k + jt0 : nullptr;
     float ksc_next = 1.0f;
-    if constexpr (QUANT)
+    if constexpr (QUANT && !FP4)
       if (n > 0) ksc_next = ld_global_f32(ksrc);
     constexpr int kPoly = QUANT ? kPolyEveryQ : kPolyEvery;
     if constexpr (ROPE) {
@@ -771,9 +826,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
       __syncwarp();
       if (lane == 0) mbar_arrive(p_ready(q, h));
     };
-    if constexpr (!DIAG) {
+    if constexpr (!DIAG && !FP4) {
     // (the kernels without the band mode keep this straight-line form of the tile loop;
-    // the band mode below compiles the tile body once per kind of score)
+    // the band and FP4 modes below compile the tile body once per kind of score)
     for (int j = 0; j < n && ok; ++j) {
       const float ksc = ksc_next;
       if constexpr (QUANT)
@@ -909,9 +964,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
     } else {
     for (int j = 0; j < n && ok; ++j) {
       const float ksc = ksc_next;
-      if constexpr (QUANT)
+      if constexpr (QUANT && !FP4)
         if (j + 1 < n) ksc_next = ld_global_f32(ksrc + j + 1);
-      // DIAG: a band tile's scores are float32 products of the 16-bit inputs
+      // DIAG: a band tile's scores are float32 products of the 16-bit inputs; FP4:
+      // every tile's are (block-scaled MMA)
       const bool band = in_band(jt0 + j);
       // The tile's body, compiled once per kind of score: FS (the diagonal band
       // mode's band tiles) reads float32 scores, otherwise INT8 products (quantised)
@@ -1054,10 +1110,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG>::kThreads,
         }
         return true;
       };
-      if (DIAG && band)
+      if constexpr (FP4) {
         ok = tile(std::true_type{});
-      else
-        ok = tile(std::false_type{});
+      } else {
+        if (DIAG && band)
+          ok = tile(std::true_type{});
+        else
+          ok = tile(std::false_type{});
+      }
     }
     }
 

@@ -213,6 +213,35 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d, uint32_t a_tmem, uint64_t 
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T for MXFP4 operands (E2M1 elements, one E8M0
+// scale per 32 along K), K = 64 per instruction; the two scales of a row are
+// bytes `id`, id + 1 of its 32-bit cell at sfa / sfb (the id is carried in the
+// top two bits of the tensor-memory address).
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], "
+      "[%5], p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accum)
+      : "memory");
+}
+
+// Copies 32 rows x 16 bytes from shared memory (descriptor `src`) into 4 columns of
+// tensor memory at `taddr`, the same data into each of the four 32-lane quarters
+// (the layout of block scale factors for a 128-row operand).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src)
+               : "memory");
+}
+
+// Instruction descriptor of the block-scaled kinds: A and B formats (E2M1 = 1 in
+// kind::mxf4), N / 8 at bit 17, E8M0 scales (bit 23), M / 16 at bit 24.
+__host__ __device__ constexpr uint32_t instr_desc_mx(uint32_t a_fmt, uint32_t b_fmt, uint32_t M,
+                                                     uint32_t N) {
+  return (a_fmt << 7) | (b_fmt << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor (Blackwell layout: version 1 in bits 46-47).
 // layout: 0 = no swizzle, 2 = 128-byte swizzle, 4 = 64-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,

@@ -259,6 +259,71 @@ __global__ void __launch_bounds__(256, QuantQkCfg<D, ROPE>::kCtasPerSm) quant_qk
   }
 }
 
+// MXFP4 quantiser of the FP4 mode (head_dim 64), after the OCP Microscaling
+// Formats conversion: per row and block of 32 channels, the E8M0 scale 2^e with
+// e = floor(log2(amax)) - 2 (2 is the largest E2M1 exponent; clamped to
+// [-127, 127]; amax = 0 gives e = -127), and codes E2M1(x * 2^-e) rounded to
+// nearest-even and saturated to +-6 (cvt.rn.satfinite.e2m1x2).  x * 2^-e is an
+// exact power-of-two scaling (a result that would be subnormal is far below
+// E2M1's resolution and rounds to zero either way).
+//
+// Rows come as `nseq` sequences of L rows (Q: the G * Sq stacked rows of a unit;
+// K: the keys of a (batch, kv head)); each sequence has `tiles` 128-row tiles
+// (at least ceil(L / 128); rows past L are padding).  Block = one tile, thread =
+// (row, channel block): codes [row][32 B] (channel 2i in the low nibble), scales
+// in the tensor core's 512-byte chunk per tile: row r, block b at byte
+// (r % 32) * 16 + (r / 32) * 4 + b; padding rows and the unused bytes b = 2, 3
+// hold 127 (scale 1).
+template <bool F16>
+__global__ void __launch_bounds__(256) mxfp4_qk_kernel(const uint16_t* __restrict__ x,
+                                                       uint8_t* __restrict__ codes,
+                                                       uint8_t* __restrict__ sf, int L, int tiles) {
+  const int seq = blockIdx.y, t = blockIdx.x;
+  const int r = threadIdx.x >> 1, b = threadIdx.x & 1;
+  const int row = t * 128 + r;
+  uint8_t* chunk = sf + ((size_t)seq * tiles + t) * 512 + (r & 31) * 16 + (r >> 5) * 4;
+  if (row >= L) {
+    chunk[b] = 127;
+    chunk[2 + b] = 127;
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)seq * L + row) * 64 + 32 * b);
+  float f[32];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float g[8];
+    unpack8<F16>(ld_nc_v4(src + k), g);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[8 * k + e] = g[e];
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(f[e]));
+  int ex = amax > 0.0f ? ilogbf(amax) - 2 : -127;
+  ex = max(-127, min(127, ex));
+  chunk[b] = static_cast<uint8_t>(ex + 127);
+  chunk[2 + b] = 127;
+  const float inv = __int_as_float((127 - ex) << 23);  // 2^-ex, a normal float for ex <= 126
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 8 * k + 2 * i;
+      uint16_t pair;
+      // the first source lands in the high nibble: channel e + 1 high, e low
+      asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+          : "=h"(pair)
+          : "f"(__fmul_rn(f[e + 1], inv)), "f"(__fmul_rn(f[e], inv)));
+      word |= static_cast<uint32_t>(pair & 0xFF) << (8 * i);
+    }
+    w[k] = word;
+  }
+  *reinterpret_cast<uint4*>(codes + ((size_t)seq * L + row) * 32 + 16 * b) =
+      make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // grid: (ceil(S/kVTok), B*Hkv), 256 threads.  Channel maxima of |V| as float
 // bit patterns (non-negative floats order like unsigned integers).
 constexpr int kVTok = 256;

@@ -82,7 +82,8 @@ WORKLOADS = {
                        seed=1001),
     "decode_window": Workload("decode_window", 1, 16, 8, 4, 4133, 128, "fp16", causal=True,
                               start_pos=4129, window_lo=40, seed=1011),
-    "image": Workload("image", 2, 10, 10, 4096, 4096, 64, "bf16", modes=("exact", "quant"),
+    "image": Workload("image", 2, 10, 10, 4096, 4096, 64, "bf16",
+                      modes=("exact", "quant", "fp4"),
                       seed=1002, k_channel_offset_var=2.0),
     "video": Workload("video", 1, 40, 40, 32760, 32760, 128, "bf16", modes=("exact", "quant"),
                       seed=1003, oracle_rows=256),

@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video", choices=sorted(WORKLOADS))
-    ap.add_argument("--precision", default="exact", choices=["exact", "quant", "mixed"])
+    ap.add_argument("--precision", default="exact", choices=["exact", "quant", "mixed", "fp4"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -502,12 +502,14 @@ def run_native(args):
         ms_q = time_steps(lambda: att.quantize(q, k, v, qbufs=qb), args.steps, 2)
         q_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, v))
         q_bytes += sum(t.numel() * t.element_size()
-                       for t in (qb.q, qb.k, qb.q_scale, qb.k_scale, qb.v_t, qb.v_scale))
+                       for t in (qb.q, qb.k, qb.q_scale, qb.k_scale, qb.v_t, qb.v_scale,
+                                 qb.q_sf, qb.k_sf) if t is not None)
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         gbs = q_bytes / (ms_q * 1e-3) / 1e9
         quantiser = {"bound": "hbm", "ms": ms_q, "bytes": q_bytes, "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm,
-                     "kernels": "quant_qk_kernel (Q, K), v_amax_kernel, v_quant_kernel"}
+                     "kernels": ("mxfp4_qk_kernel (Q, K)" if precision == "fp4"
+                                 else "quant_qk_kernel (Q, K)") + ", v_amax_kernel, v_quant_kernel"}
     att.check_error()
 
     # ---- end to end through the public API with host buffers
@@ -540,7 +542,8 @@ def run_native(args):
                            ("llm", "exact"), ("llm", "quant"), ("image", "exact"),
                            ("image", "quant"), ("decode", "exact"), ("decode_window", "exact"),
                            ("llm_window", "exact"), ("video_rope", "exact"),
-                           ("video_rope", "quant"), ("llm_rope", "exact"), ("llm", "mixed")):
+                           ("video_rope", "quant"), ("llm_rope", "exact"), ("llm", "mixed"),
+                           ("image", "fp4")):
             if name == w.name and prec == precision:
                 continue
             wx = WORKLOADS[name]

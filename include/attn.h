@@ -72,8 +72,22 @@ typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype;
  * diagonal band -- the tiles some row of a 256-row query tile must partly mask --
  * get Q K^T from the 16-bit inputs (float32 scores); P and V stay FP8 E4M3.
  * Without a causal mask there is no band and it computes what ATTN_INT8QK_FP8PV
- * does.  It always runs the single-pass kernel (num_splits 0 or 1). */
-typedef enum { ATTN_EXACT = 0, ATTN_INT8QK_FP8PV = 1, ATTN_MIXED_DIAG = 2 } attn_precision;
+ * does.  It always runs the single-pass kernel (num_splits 0 or 1).
+ * ATTN_MXFP4QK_FP8PV is opt-in: the FP4 microscaled mode.  Q and K are quantised to
+ * MXFP4 (OCP Microscaling: E2M1 elements, one E8M0 power-of-two scale per 32
+ * channels of a row) and Q K^T runs on the block-scaled tensor-core MMA; P and V
+ * stay FP8 E4M3 as in ATTN_INT8QK_FP8PV.  FP4 attention and the MXFP formats on B200
+ * are named on the pages "Ядра attention на домашней RTX 5080" (table of section
+ * "1 · Только ядро", SageAttention 3) and "Transformers Get a Turbo Boost with
+ * Mixed-Precision Magic".  head_dim 64 only: the scale factors live in tensor
+ * memory, which the head_dim-128 kernel fills with its scores and outputs.  Single-
+ * pass kernel only (num_splits 0 or 1); no RoPE. */
+typedef enum {
+  ATTN_EXACT = 0,
+  ATTN_INT8QK_FP8PV = 1,
+  ATTN_MIXED_DIAG = 2,
+  ATTN_MXFP4QK_FP8PV = 3
+} attn_precision;
 
 typedef struct {
   int batch;       /* B >= 1 */
@@ -121,11 +135,20 @@ typedef struct {
   float beta_slow;
 } attn_rope_freq;
 
-/* Caller-owned device buffers of the quantised mode (all 16-byte aligned):
+/* Caller-owned device buffers of the quantised modes (all 16-byte aligned):
  *   q       int8   [B, Hq,  Sq,  D]          q_scale float [B, Hq,  ceil(Sq/128)]
  *   k       int8   [B, Hkv, Skv, D]          k_scale float [B, Hkv, ceil(Skv/128)]
  *   v_t     uint8  [B, Hkv, D, ceil(Skv/128)*128]  E4M3 codes of V, transposed,
- *                                            zero padded;  v_scale float [B, Hkv, D] */
+ *                                            zero padded;  v_scale float [B, Hkv, D]
+ * In the FP4 mode (ATTN_MXFP4QK_FP8PV) q and k hold packed E2M1 codes instead, two
+ * per byte (channel 2i in the low nibble): q [B, Hq, Sq, D/2], k [B, Hkv, Skv, D/2];
+ * q_scale and k_scale are unused (may be NULL); and q_sf, k_sf hold the E8M0 scale
+ * bytes in the tensor core's layout: one 512-byte chunk per 128-row tile, row r of
+ * the tile and channel block b (of 32) at byte (r % 32) * 16 + (r / 32) * 4 + b
+ * (b = 2, 3 unused).  Q's tiles run over the rows of a (batch, kv head) unit, its
+ * query heads stacked (G * Sq rows), rounded up to an even tile count:
+ * q_sf [B * Hkv][2 * ceil(G * Sq / 256)][512]; K's over each (batch, kv head)'s
+ * keys: k_sf [B * Hkv][ceil(Skv / 128)][512] (attn_qbufs_sf_sizes gives the sizes). */
 typedef struct {
   int8_t *q;
   int8_t *k;
@@ -133,6 +156,8 @@ typedef struct {
   float *k_scale;
   uint8_t *v_t;
   float *v_scale;
+  uint8_t *q_sf;  /* FP4 mode only (else ignored, may be NULL) */
+  uint8_t *k_sf;
 } attn_qbufs;
 
 typedef struct attn_ctx attn_ctx;
@@ -146,12 +171,16 @@ typedef struct attn_ctx attn_ctx;
  * (head_dim not 64/128), ATTN_ERR_CUDA (no device), ATTN_ERR_OOM. */
 attn_status attn_create(const attn_params *p, attn_ctx **out);
 
-/* Quantised and diagonal band modes, step 1 (the per-block quantiser): reads q, k, v (dtype of
+/* Quantised, diagonal band and FP4 modes, step 1 (the quantisers): reads q, k, v (dtype of
  * the context) and writes every buffer of *qb.  Q and K: per (b, h, 128-token
  * block) s = max|x| / 127 and code = clamp(round_half_even(x / s), +-127), s = 0
  * for an all-zero block.  V: per (b, hkv, channel) s = max|v| / 448 and code =
  * E4M3(v / s) rounded to nearest-even and saturated.  Each step is one
- * correctly rounded float32 operation, so the bytes are reproducible.  With
+ * correctly rounded float32 operation, so the bytes are reproducible.  FP4 mode,
+ * Q and K: per row and block of 32 channels, the E8M0 scale 2^e with
+ * e = floor(log2(max|x|)) - 2 (clamped to [-127, 127]; an all-zero block takes
+ * e = -127) and codes = E2M1(x / 2^e) rounded to nearest-even and saturated to +-6
+ * (the OCP MX conversion; x / 2^e is exact).  With
  * RoPE, Q and K (K unless rope_keys_rotated) are rotated in float32 first and
  * the codes are those of the rotated values.
  * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, context not in the
@@ -293,10 +322,15 @@ void attn_destroy(attn_ctx *c);
 /* Static string naming a status code. */
 const char *attn_status_string(attn_status s);
 
-/* Sizes, in bytes, of the caller-owned buffers of the quantised mode for `p`,
- * in the order of attn_qbufs (q, k, q_scale, k_scale, v_t, v_scale).  Pure
- * host arithmetic.  Errors: ATTN_ERR_INVALID_ARG. */
+/* Sizes, in bytes, of the caller-owned buffers of the quantised modes for `p`,
+ * in the order of attn_qbufs (q, k, q_scale, k_scale, v_t, v_scale); in the FP4
+ * mode q and k are the packed codes and the two scale sizes are 0.  Pure host
+ * arithmetic.  Errors: ATTN_ERR_INVALID_ARG. */
 attn_status attn_qbufs_sizes(const attn_params *p, size_t sizes[6]);
+
+/* FP4 mode: sizes in bytes of q_sf and k_sf for `p` (0 in the other modes).
+ * Pure host arithmetic.  Errors: ATTN_ERR_INVALID_ARG. */
+attn_status attn_qbufs_sf_sizes(const attn_params *p, size_t sizes[2]);
 
 /* Number of key/value splits the context uses (1 = the single-pass kernel). */
 int attn_num_splits(const attn_ctx *c);

@@ -46,12 +46,17 @@ def _params(**kw):
     (dict(window_size=-1), _abi.ATTN_ERR_INVALID_ARG),
     (dict(causal=2), _abi.ATTN_ERR_INVALID_ARG),
     (dict(dtype=7), _abi.ATTN_ERR_INVALID_ARG),
-    (dict(precision=3), _abi.ATTN_ERR_INVALID_ARG),
     (dict(scale=float("nan")), _abi.ATTN_ERR_INVALID_ARG),
     (dict(num_splits=-1), _abi.ATTN_ERR_INVALID_ARG),
     (dict(num_splits=100000), _abi.ATTN_ERR_INVALID_ARG),
     (dict(head_dim=96), _abi.ATTN_ERR_UNSUPPORTED),
     (dict(head_dim=256), _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(precision=4), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(precision=3, head_dim=128), _abi.ATTN_ERR_UNSUPPORTED),   # FP4: head_dim 64 only
+    (dict(precision=3, rope_dim=64), _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(precision=3, num_splits=2), _abi.ATTN_ERR_INVALID_ARG),    # single-pass modes
+    (dict(precision=2, num_splits=2), _abi.ATTN_ERR_INVALID_ARG),
+    (dict(precision=2, rope_dim=64), _abi.ATTN_ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_params_before_any_device_call(kw, status):
     L = afb.lib()
@@ -90,6 +95,17 @@ def test_qbufs_sizes():
     assert vt == 2 * 2 * 128 * 33 * 128 and vs == 2 * 2 * 128 * 4
     with pytest.raises(afb.AttnError):
         afb.attn_qbufs_sizes(_params(head_dim=80))
+    # FP4 mode: packed codes, no FP32 Q/K scales, E8M0 chunks per 128 rows (Q's rows
+    # stacked per unit and rounded to an even tile count)
+    p4 = _params(batch=2, n_q_heads=8, n_kv_heads=2, q_len=300, kv_len=4133, head_dim=64,
+                 precision=3)
+    q, k, qs, ks, vt, vs = afb.attn_qbufs_sizes(p4)
+    assert q == 2 * 8 * 300 * 32 and k == 2 * 2 * 4133 * 32 and qs == ks == 0
+    assert vt == 2 * 2 * 64 * 33 * 128 and vs == 2 * 2 * 64 * 4
+    from attention_forward_flash_b200 import _abi as abi
+    qsf, ksf = abi.attn_qbufs_sf_sizes(p4)
+    assert qsf == 4 * (2 * ((4 * 300 + 255) // 256)) * 512 and ksf == 4 * 33 * 512
+    assert abi.attn_qbufs_sf_sizes(_params()) == [0, 0]
 
 
 C_CALLER = r"""
@@ -113,6 +129,7 @@ int main(void) {
   attn_forward_paged(c, NULL, NULL, NULL, table, 1, NULL, NULL, NULL);
   attn_get_error(c, NULL);
   attn_qbufs_sizes(&p, sizes);
+  attn_qbufs_sf_sizes(&p, sizes);
   attn_num_splits(c);
   attn_debug_set(c, 0u);
   attn_debug_exp2(NULL, NULL, 0, NULL);
