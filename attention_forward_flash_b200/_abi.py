@@ -10,12 +10,13 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_OOM
 ATTN_BF16, ATTN_FP16 = 0, 1
 ATTN_EXACT, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG, ATTN_MXFP4QK_FP8PV = 0, 1, 2, 3
 ATTN_ROPE_PLAIN, ATTN_ROPE_NTK, ATTN_ROPE_YARN = 0, 1, 2
+ATTN_PATH_SINGLE_PASS, ATTN_PATH_SPLIT_MERGE, ATTN_PATH_DECODE = 1, 2, 3
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
             "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host",
             "attn_forward_paged", "attn_rope_table", "attn_set_rope_table", "attn_rope_apply",
-            "attn_qbufs_sf_sizes")
+            "attn_qbufs_sf_sizes", "attn_kernel_path")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -85,6 +86,8 @@ def lib():
         L.attn_qbufs_sf_sizes.restype = c_int
         L.attn_num_splits.argtypes = [vp]
         L.attn_num_splits.restype = c_int
+        L.attn_kernel_path.argtypes = [vp]
+        L.attn_kernel_path.restype = c_int
         L.attn_debug_set.argtypes = [vp, ctypes.c_uint]
         L.attn_debug_set.restype = c_int
         L.attn_debug_exp2.argtypes = [vp, vp, ctypes.c_size_t, vp]
@@ -152,6 +155,10 @@ def attn_qbufs_sf_sizes(params: AttnParams):
 
 def attn_num_splits(ctx):
     return lib().attn_num_splits(ctx)
+
+
+def attn_kernel_path(ctx):
+    return lib().attn_kernel_path(ctx)
 
 
 def attn_debug_set(ctx, flags):

@@ -136,6 +136,12 @@ class Attention:
     def num_splits(self):
         return _abi.attn_num_splits(self.ctx)
 
+    @property
+    def kernel_path(self):
+        """``"single_pass"``, ``"split_merge"`` or ``"decode"`` (``attn_kernel_path``)."""
+        return {_abi.ATTN_PATH_SINGLE_PASS: "single_pass", _abi.ATTN_PATH_SPLIT_MERGE:
+                "split_merge", _abi.ATTN_PATH_DECODE: "decode"}[_abi.attn_kernel_path(self.ctx)]
+
     def _check_inputs(self, q, k, v, on_cuda=True):
         p = self.params
         want_q = (p.batch, p.n_q_heads, p.q_len, p.head_dim)

@@ -13,8 +13,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB = os.path.join(HERE, "libattn.so")
 SOURCES = [os.path.join(HERE, "csrc", "attn_api.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "flash_fwd.cuh", "quant.cuh",
-                                                          "merge.cuh", "device_once.h")] + [
+DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in (
+    "ptx.cuh", "flash_fwd.cuh", "quant.cuh", "merge.cuh", "rope.cuh", "decode.cuh",
+    "device_once.h")] + [
     os.path.join(os.path.dirname(HERE), "include", "attn.h")]
 
 

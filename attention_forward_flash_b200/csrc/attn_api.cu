@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "decode.cuh"
 #include "device_once.h"
 #include "flash_fwd.cuh"
 #include "merge.cuh"
@@ -45,6 +46,9 @@ struct attn_ctx {
   int R;           // stacked rows per unit
   int units;       // batch * n_kv_heads
   int split_path;  // 1: single-query-tile kernel + merge; 0: two-query-tile kernel
+  int decode;      // 1: flash_decode_kernel (one cluster of `splits` CTAs per unit)
+  int dec_chunk0;  // decode kernel: first key chunk of the rows' visible union
+  int dec_nchunks; //   and its number of chunks
   int splits;
   int tiles_per_split;
   int row_tiles;
@@ -113,14 +117,14 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 }
 
 // 4-D tiled map of a paged key/value pool [blocks][kv heads][128 positions][D]:
-// dims (D, 128, kv heads, blocks), box (64 channels, 128 positions, 1, 1).
+// dims (D, 128, kv heads, blocks), box (64 channels, `rows` positions, 1, 1).
 bool make_pool_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t D,
-                   uint64_t hkv, uint64_t blocks) {
+                   uint64_t hkv, uint64_t blocks, uint32_t rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {D, 128, hkv, blocks};
   cuuint64_t strides[3] = {D * 2, 128 * D * 2, hkv * 128 * D * 2};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -141,6 +145,107 @@ bool set_smem(int bytes) {
     return cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
            cudaSuccess;
   });
+}
+
+// The decode kernel's attributes, once per device: its dynamic shared memory, and
+// clusters of up to 16 CTAs (above the portable 8).
+template <auto Kern>
+bool set_decode_attrs(int bytes) {
+  static PerDeviceOnce<> once;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  return once.ensure(dev, [&] {
+    return cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(Kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+               cudaSuccess;
+  });
+}
+
+// Launch configuration of the decode kernel: `units` clusters of `splits` CTAs.
+template <int D>
+cudaLaunchConfig_t decode_config(int units, int splits, cudaStream_t st,
+                                 cudaLaunchAttribute* at) {
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = static_cast<unsigned>(splits);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * splits));
+  cfg.blockDim = dim3(DecCfg<D>::kThreads);
+  cfg.dynamicSmemBytes = DecCfg<D>::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Clusters of `splits` decode CTAs that the current device holds at once (0 if none
+// or on error).
+template <int D>
+int decode_max_clusters(int units, int splits) {
+  constexpr auto kern = flash_decode_kernel<D, false, false, false>;
+  if (!set_decode_attrs<kern>(DecCfg<D>::kSmemBytes)) return 0;
+  cudaLaunchAttribute at[1];
+  const cudaLaunchConfig_t cfg = decode_config<D>(units, splits, nullptr, at);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int D, bool F16, bool PAGED, bool ROPE>
+attn_status launch_decode(const attn_ctx* c, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const DecArgs& a, int nu, cudaStream_t st) {
+  constexpr auto kern = flash_decode_kernel<D, F16, PAGED, ROPE>;
+  if (!set_decode_attrs<kern>(DecCfg<D>::kSmemBytes)) return ATTN_ERR_CUDA;
+  cudaLaunchAttribute at[1];
+  const cudaLaunchConfig_t cfg = decode_config<D>(nu, c->splits, st, at);
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, a) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool PAGED>
+attn_status dispatch_decode(const attn_ctx* c, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const DecArgs& a, int nu, cudaStream_t st) {
+  const bool rope = a.rope_table != nullptr;
+  if (c->p.dtype == ATTN_FP16)
+    return rope ? launch_decode<D, true, PAGED, true>(c, mk, mv, a, nu, st)
+                : launch_decode<D, true, PAGED, false>(c, mk, mv, a, nu, st);
+  return rope ? launch_decode<D, false, PAGED, true>(c, mk, mv, a, nu, st)
+              : launch_decode<D, false, PAGED, false>(c, mk, mv, a, nu, st);
+}
+
+// Decode-kernel arguments for the units whose Q, O and lse start at q, o, lse.
+DecArgs decode_args(const attn_ctx* c, const void* q, void* o, float* lse) {
+  const attn_params& p = c->p;
+  DecArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.o = static_cast<uint16_t*>(o);
+  a.lse = lse;
+  a.R = c->R;
+  a.Sq = p.q_len;
+  a.Skv = p.kv_len;
+  a.start_pos = p.start_pos;
+  a.causal = p.causal;
+  a.window_lo = p.window_lo;
+  a.window_size = p.window_size;
+  a.chunk0 = c->dec_chunk0;
+  a.n_chunks = c->dec_nchunks;
+  a.scale_log2 = c->scale * 1.4426950408889634f;
+  if (p.rope_dim > 0) {
+    a.rope_table = c->rope_table;
+    a.rope_R = p.rope_dim;
+    a.rope_inter = p.rope_interleaved;
+  }
+  a.err = c->err;
+  a.debug = c->debug;
+  return a;
+}
+
+inline uint32_t decode_chunk(int head_dim) {
+  return head_dim == 128 ? DecCfg<128>::kChunk : DecCfg<64>::kChunk;
 }
 
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
@@ -517,6 +622,25 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
       f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t R = c->R, Sk = p.kv_len, U = nu;
   MapCache& mc = c->maps[slot];
+  if (c->decode) {  // K and V in boxes of one key chunk; Q and O by plain loads and stores
+    const void* key[6] = {k, v, nullptr, nullptr, nullptr, nullptr};
+    bool hit = mc.valid && mc.nu == nu;
+    for (int i = 0; i < 6; ++i) hit = hit && mc.key[i] == key[i];
+    if (!hit) {
+      const uint32_t rows = decode_chunk(D);
+      bool ok = make_map(&mc.m.k, t16, k, D, Sk, U, D * 2, Sk * D * 2, 64, rows,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+      ok &= make_map(&mc.m.v, t16, v, D, Sk, U, D * 2, Sk * D * 2, 64, rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+      mc.valid = ok;
+      mc.nu = nu;
+      for (int i = 0; i < 6; ++i) mc.key[i] = key[i];
+      if (!ok) return ATTN_ERR_CUDA;
+    }
+    const DecArgs a = decode_args(c, q, o, lse);
+    return D == 128 ? dispatch_decode<128, false>(c, mc.m.k, mc.m.v, a, nu, st)
+                    : dispatch_decode<64, false>(c, mc.m.k, mc.m.v, a, nu, st);
+  }
   const void* key[6] = {quant ? static_cast<const void*>(qb->q) : q,
                         quant ? static_cast<const void*>(qb->k) : k,
                         quant ? static_cast<const void*>(qb->v_t) : v, o,
@@ -677,6 +801,15 @@ size_t d2h_piece_bytes(size_t out_per_unit, size_t in_per_unit) {
 
 // Marks the end of a call's work on `st` (everything it enqueued, errors included).
 attn_status mark_done(attn_ctx* c, attn_status s, cudaStream_t st) {
+  // A call captured into a CUDA graph runs when the graph is launched: the event
+  // cannot mark it (an event last recorded during capture cannot be waited for
+  // outside the graph), so it keeps marking the context's last direct call.
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return s == ATTN_OK ? ATTN_ERR_CUDA : s;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return s;
   if (cudaEventRecord(c->done_ev, st) != cudaSuccess && s == ATTN_OK) return ATTN_ERR_CUDA;
   return s;
 }
@@ -765,6 +898,35 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   int splits = 1;
   if (p->precision == ATTN_MIXED_DIAG || p->precision == ATTN_MXFP4QK_FP8PV) {
     // single-pass kernel only (the band and FP4 modes have no split-KV variant)
+  } else if (p->precision == ATTN_EXACT && c->R <= 16 && p->kv_len > 0 &&
+             (p->num_splits == 0 ||
+              (p->num_splits > 1 && p->num_splits <= DecCfg<128>::kMaxSplits))) {
+    // Decode-shaped (at most 16 stacked rows per unit): the cluster kernel.  The
+    // union of the rows' visible key ranges: row 0 has the lowest lower bound,
+    // the last position the highest upper bound.
+    const int chunk = static_cast<int>(decode_chunk(p->head_dim));
+    long long lo = std::max(p->window_lo, 0);
+    if (p->window_size > 0)
+      lo = std::max<long long>(lo, static_cast<long long>(p->start_pos) - p->window_size + 1);
+    long long hi = p->kv_len - 1;
+    if (p->causal)
+      hi = std::min<long long>(hi, static_cast<long long>(p->start_pos) + p->q_len - 1);
+    c->decode = 1;
+    c->dec_chunk0 = lo <= hi ? static_cast<int>(lo / chunk) : 0;
+    c->dec_nchunks = lo <= hi ? static_cast<int>(hi / chunk - lo / chunk + 1) : 0;
+    // about one CTA per SM over all units (at most 16 per cluster, at most one chunk
+    // each), then as large a cluster as lets every unit's cluster (or as many as
+    // the SMs hold) be resident at once
+    int S = p->num_splits > 1 ? p->num_splits
+                              : std::max(1, std::min(DecCfg<128>::kMaxSplits, sms / c->units));
+    S = std::max(1, std::min(S, std::max(c->dec_nchunks, 1)));
+    while (S > 1) {
+      const int n = p->head_dim == 128 ? decode_max_clusters<128>(c->units, S)
+                                       : decode_max_clusters<64>(c->units, S);
+      if (n >= std::min(c->units, std::max(1, sms / S))) break;
+      --S;
+    }
+    splits = S;
   } else if (p->num_splits > 1) {
     split = true;
     splits = p->num_splits;
@@ -775,11 +937,13 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
       splits = std::max(1, std::min(kv_tiles, ceil_div(2 * sms, base)));  // two CTAs per SM
     }
   }
-  splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
-  splits = std::min(splits, kMergeMaxSplits);
+  if (!c->decode) {
+    splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
+    splits = std::min(splits, kMergeMaxSplits);
+  }
   c->split_path = split ? 1 : 0;
   c->tiles_per_split = std::max(1, ceil_div(kv_tiles, splits));
-  c->splits = split ? std::max(1, ceil_div(kv_tiles, c->tiles_per_split)) : 1;
+  c->splits = split ? std::max(1, ceil_div(kv_tiles, c->tiles_per_split)) : (c->decode ? splits : 1);
   c->row_tiles = ceil_div(c->R, split ? 128 : 256);
 
   // workspace: error word | V channel maxima | split partials
@@ -856,9 +1020,18 @@ void attn_destroy(attn_ctx* c) {
     cudaEventDestroy(c->pev_start);
   }
   delete c;
+  cudaGetLastError();  // these calls report nothing: leave no error for the next launch check
 }
 
-int attn_num_splits(const attn_ctx* c) { return c ? (c->split_path ? c->splits : 1) : 0; }
+int attn_num_splits(const attn_ctx* c) {
+  return c ? ((c->split_path || c->decode) ? c->splits : 1) : 0;
+}
+
+int attn_kernel_path(const attn_ctx* c) {
+  if (!c) return 0;
+  return c->decode ? ATTN_PATH_DECODE : (c->split_path ? ATTN_PATH_SPLIT_MERGE
+                                                       : ATTN_PATH_SINGLE_PASS);
+}
 
 attn_status attn_debug_set(attn_ctx* c, unsigned flags) {
   if (!c) return ATTN_ERR_INVALID_ARG;
@@ -932,6 +1105,19 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
   }
   const CUtensorMapDataType t16 =
       f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (c->decode) {
+    CUtensorMap mk, mv;
+    const uint32_t crow = decode_chunk(D);
+    bool ok = make_pool_map(&mk, t16, k_pool, D, p.n_kv_heads, num_blocks, crow);
+    ok &= make_pool_map(&mv, t16, v_pool, D, p.n_kv_heads, num_blocks, crow);
+    if (!ok) return ATTN_ERR_CUDA;
+    DecArgs a = decode_args(c, q, o, lse);
+    a.block_table = block_table;
+    a.bt_stride = ceil_div(p.kv_len, 128);
+    a.n_kv_heads = p.n_kv_heads;
+    return D == 128 ? dispatch_decode<128, true>(c, mk, mv, a, c->units, st)
+                    : dispatch_decode<64, true>(c, mk, mv, a, c->units, st);
+  }
   const uint64_t R = c->R, U = c->units;
   FwdMaps m;
   bool ok = make_map(&m.q, t16, q, D, R, U, D * 2, R * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);

@@ -87,8 +87,6 @@ struct FwdArgs {
   int q_tiles;
 };
 
-constexpr int kErrTimeout = 1;
-
 // DIAG (quantised mode only): the key tiles of the causal diagonal band get
 // Q K^T from the 16-bit inputs; 16-bit Q tiles sit next to the INT8 ones and one
 // 16-bit K tile buffer serves the band tiles (the ring carries the rest).

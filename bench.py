@@ -186,7 +186,7 @@ def make_attention(w: Workload, precision):
 
 
 def launches_per_step(att, precision):
-    n = 1 + (1 if att.num_splits > 1 else 0)
+    n = 1 + (1 if att.kernel_path == "split_merge" else 0)  # the merge kernel
     if precision != "exact":
         n += 4  # Q and K block quantisers, V channel maxima, V quantiser
     elif att.params.rope_dim > 0 and not att.params.rope_keys_rotated:

@@ -316,7 +316,9 @@ attn_status attn_get_error(attn_ctx *c, void *stream);
  * stream, and the streams of attn_forward_host's pipeline), then frees the
  * workspace.  Work of other contexts or libraries on the device is not waited
  * for by this call (the CUDA runtime's cudaFree may still synchronise the
- * device).  NULL is ignored. */
+ * device).  Calls captured into a CUDA graph are not waited for: destroy the
+ * context only after every launch of such a graph has finished (the graph
+ * refers to the workspace).  NULL is ignored. */
 void attn_destroy(attn_ctx *c);
 
 /* Static string naming a status code. */
@@ -332,11 +334,35 @@ attn_status attn_qbufs_sizes(const attn_params *p, size_t sizes[6]);
  * Pure host arithmetic.  Errors: ATTN_ERR_INVALID_ARG. */
 attn_status attn_qbufs_sf_sizes(const attn_params *p, size_t sizes[2]);
 
-/* Number of key/value splits the context uses (1 = the single-pass kernel). */
+/* Number of key/value splits the context uses (1 = no split), 0 for NULL. */
 int attn_num_splits(const attn_ctx *c);
 
+/* The kernel a context runs, fixed by attn_create:
+ *   ATTN_PATH_SINGLE_PASS  the tensor-core kernel, 256 query rows per CTA, every key;
+ *   ATTN_PATH_SPLIT_MERGE  one 128-row query tile per CTA, the keys split across
+ *                          CTAs, then a merge kernel (few rows per kv head, or too few
+ *                          CTAs to fill the GPU);
+ *   ATTN_PATH_DECODE       exact mode with at most 16 stacked rows per unit
+ *                          (Hq/Hkv * q_len <= 16, e.g. decode steps) and num_splits
+ *                          0 or 2..16: one thread-block cluster of num_splits CTAs per
+ *                          (batch, kv head); each CTA streams an equal run of the
+ *                          rows' visible keys, and the CTAs merge their partial
+ *                          results through distributed shared memory in the same
+ *                          launch.  The split key range is the union of the rows'
+ *                          visible ranges; the merge is the qsa2 audit's ("round 21
+ *                          track b -- qsa2", "implementation and review": cached
+ *                          per-split maxima and weights, one denominator).
+ * Returns 0 for NULL. */
+typedef enum {
+  ATTN_PATH_SINGLE_PASS = 1,
+  ATTN_PATH_SPLIT_MERGE = 2,
+  ATTN_PATH_DECODE = 3
+} attn_kernel_path_kind;
+int attn_kernel_path(const attn_ctx *c);
+
 /* TEST HOOK.  Bit 0 of `flags` makes the next attn_forward's loader skip the
- * second key tile of every CTA, so that the waits on it run out: the kernel then
+ * second key tile of every CTA (ATTN_PATH_DECODE: the second key chunk of the
+ * first warp of the first CTA), so that the waits on it run out: the kernel then
  * records ATTN_ERR_TIMEOUT in the context and returns without hanging.  Bit 1
  * does the same to attn_quantize_qk: the first CTA of the Q quantiser never
  * loads its second block.  The hook exists only to test that error path; 0

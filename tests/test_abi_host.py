@@ -78,6 +78,7 @@ def test_null_arguments():
     assert L.attn_get_error(None, None) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_debug_set(None, 0) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_num_splits(None) == 0
+    assert L.attn_kernel_path(None) == 0
     L.attn_destroy(None)
 
 
@@ -131,6 +132,7 @@ int main(void) {
   attn_qbufs_sizes(&p, sizes);
   attn_qbufs_sf_sizes(&p, sizes);
   attn_num_splits(c);
+  if (attn_kernel_path(c) == ATTN_PATH_DECODE) return 2;
   attn_debug_set(c, 0u);
   attn_debug_exp2(NULL, NULL, 0, NULL);
   attn_forward_splitkv_noalloc(&p, NULL, NULL, NULL, NULL, NULL, &err, NULL);

@@ -396,14 +396,17 @@ def _ramp_inputs(D, Sq, Skv, G, seed):
 
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [7.5, 8.5, 20.0])
-@pytest.mark.parametrize("split", [False, True])
-def test_exact_rescale_forced(D, G, split):
-    Sq = 8 if split else 300          # few rows take the split-KV kernel
+@pytest.mark.parametrize("path", ["single_pass", "split_merge", "decode"])
+def test_exact_rescale_forced(D, G, path):
+    # 300 rows: the single-pass kernel; 40 rows with 3 forced splits: the split-KV
+    # kernel and its merge; 8 rows: the decode kernel (its own online softmax
+    # rescales on every chunk whose maximum grows)
+    Sq, splits = {"single_pass": (300, 1), "split_merge": (40, 3), "decode": (8, 3)}[path]
     Skv = 10 * 128 + 37
     q, k, v = _ramp_inputs(D, Sq, Skv, G, seed=int(7000 + 10 * G + D))
     w = Workload("ramp", 1, 2, 2, Sq, Skv, D, "bf16", seed=0)
-    o, lse, att = run_gpu(w, q, k, v, num_splits=3 if split else 1)
-    assert (att.num_splits == 3) == split
+    o, lse, att = run_gpu(w, q, k, v, num_splits=splits)
+    assert att.kernel_path == path and att.num_splits == splits
     ro, rl = oracle_for(w, q, k, v)
     check_exact(o, ro, f"G={G}")
     check_lse(lse, rl, f"G={G}")
