@@ -10,7 +10,8 @@ ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_OOM
 ATTN_BF16, ATTN_FP16 = 0, 1
 ATTN_EXACT, ATTN_INT8QK_FP8PV, ATTN_MIXED_DIAG, ATTN_MXFP4QK_FP8PV = 0, 1, 2, 3
 ATTN_ROPE_PLAIN, ATTN_ROPE_NTK, ATTN_ROPE_YARN = 0, 1, 2
-ATTN_PATH_SINGLE_PASS, ATTN_PATH_SPLIT_MERGE, ATTN_PATH_DECODE = 1, 2, 3
+ATTN_PATH_SINGLE_PASS, ATTN_PATH_SPLIT_MERGE, ATTN_PATH_DECODE, ATTN_PATH_SINGLE_PASS_TAIL = \
+    1, 2, 3, 4
 
 EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error", "attn_destroy",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",

@@ -138,9 +138,12 @@ class Attention:
 
     @property
     def kernel_path(self):
-        """``"single_pass"``, ``"split_merge"`` or ``"decode"`` (``attn_kernel_path``)."""
+        """``"single_pass"``, ``"single_pass_tail"``, ``"split_merge"`` or ``"decode"``
+        (``attn_kernel_path``)."""
         return {_abi.ATTN_PATH_SINGLE_PASS: "single_pass", _abi.ATTN_PATH_SPLIT_MERGE:
-                "split_merge", _abi.ATTN_PATH_DECODE: "decode"}[_abi.attn_kernel_path(self.ctx)]
+                "split_merge", _abi.ATTN_PATH_DECODE: "decode",
+                _abi.ATTN_PATH_SINGLE_PASS_TAIL: "single_pass_tail"}[
+                    _abi.attn_kernel_path(self.ctx)]
 
     def _check_inputs(self, q, k, v, on_cuda=True):
         p = self.params

@@ -49,6 +49,15 @@ struct attn_ctx {
   int decode;      // 1: flash_decode_kernel (one cluster of `splits` CTAs per unit)
   int dec_chunk0;  // decode kernel: first key chunk of the rows' visible union
   int dec_nchunks; //   and its number of chunks
+  int dec_nsw;     //   ring slots per warp
+  int dec_owner_slots;  // partial-row slots of its merge area
+  int dec_smem;    //   dynamic shared memory per CTA
+  // Single-pass kernel whose grid ends in a short last wave: its last tail_items
+  // CTAs run as the split kernel with tail_k key splits (partials in the workspace).
+  int tail_items;
+  int tail_k;
+  float* tail_opart;
+  float* tail_lse;
   int splits;
   int tiles_per_split;
   int row_tiles;
@@ -164,7 +173,7 @@ bool set_decode_attrs(int bytes) {
 
 // Launch configuration of the decode kernel: `units` clusters of `splits` CTAs.
 template <int D>
-cudaLaunchConfig_t decode_config(int units, int splits, cudaStream_t st,
+cudaLaunchConfig_t decode_config(int units, int splits, int smem, cudaStream_t st,
                                  cudaLaunchAttribute* at) {
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = static_cast<unsigned>(splits);
@@ -173,7 +182,7 @@ cudaLaunchConfig_t decode_config(int units, int splits, cudaStream_t st,
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(units * splits));
   cfg.blockDim = dim3(DecCfg<D>::kThreads);
-  cfg.dynamicSmemBytes = DecCfg<D>::kSmemBytes;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
@@ -184,10 +193,11 @@ cudaLaunchConfig_t decode_config(int units, int splits, cudaStream_t st,
 // or on error).
 template <int D>
 int decode_max_clusters(int units, int splits) {
-  constexpr auto kern = flash_decode_kernel<D, false, false, false>;
-  if (!set_decode_attrs<kern>(DecCfg<D>::kSmemBytes)) return 0;
+  constexpr auto kern = flash_decode_kernel<D, false, false, false, false>;
+  if (!set_decode_attrs<kern>(DecCfg<D>::kMaxSmem)) return 0;
   cudaLaunchAttribute at[1];
-  const cudaLaunchConfig_t cfg = decode_config<D>(units, splits, nullptr, at);
+  // every launch takes more than half an SM's shared memory: one CTA per SM
+  const cudaLaunchConfig_t cfg = decode_config<D>(units, splits, DecCfg<D>::kMaxSmem, nullptr, at);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -196,25 +206,33 @@ int decode_max_clusters(int units, int splits) {
   return n;
 }
 
-template <int D, bool F16, bool PAGED, bool ROPE>
+template <int D, bool F16, bool PAGED, bool ROPE, bool TR>
 attn_status launch_decode(const attn_ctx* c, const CUtensorMap& mk, const CUtensorMap& mv,
                           const DecArgs& a, int nu, cudaStream_t st) {
-  constexpr auto kern = flash_decode_kernel<D, F16, PAGED, ROPE>;
-  if (!set_decode_attrs<kern>(DecCfg<D>::kSmemBytes)) return ATTN_ERR_CUDA;
+  constexpr auto kern = flash_decode_kernel<D, F16, PAGED, ROPE, TR>;
+  if (!set_decode_attrs<kern>(DecCfg<D>::kMaxSmem)) return ATTN_ERR_CUDA;
   cudaLaunchAttribute at[1];
-  const cudaLaunchConfig_t cfg = decode_config<D>(nu, c->splits, st, at);
+  const cudaLaunchConfig_t cfg = decode_config<D>(nu, c->splits, c->dec_smem, st, at);
   return cudaLaunchKernelEx(&cfg, kern, mk, mv, a) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+template <int D, bool PAGED, bool TR>
+attn_status dispatch_decode_t(const attn_ctx* c, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const DecArgs& a, int nu, cudaStream_t st) {
+  const bool rope = a.rope_table != nullptr;
+  if (c->p.dtype == ATTN_FP16)
+    return rope ? launch_decode<D, true, PAGED, true, TR>(c, mk, mv, a, nu, st)
+                : launch_decode<D, true, PAGED, false, TR>(c, mk, mv, a, nu, st);
+  return rope ? launch_decode<D, false, PAGED, true, TR>(c, mk, mv, a, nu, st)
+              : launch_decode<D, false, PAGED, false, TR>(c, mk, mv, a, nu, st);
+}
+
+// At most 8 rows per unit: the transposed products (no padding rows in the MMAs).
 template <int D, bool PAGED>
 attn_status dispatch_decode(const attn_ctx* c, const CUtensorMap& mk, const CUtensorMap& mv,
                             const DecArgs& a, int nu, cudaStream_t st) {
-  const bool rope = a.rope_table != nullptr;
-  if (c->p.dtype == ATTN_FP16)
-    return rope ? launch_decode<D, true, PAGED, true>(c, mk, mv, a, nu, st)
-                : launch_decode<D, true, PAGED, false>(c, mk, mv, a, nu, st);
-  return rope ? launch_decode<D, false, PAGED, true>(c, mk, mv, a, nu, st)
-              : launch_decode<D, false, PAGED, false>(c, mk, mv, a, nu, st);
+  return c->R <= 8 ? dispatch_decode_t<D, PAGED, true>(c, mk, mv, a, nu, st)
+                   : dispatch_decode_t<D, PAGED, false>(c, mk, mv, a, nu, st);
 }
 
 // Decode-kernel arguments for the units whose Q, O and lse start at q, o, lse.
@@ -241,6 +259,8 @@ DecArgs decode_args(const attn_ctx* c, const void* q, void* o, float* lse) {
   }
   a.err = c->err;
   a.debug = c->debug;
+  a.nsw = c->dec_nsw;
+  a.owner_slots = c->dec_owner_slots;
   return a;
 }
 
@@ -261,7 +281,7 @@ attn_status launch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, in
 
 template <int D, bool QUANT, bool F16, bool WIN, bool ROPE>
 attn_status dispatch_win(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool split) {
   // the diagonal band mode: single-pass quantised kernel with 16-bit band tiles
   if constexpr (QUANT) {
     if (c->p.precision == ATTN_MIXED_DIAG)
@@ -273,8 +293,7 @@ attn_status dispatch_win(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, 
       return launch_fwd<D, 2, true, F16, false, false, WIN, false, false, true>(c, m, a, grid,
                                                                                 st);
   }
-  if (c->split_path)
-    return launch_fwd<D, 1, QUANT, F16, true, true, WIN, ROPE>(c, m, a, grid, st);
+  if (split) return launch_fwd<D, 1, QUANT, F16, true, true, WIN, ROPE>(c, m, a, grid, st);
   // Exact mode keeps a second (float32) row sum only when the caller asks for lse
   // (the quantised mode's only sum is the float32 one).
   if constexpr (!QUANT) {
@@ -286,30 +305,30 @@ attn_status dispatch_win(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, 
 
 template <int D, bool QUANT, bool F16, bool ROPE>
 attn_status dispatch_rope(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool split) {
   if (a.window_size > 0)
-    return dispatch_win<D, QUANT, F16, true, ROPE>(c, m, a, grid, st);
-  return dispatch_win<D, QUANT, F16, false, ROPE>(c, m, a, grid, st);
+    return dispatch_win<D, QUANT, F16, true, ROPE>(c, m, a, grid, st, split);
+  return dispatch_win<D, QUANT, F16, false, ROPE>(c, m, a, grid, st, split);
 }
 
 // Exact mode with RoPE: the variant that rotates the staged Q tile (the keys
 // arrive rotated); the quantised mode rotates in its quantiser.
 template <int D, bool QUANT, bool F16>
 attn_status dispatch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool split) {
   if constexpr (!QUANT) {
     if (a.rope_table != nullptr)
-      return dispatch_rope<D, QUANT, F16, true>(c, m, a, grid, st);
+      return dispatch_rope<D, QUANT, F16, true>(c, m, a, grid, st, split);
   }
-  return dispatch_rope<D, QUANT, F16, false>(c, m, a, grid, st);
+  return dispatch_rope<D, QUANT, F16, false>(c, m, a, grid, st, split);
 }
 
 // The merge is a programmatic dependent launch of the split kernel: its launch
 // overlaps the split kernel's tail, and it waits on the grid dependency before
 // reading the partials.
 template <int D, bool F16>
-attn_status launch_merge(const attn_ctx* c, void* o, float* lse, cudaStream_t st) {
-  const int rows = c->units * c->R;
+attn_status launch_merge_rows(const float* op, const float* lp, uint16_t* out, float* lse,
+                              int rows, int stride, int splits, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows);
   cfg.blockDim = dim3(32 * kMergeWarps);
@@ -320,14 +339,17 @@ attn_status launch_merge(const attn_ctx* c, void* o, float* lse, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const float* op = c->o_part;
-  const float* lp = c->lse_part;
-  uint16_t* out = static_cast<uint16_t*>(o);
-  const int splits = c->splits;
-  if (cudaLaunchKernelEx(&cfg, splitkv_merge_kernel<D, F16>, op, lp, out, lse, rows, splits) !=
+  if (cudaLaunchKernelEx(&cfg, splitkv_merge_kernel<D, F16>, op, lp, out, lse, stride, splits) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool F16>
+attn_status launch_merge(const attn_ctx* c, void* o, float* lse, cudaStream_t st) {
+  const int rows = c->units * c->R;
+  return launch_merge_rows<D, F16>(c->o_part, c->lse_part, static_cast<uint16_t*>(o), lse, rows,
+                                   rows, c->splits, st);
 }
 
 attn_status validate(const attn_params* p) {
@@ -701,6 +723,7 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
   a.lse = lse;
   a.o_part = c->o_part;
   a.lse_part = c->lse_part;
+  a.part_rows = c->units * c->R;  // split path: every row
   if (quant) {
     a.q_scale = qb->q_scale;
     a.k_scale = qb->k_scale;
@@ -721,26 +744,69 @@ attn_status forward_units(attn_ctx* c, int u0, int nu, const void* q, const void
     a.q_tiles = fp4_q_tiles(p);
   }
   a.tph = causal_band_tiles(c);
-  const int grid = nu * c->row_tiles * (c->split_path ? c->splits : 1);
 
-  attn_status s;
-  if (D == 128) {
-    if (quant) s = f16 ? dispatch_fwd<128, true, true>(c, m, a, grid, st)
-                       : dispatch_fwd<128, true, false>(c, m, a, grid, st);
-    else s = f16 ? dispatch_fwd<128, false, true>(c, m, a, grid, st)
-                 : dispatch_fwd<128, false, false>(c, m, a, grid, st);
-  } else {
-    if (quant) s = f16 ? dispatch_fwd<64, true, true>(c, m, a, grid, st)
-                       : dispatch_fwd<64, true, false>(c, m, a, grid, st);
-    else s = f16 ? dispatch_fwd<64, false, true>(c, m, a, grid, st)
-                 : dispatch_fwd<64, false, false>(c, m, a, grid, st);
-  }
-  if (s != ATTN_OK) return s;
+  auto run = [&](const FwdArgs& fa, int grid, bool split) -> attn_status {
+    if (D == 128) {
+      if (quant) return f16 ? dispatch_fwd<128, true, true>(c, m, fa, grid, st, split)
+                            : dispatch_fwd<128, true, false>(c, m, fa, grid, st, split);
+      return f16 ? dispatch_fwd<128, false, true>(c, m, fa, grid, st, split)
+                 : dispatch_fwd<128, false, false>(c, m, fa, grid, st, split);
+    }
+    if (quant) return f16 ? dispatch_fwd<64, true, true>(c, m, fa, grid, st, split)
+                          : dispatch_fwd<64, true, false>(c, m, fa, grid, st, split);
+    return f16 ? dispatch_fwd<64, false, true>(c, m, fa, grid, st, split)
+               : dispatch_fwd<64, false, false>(c, m, fa, grid, st, split);
+  };
+  // merge of the partials of rows row0 .. row0 + rows - 1 (of this call's units);
+  // split sp of a row is at sp * stride in the partial buffers op, lp
+  auto merge = [&](const float* op, const float* lp, size_t row0, int rows, int stride,
+                   int splits) -> attn_status {
+    uint16_t* out = static_cast<uint16_t*>(o) + row0 * D;
+    float* l = lse ? lse + row0 : nullptr;
+    if (D == 128)
+      return f16 ? launch_merge_rows<128, true>(op, lp, out, l, rows, stride, splits, st)
+                 : launch_merge_rows<128, false>(op, lp, out, l, rows, stride, splits, st);
+    return f16 ? launch_merge_rows<64, true>(op, lp, out, l, rows, stride, splits, st)
+               : launch_merge_rows<64, false>(op, lp, out, l, rows, stride, splits, st);
+  };
   if (c->split_path) {
-    if (D == 128) s = f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
-    else s = f16 ? launch_merge<64, true>(c, o, lse, st) : launch_merge<64, false>(c, o, lse, st);
+    const attn_status s = run(a, nu * c->row_tiles * c->splits, true);
+    if (s != ATTN_OK) return s;
+    const int rows = c->units * c->R;
+    return merge(c->o_part, c->lse_part, 0, rows, rows, c->splits);
   }
-  return s;
+  const int nctas = nu * c->row_tiles;
+  if (c->tail_items > 0) {
+    // Short last wave: the last tail_items CTAs of the whole problem's single-pass
+    // grid (256 rows each) run instead as the split kernel over their 128-row tiles
+    // with tail_k key splits, and a merge of those rows; the others fill whole
+    // waves.  A range of units takes the same split for the same rows, so every
+    // row is computed the same way whatever the range (partials by global row).
+    const int main_g = c->units * c->row_tiles - c->tail_items;  // first tail CTA
+    const int first = u0 * c->row_tiles;                          // this range's first
+    const int n_main = std::max(0, std::min(nctas, main_g - first));
+    const int n_tail = nctas - n_main;
+    attn_status s = ATTN_OK;
+    if (n_main > 0) s = run(a, n_main, false);
+    if (s != ATTN_OK || n_tail == 0) return s;
+    const int pstride = c->tail_items * 256;                   // partial rows (whole tail)
+    FwdArgs at = a;
+    at.row_tiles = c->R / 128;
+    at.splits = c->tail_k;
+    at.tiles_per_split = ceil_div(ceil_div(p.kv_len, 128), c->tail_k);
+    at.tile0 = 2 * n_main;
+    at.part_row0 = main_g * 256 - u0 * c->R;                   // range-local row of partial 0
+    at.part_rows = pstride;
+    at.o_part = c->tail_opart;
+    at.lse_part = c->tail_lse;
+    at.tph = 0;
+    s = run(at, 2 * n_tail * c->tail_k, true);
+    if (s != ATTN_OK) return s;
+    const size_t p0 = static_cast<size_t>(first + n_main - main_g) * 256;  // first partial row
+    return merge(c->tail_opart + p0 * D, c->tail_lse + p0, static_cast<size_t>(n_main) * 256,
+                 n_tail * 256, pstride, c->tail_k);
+  }
+  return run(a, nctas, false);
 }
 
 // Creates attn_forward_host's streams and events on the current device (all or none).
@@ -927,6 +993,16 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
       --S;
     }
     splits = S;
+    // the merge area for this S, and two ring slots per warp: the K/V stream is
+    // bound by the bytes the whole GPU has in flight, and a third slot per warp
+    // measured slower (decode workload: 9.3 against 8.2 us per call back to back)
+    const int rpo = (c->R + S - 1) / S;
+    const bool d128 = p->head_dim == 128;
+    c->dec_owner_slots = DecCfg<128>::kWarps * S * rpo;
+    const int nsw = 2;
+    c->dec_nsw = nsw;
+    c->dec_smem = d128 ? DecCfg<128>::smem_bytes(nsw, c->dec_owner_slots)
+                       : DecCfg<64>::smem_bytes(nsw, c->dec_owner_slots);
   } else if (p->num_splits > 1) {
     split = true;
     splits = p->num_splits;
@@ -960,6 +1036,26 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
     lpart_off = off;
     off += (2 * static_cast<size_t>(c->splits) * rows * 4 + 255) / 256 * 256;
   }
+  // Tail of the single-pass grid (non-causal, whole 256-row tiles, library's split
+  // choice; the band and FP4 modes have no split variant): when the CTAs leave a
+  // last wave at most half full, its CTAs' keys are split instead.
+  size_t topart_off = 0, tlse_off = 0;
+  if (!split && !c->decode && !p->causal && p->num_splits == 0 && c->R % 256 == 0 &&
+      (p->precision == ATTN_EXACT || p->precision == ATTN_INT8QK_FP8PV)) {
+    const int nctas = c->units * (c->R / 256);
+    const int T = nctas % sms;
+    if (nctas > sms && T > 0 && 2 * T <= sms && kv_tiles >= 2) {
+      // the split kernel holds two CTAs per SM: 2 T tiles x k splits <= 2 x #SM
+      const int k = std::max(2, std::min(std::min(sms / T, kv_tiles), kMergeMaxSplits));
+      c->tail_items = T;
+      c->tail_k = k;
+      const size_t rows = static_cast<size_t>(T) * 256;
+      topart_off = off;
+      off += (static_cast<size_t>(k) * rows * p->head_dim * 4 + 255) / 256 * 256;
+      tlse_off = off;
+      off += (2 * static_cast<size_t>(k) * rows * 4 + 255) / 256 * 256;
+    }
+  }
   if (cudaEventCreateWithFlags(&c->done_ev, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
     delete c;
@@ -987,6 +1083,8 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   c->v_amax = vamax_off ? reinterpret_cast<unsigned*>(base + vamax_off) : nullptr;
   c->o_part = split ? reinterpret_cast<float*>(base + opart_off) : nullptr;
   c->lse_part = split ? reinterpret_cast<float*>(base + lpart_off) : nullptr;
+  c->tail_opart = c->tail_items ? reinterpret_cast<float*>(base + topart_off) : nullptr;
+  c->tail_lse = c->tail_items ? reinterpret_cast<float*>(base + tlse_off) : nullptr;
   if (cudaMemset(c->err, 0, 256) != cudaSuccess) {
     cudaFree(c->ws);
     if (c->ws_k) cudaFree(c->ws_k);
@@ -1029,8 +1127,9 @@ int attn_num_splits(const attn_ctx* c) {
 
 int attn_kernel_path(const attn_ctx* c) {
   if (!c) return 0;
-  return c->decode ? ATTN_PATH_DECODE : (c->split_path ? ATTN_PATH_SPLIT_MERGE
-                                                       : ATTN_PATH_SINGLE_PASS);
+  if (c->decode) return ATTN_PATH_DECODE;
+  if (c->split_path) return ATTN_PATH_SPLIT_MERGE;
+  return c->tail_items > 0 ? ATTN_PATH_SINGLE_PASS_TAIL : ATTN_PATH_SINGLE_PASS;
 }
 
 attn_status attn_debug_set(attn_ctx* c, unsigned flags) {
@@ -1153,6 +1252,7 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
   a.lse = lse;
   a.o_part = c->o_part;
   a.lse_part = c->lse_part;
+  a.part_rows = c->units * c->R;  // split path: every row
   a.nblk_q = ceil_div(p.q_len, 128);
   a.nblk_k = ceil_div(p.kv_len, 128);
   a.err = c->err;
@@ -1160,11 +1260,11 @@ static attn_status forward_paged_impl(attn_ctx* c, const void* q, const void* k_
   const int grid = c->units * c->row_tiles * (c->split_path ? c->splits : 1);
   attn_status s;
   if (D == 128)
-    s = f16 ? dispatch_fwd<128, false, true>(c, m, a, grid, st)
-            : dispatch_fwd<128, false, false>(c, m, a, grid, st);
+    s = f16 ? dispatch_fwd<128, false, true>(c, m, a, grid, st, c->split_path)
+            : dispatch_fwd<128, false, false>(c, m, a, grid, st, c->split_path);
   else
-    s = f16 ? dispatch_fwd<64, false, true>(c, m, a, grid, st)
-            : dispatch_fwd<64, false, false>(c, m, a, grid, st);
+    s = f16 ? dispatch_fwd<64, false, true>(c, m, a, grid, st, c->split_path)
+            : dispatch_fwd<64, false, false>(c, m, a, grid, st, c->split_path);
   if (s != ATTN_OK || !c->split_path) return s;
   if (D == 128)
     return f16 ? launch_merge<128, true>(c, o, lse, st) : launch_merge<128, false>(c, o, lse, st);
@@ -1475,19 +1575,20 @@ extern "C" attn_status attn_forward_splitkv_noalloc(const attn_params* p, const 
   a.lse = lse;
   a.o_part = c.o_part;
   a.lse_part = c.lse_part;
+  a.part_rows = c.units * c.R;  // split path: every row
   a.nblk_q = ceil_div(p->q_len, 128);
   a.nblk_k = kv_tiles;
   a.err = c.err;
   a.debug = 0;
   const int grid = c.units * c.row_tiles * c.splits;
   if (D == 128) {
-    st = f16 ? dispatch_fwd<128, false, true>(&c, m, a, grid, s)
-             : dispatch_fwd<128, false, false>(&c, m, a, grid, s);
+    st = f16 ? dispatch_fwd<128, false, true>(&c, m, a, grid, s, true)
+             : dispatch_fwd<128, false, false>(&c, m, a, grid, s, true);
     if (st == ATTN_OK)
       st = f16 ? launch_merge<128, true>(&c, o, lse, s) : launch_merge<128, false>(&c, o, lse, s);
   } else {
-    st = f16 ? dispatch_fwd<64, false, true>(&c, m, a, grid, s)
-             : dispatch_fwd<64, false, false>(&c, m, a, grid, s);
+    st = f16 ? dispatch_fwd<64, false, true>(&c, m, a, grid, s, true)
+             : dispatch_fwd<64, false, false>(&c, m, a, grid, s, true);
     if (st == ATTN_OK)
       st = f16 ? launch_merge<64, true>(&c, o, lse, s) : launch_merge<64, false>(&c, o, lse, s);
   }

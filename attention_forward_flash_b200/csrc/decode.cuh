@@ -70,6 +70,8 @@ struct DecArgs {
   int rope_inter;
   unsigned* err;
   unsigned debug;  // bit 0: warp 0 of CTA 0 never loads its second chunk (timeout test)
+  int nsw;          // ring slots per warp (2 .. DecCfg::kMaxNsw)
+  int owner_slots;  // partial-row slots of the merge area (warps * S * ceil(R / S))
 };
 
 template <int D>
@@ -84,23 +86,32 @@ struct DecCfg {
   static constexpr int kHalfBoxes = D / 64;               // boxes per chunk of K (or V)
   static constexpr int kKVBytes = kHalfBoxes * kBox;      // one chunk of K (or V)
   static constexpr int kSlotBytes = 2 * kKVBytes;         // K then V: 16 KB
-  static constexpr int kSlots = 2 * kWarps;               // two per warp
-  static constexpr int kRingBytes = kSlots * kSlotBytes;  // 128 KB
-  static constexpr int kQStride = D + 8;                  // staged Q row, 16-bit elements
-  static constexpr int kQOff = kRingBytes;
+  static constexpr int kMaxNsw = 4;                       // ring slots per warp, at most
+  // (the host takes 2: deeper rings measured slower on the decode workload)
+  // Fixed area (compile-time offsets), then the ring, then the merge area, whose
+  // sizes the host picks per problem (DecArgs::nsw, owner_slots):
+  //   Q rows [16][kQStride] 16-bit | owner weights [16][64] and (M, L, LF) [16][4] |
+  //   barriers [kWarps * kMaxNsw] | abort flag | pad | ring [kWarps * nsw][16 KB] |
+  //   partial O rows [owner_slots][kMoStride] | partial (m, l, lf, -) [owner_slots]
   // Merge area: every warp of the cluster writes its partial result for each row
   // into the CTA that owns the row (row r: CTA r mod S), partial p = split * kWarps +
   // warp at row slot p * ceil(R/S) + r / S.  With R, S <= 16, S * ceil(R/S) <= 31.
-  static constexpr int kMaxSlots = 31 * kWarps;
-  static constexpr int kMoStride = D + 4;                 // floats per partial O row
-  static constexpr int kMoOff = kQOff + 16 * kQStride * 2;
-  static constexpr int kMsOff = kMoOff + kMaxSlots * kMoStride * 4;  // (m, l, lf, -) per slot
-  static constexpr int kWtOff = kMsOff + kMaxSlots * 16;  // owner: weights [16][64], M/L/LF [16][4]
+  static constexpr int kQStride = D + 8;                  // staged Q row, 16-bit elements
+  static constexpr int kQOff = 0;
+  static constexpr int kWtOff = kQOff + 16 * kQStride * 2;
   static constexpr int kBarOff = kWtOff + 16 * 64 * 4 + 16 * 16;
-  static constexpr int kMiscOff = kBarOff + 8 * kSlots;   // abort flag
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024; // + alignment slack
-  static_assert(kMoOff % 16 == 0 && (kMoStride * 4) % 16 == 0, "merge area alignment");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static constexpr int kMiscOff = kBarOff + 8 * kWarps * kMaxNsw;
+  static constexpr int kRingOff = (kMiscOff + 16 + 1023) / 1024 * 1024;
+  static constexpr int kMaxOwnerSlots = 31 * kWarps;
+  static constexpr int kMoStride = D + 4;                 // floats per partial O row
+  static constexpr int kOwnerSlotBytes = kMoStride * 4 + 16;
+  static constexpr int kMaxSmem = 227 * 1024;
+  // dynamic shared memory of a launch (+ 1 KB to align the base)
+  static constexpr int smem_bytes(int nsw, int owner_slots) {
+    return kRingOff + kWarps * nsw * kSlotBytes + owner_slots * kOwnerSlotBytes + 1024;
+  }
+  static_assert((kMoStride * 4) % 16 == 0 && kSlotBytes % 1024 == 0, "merge area alignment");
+  static_assert(smem_bytes(2, kMaxOwnerSlots) <= kMaxSmem, "shared memory");
 };
 
 // ------------------------------------------------------- warp-level MMA, cluster
@@ -163,7 +174,18 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
+// Transpose of an 8x8 16-bit matrix held one 32-bit pair per thread (row lane/4,
+// columns 2 (lane%4), +1): afterwards each thread holds the same positions of the
+// transpose.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 // Stores into (possibly another CTA's) shared memory of the cluster.
+__device__ __forceinline__ void st_dsmem(uint32_t addr, float a) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
+}
 __device__ __forceinline__ void st_dsmem_v2(uint32_t addr, float a, float b) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b)
                : "memory");
@@ -210,13 +232,18 @@ __device__ __forceinline__ uint32_t swz_addr(uint32_t base, int row, int cc) {
 }
 
 // grid: units * S CTAs in clusters of S (S = splits per unit, <= 16); 128 threads.
-template <int D, bool F16, bool PAGED, bool ROPE>
+// TR (at most 8 rows per unit): the products are taken transposed, S^T = K Q^T and
+// O^T = V^T P^T, so that the keys and channels fill the M = 16 side of each MMA and
+// the rows the N = 8 side (no padding rows); P^T goes from the S^T accumulators to
+// the B operand of the second product by an in-register 8x8 transpose (movmatrix).
+template <int D, bool F16, bool PAGED, bool ROPE, bool TR>
 __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     flash_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecArgs a) {
   using C = DecCfg<D>;
   constexpr int kNT = C::kNT;
-  constexpr int kDN = D / 8;  // O n-tiles
+  constexpr int kMS = C::kChunk / 16;          // TR: S^T m-tiles (16 keys) per chunk
+  constexpr int kDN = TR ? D / 16 : D / 8;     // O n-tiles of 8 (TR: O^T m-tiles of 16) channels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -227,6 +254,10 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   const int u = blockIdx.x / S;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff);
   const uint32_t bar0 = smem_u32(smem + C::kBarOff);
+  const int nsw = a.nsw;
+  uint8_t* ring = smem + C::kRingOff;
+  uint8_t* mo_base = ring + C::kWarps * nsw * C::kSlotBytes;
+  uint8_t* ms_base = mo_base + a.owner_slots * C::kMoStride * 4;
   uint16_t* qs = reinterpret_cast<uint16_t*>(smem + C::kQOff);
 
   // This CTA's chunks: an even share of the union range; warp w's: every
@@ -239,12 +270,12 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   };
   const int n_mine = chunks_of(warp);
 
-  // The i-th chunk of warp w into slot 2 * w + (i & 1) (one thread).
+  // The i-th chunk of warp w into slot nsw * w + i % nsw (one thread).
   auto issue = [&](int w, int i) {
     if ((a.debug & 1u) && i == 1 && w == 0 && blockIdx.x == 0) return;  // timeout test
     const int key0 = (a.chunk0 + c_begin + w + C::kWarps * i) * C::kChunk;
-    const int slot = 2 * w + (i & 1);
-    const uint32_t dst = smem_u32(smem + slot * C::kSlotBytes);
+    const int slot = nsw * w + i % nsw;
+    const uint32_t dst = smem_u32(ring + slot * C::kSlotBytes);
     const uint32_t bar = bar0 + 8 * slot;
     mbar_arrive_expect_tx(bar, C::kSlotBytes);
     if constexpr (PAGED) {
@@ -267,7 +298,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   // The barriers first; then every warp starts its first two chunks before anything
   // else, so that the whole CTA's loads are in flight while Q is staged.
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kSlots; ++i) mbar_init(bar0 + 8 * i, 1);
+    for (int i = 0; i < C::kWarps * nsw; ++i) mbar_init(bar0 + 8 * i, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -275,8 +306,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   if (lane == 0) {
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    if (n_mine > 0) issue(warp, 0);
-    if (n_mine > 1) issue(warp, 1);
+    for (int i = 0; i < n_mine && i < nsw; ++i) issue(warp, i);
   }
   // Stage the unit's rows (zeros past R), 16 bytes per thread and step.
   const uint16_t* qsrc = a.q + static_cast<size_t>(u) * a.R * D;
@@ -288,7 +318,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   }
   __syncthreads();  // Q staged
   cluster_arrive_relaxed();  // this CTA runs (waited for before the first remote store)
-  int issued = min(n_mine, 2);
+  int issued = min(n_mine, nsw);
   if constexpr (ROPE) {
     // rotate each pair of the staged rows: the same float32 operations and 16-bit
     // rounding as every other rotation of the library
@@ -306,22 +336,24 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     }
     __syncthreads();
   }
-  // Q fragments (A operand: rows g and g + 8, channels 16 ks + 2t (+1, +8, +9))
+  // Q fragments: the A operand (rows g and g + 8, channels 16 ks + 2t (+1, +8, +9)),
+  // or with TR the B operand of S^T (row g, the same channels; words 0 and 2).
   uint32_t qa[D / 16][4];
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
     const uint16_t* r0 = qs + g * C::kQStride + 16 * ks + 2 * t;
     const uint16_t* r1 = r0 + 8 * C::kQStride;
     qa[ks][0] = *reinterpret_cast<const uint32_t*>(r0);
-    qa[ks][1] = *reinterpret_cast<const uint32_t*>(r1);
+    qa[ks][1] = TR ? 0u : *reinterpret_cast<const uint32_t*>(r1);
     qa[ks][2] = *reinterpret_cast<const uint32_t*>(r0 + 8);
-    qa[ks][3] = *reinterpret_cast<const uint32_t*>(r1 + 8);
+    qa[ks][3] = TR ? 0u : *reinterpret_cast<const uint32_t*>(r1 + 8);
   }
-  // visible key range of this thread's two rows (a padding row sees nothing)
+  // visible key range of this thread's two rows (g and g + 8; TR: 2t and 2t + 1; a
+  // padding row sees nothing)
   int lo[2], hi[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int r = g + 8 * h;
+    const int r = TR ? 2 * t + h : g + 8 * h;
     const int p = a.start_pos + r % a.Sq;
     lo[h] = max(a.window_lo, 0);
     if (a.window_size > 0) lo[h] = max(lo[h], p - a.window_size + 1);
@@ -339,8 +371,8 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   int done = 0;
   bool ok = true;
   for (int i = 0; i < n_mine; ++i) {
-    const int slot = 2 * warp + (i & 1);
-    ok = __all_sync(0xffffffffu, mbar_wait(bar0 + 8 * slot, (i >> 1) & 1, abort_flag));
+    const int slot = nsw * warp + i % nsw;
+    ok = __all_sync(0xffffffffu, mbar_wait(bar0 + 8 * slot, (i / nsw) & 1, abort_flag));
     if (!ok) {
       if (lane == 0) {
         *abort_flag = 1;
@@ -349,13 +381,13 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
       break;
     }
     const int key0 = (a.chunk0 + c_begin + warp + C::kWarps * i) * C::kChunk;
-    const uint32_t kb = smem_u32(smem + slot * C::kSlotBytes);
+    const uint32_t kb = smem_u32(ring + slot * C::kSlotBytes);
     const uint32_t vb = kb + C::kKVBytes;
     if constexpr (PAGED) {
       // keys past kv_len in the last block: clear V there (P is 0, but 0 * NaN is not)
       if (key0 + C::kChunk > a.Skv) {
         const int from = max(a.Skv - key0, 0);
-        uint4* vrow = reinterpret_cast<uint4*>(smem + slot * C::kSlotBytes + C::kKVBytes);
+        uint4* vrow = reinterpret_cast<uint4*>(ring + slot * C::kSlotBytes + C::kKVBytes);
         for (int e = lane; e < (C::kChunk - from) * (D / 8); e += 32) {
           const int row = from + e / (D / 8), cc = e % (D / 8);
           vrow[((cc >> 3) * C::kBox + row * 128) / 16 + (cc & 7)] = make_uint4(0u, 0u, 0u, 0u);
@@ -363,90 +395,172 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         __syncwarp();
       }
     }
-    // S = Q K^T for the chunk's kNT n-tiles of 8 keys (even and odd k-steps into
-    // separate accumulators: two dependency chains of D/32 MMAs per n-tile)
-    float s[kNT][4], s2[kNT][4];
+    if constexpr (TR) {
+      // S^T = K Q^T: kMS m-tiles of 16 keys (even and odd k-steps into separate
+      // accumulators)
+      float st[kMS][4], st2[kMS][4];
 #pragma unroll
-    for (int nt = 0; nt < kNT; ++nt)
+      for (int ms = 0; ms < kMS; ++ms)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.0f;
+        for (int e = 0; e < 4; ++e) st[ms][e] = st2[ms][e] = 0.0f;
 #pragma unroll
-    for (int ks2 = 0; ks2 < D / 32; ++ks2) {
+      for (int ks = 0; ks < D / 16; ++ks) {
 #pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(swz_addr<D>(kb, nt * 8 + (lane & 7), 4 * ks2 + (lane >> 3)), b0, b1, b2, b3);
-        mma16816<F16>(s[nt], qa[2 * ks2], b0, b1);
-        mma16816<F16>(s2[nt], qa[2 * ks2 + 1], b2, b3);
+        for (int ms = 0; ms < kMS; ++ms) {
+          uint32_t ka[4];
+          ldsm_x4(swz_addr<D>(kb, 16 * ms + (lane & 7) + ((lane >> 3) & 1) * 8,
+                              2 * ks + (lane >> 4)),
+                  ka[0], ka[1], ka[2], ka[3]);
+          mma16816<F16>((ks & 1) ? st2[ms] : st[ms], ka, qa[ks][0], qa[ks][2]);
+        }
       }
-    }
+      // mask, scale, running maximum per row (row 2t + h: elements e with e % 2 == h;
+      // keys 16 ms + g and + 8), reduced over the eight lanes of a column
+      float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int nt = 0; nt < kNT; ++nt)
+      for (int ms = 0; ms < kMS; ++ms) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
-    // mask, scale to base 2, running maximum per row
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int h = e >> 1;
-        const int j = key0 + nt * 8 + 2 * t + (e & 1);
-        const float x = (j < lo[h] || j > hi[h]) ? -INFINITY : s[nt][e] * a.scale_log2;
-        s[nt][e] = x;
-        mx[h] = fmaxf(mx[h], x);
+        for (int e = 0; e < 4; ++e) {
+          const int h = e & 1;
+          const int j = key0 + 16 * ms + g + (e >> 1) * 8;
+          const float x =
+              (j < lo[h] || j > hi[h]) ? -INFINITY : (st[ms][e] + st2[ms][e]) * a.scale_log2;
+          st[ms][e] = x;
+          mx[h] = fmaxf(mx[h], x);
+        }
       }
-    }
-    float bse[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-      const float mn = fmaxf(m[h], mx[h]);
-      bse[h] = mn == -INFINITY ? 0.0f : mn;
-      const float alpha = ex2(m[h] - bse[h]);  // 0 while the row has seen nothing
-      m[h] = mn;
-      la[h] *= alpha;
-      lb[h] *= alpha;
-      lf[h] *= alpha;
-#pragma unroll
-      for (int dn = 0; dn < kDN; ++dn) {
-        o[dn][2 * h] *= alpha;
-        o[dn][2 * h + 1] *= alpha;
-      }
-    }
-    // P = 2^(x - m), rounded to the 16-bit type for P V; A fragments of P V
-    uint32_t pa[kNT / 2][4];
-#pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) {
+      float bse[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const float p0 = ex2(s[nt][2 * h] - bse[h]), p1 = ex2(s[nt][2 * h + 1] - bse[h]);
-        lf[h] += p0 + p1;
-        const uint32_t w = pack16x2<F16>(p0, p1);
-        add_16x2<F16>(w, la[h], lb[h]);
-        pa[nt >> 1][(nt & 1) * 2 + h] = w;
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
+        const float mn = fmaxf(m[h], mx[h]);
+        bse[h] = mn == -INFINITY ? 0.0f : mn;
+        const float alpha = ex2(m[h] - bse[h]);
+        m[h] = mn;
+        la[h] *= alpha;
+        lb[h] *= alpha;
+        lf[h] *= alpha;
+#pragma unroll
+        for (int mt = 0; mt < kDN; ++mt) {
+          o[mt][h] *= alpha;
+          o[mt][2 + h] *= alpha;
+        }
       }
-    }
-    // O += P V: k-steps of 16 keys, two n-tiles of 8 channels per transposed load
+      // P^T (16-bit) by 8x8 blocks, transposed into the B operand of O^T += V^T P^T
+      uint32_t pb[kMS][2];
 #pragma unroll
-    for (int kk = 0; kk < kNT / 2; ++kk) {
+      for (int ms = 0; ms < kMS; ++ms) {
 #pragma unroll
-      for (int dn2 = 0; dn2 < D / 16; ++dn2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(swz_addr<D>(vb, 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8,
-                              2 * dn2 + (lane >> 4)),
-                  b0, b1, b2, b3);
-        mma16816<F16>(o[2 * dn2], pa[kk], b0, b1);
-        mma16816<F16>(o[2 * dn2 + 1], pa[kk], b2, b3);
+        for (int hk = 0; hk < 2; ++hk) {  // keys g (hk 0) and g + 8 (hk 1)
+          const float p0 = ex2(st[ms][2 * hk] - bse[0]), p1 = ex2(st[ms][2 * hk + 1] - bse[1]);
+          lf[0] += p0;
+          lf[1] += p1;
+          const uint32_t w = pack16x2<F16>(p0, p1);  // (row 2t, row 2t + 1) at one key
+          if (hk == 0) add_16x2<F16>(w, la[0], la[1]);
+          else add_16x2<F16>(w, lb[0], lb[1]);
+          pb[ms][hk] = movmatrix_t(w);
+        }
+      }
+      // O^T += V^T P^T: m-tiles of 16 channels, k-steps of 16 keys
+#pragma unroll
+      for (int kk = 0; kk < kMS; ++kk) {
+#pragma unroll
+        for (int mt = 0; mt < kDN; ++mt) {
+          uint32_t va[4];
+          ldsm_x4_t(swz_addr<D>(vb, 16 * kk + (lane & 7) + ((lane >> 4) & 1) * 8,
+                                2 * mt + ((lane >> 3) & 1)),
+                    va[0], va[1], va[2], va[3]);
+          mma16816<F16>(o[mt], va, pb[kk][0], pb[kk][1]);
+        }
+      }
+    } else {
+      // S = Q K^T for the chunk's kNT n-tiles of 8 keys (even and odd k-steps into
+      // separate accumulators: two dependency chains of D/32 MMAs per n-tile)
+      float s[kNT][4], s2[kNT][4];
+  #pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.0f;
+  #pragma unroll
+      for (int ks2 = 0; ks2 < D / 32; ++ks2) {
+  #pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(swz_addr<D>(kb, nt * 8 + (lane & 7), 4 * ks2 + (lane >> 3)), b0, b1, b2, b3);
+          mma16816<F16>(s[nt], qa[2 * ks2], b0, b1);
+          mma16816<F16>(s2[nt], qa[2 * ks2 + 1], b2, b3);
+        }
+      }
+  #pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
+      // mask, scale to base 2, running maximum per row
+      float mx[2] = {-INFINITY, -INFINITY};
+  #pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int h = e >> 1;
+          const int j = key0 + nt * 8 + 2 * t + (e & 1);
+          const float x = (j < lo[h] || j > hi[h]) ? -INFINITY : s[nt][e] * a.scale_log2;
+          s[nt][e] = x;
+          mx[h] = fmaxf(mx[h], x);
+        }
+      }
+      float bse[2];
+  #pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+        const float mn = fmaxf(m[h], mx[h]);
+        bse[h] = mn == -INFINITY ? 0.0f : mn;
+        const float alpha = ex2(m[h] - bse[h]);  // 0 while the row has seen nothing
+        m[h] = mn;
+        la[h] *= alpha;
+        lb[h] *= alpha;
+        lf[h] *= alpha;
+  #pragma unroll
+        for (int dn = 0; dn < kDN; ++dn) {
+          o[dn][2 * h] *= alpha;
+          o[dn][2 * h + 1] *= alpha;
+        }
+      }
+      // P = 2^(x - m), rounded to the 16-bit type for P V; A fragments of P V
+      uint32_t pa[kNT / 2][4];
+  #pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float p0 = ex2(s[nt][2 * h] - bse[h]), p1 = ex2(s[nt][2 * h + 1] - bse[h]);
+          lf[h] += p0 + p1;
+          const uint32_t w = pack16x2<F16>(p0, p1);
+          add_16x2<F16>(w, la[h], lb[h]);
+          pa[nt >> 1][(nt & 1) * 2 + h] = w;
+        }
+      }
+      // O += P V: k-steps of 16 keys, two n-tiles of 8 channels per transposed load
+  #pragma unroll
+      for (int kk = 0; kk < kNT / 2; ++kk) {
+  #pragma unroll
+        for (int dn2 = 0; dn2 < D / 16; ++dn2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(swz_addr<D>(vb, 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8,
+                                2 * dn2 + (lane >> 4)),
+                    b0, b1, b2, b3);
+          mma16816<F16>(o[2 * dn2], pa[kk], b0, b1);
+          mma16816<F16>(o[2 * dn2 + 1], pa[kk], b2, b3);
+        }
       }
     }
     ++done;
     __syncwarp();
-    if (i + 2 < n_mine) {
+    if (i + nsw < n_mine) {
       if (lane == 0) {
         fence_proxy_async_smem();  // this warp's reads (and clears) before the next copy
-        issue(warp, i + 2);
+        issue(warp, i + nsw);
       }
       ++issued;
     }
@@ -454,9 +568,9 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   // Never leave with a copy in flight into this CTA's shared memory.
   if (!ok && lane == 0) {
     for (int i = done; i < issued; ++i) {
-      const uint32_t bar = bar0 + 8 * (2 * warp + (i & 1));
+      const uint32_t bar = bar0 + 8 * (nsw * warp + i % nsw);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait_sleep(bar, (i >> 1) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      while (!mbar_try_wait_sleep(bar, (i / nsw) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
   }
@@ -464,10 +578,11 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     l[h] = la[h] + lb[h];
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
-    lf[h] += __shfl_xor_sync(0xffffffffu, lf[h], 1);
-    lf[h] += __shfl_xor_sync(0xffffffffu, lf[h], 2);
+#pragma unroll
+    for (int o2 = TR ? 4 : 1; o2 <= (TR ? 16 : 2); o2 <<= 1) {
+      l[h] += __shfl_xor_sync(0xffffffffu, l[h], o2);
+      lf[h] += __shfl_xor_sync(0xffffffffu, lf[h], o2);
+    }
   }
 
   // ---- merge: each warp writes its partial (m, l, lf, O) of every row into the
@@ -475,20 +590,29 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   // combines its rows' S * kWarps partials with one denominator and writes them.
   const int rpo = (a.R + S - 1) / S;            // rows per owner
   const int np = S * C::kWarps;                 // partials per row
-  const uint32_t mo_u = smem_u32(smem + C::kMoOff), ms_u = smem_u32(smem + C::kMsOff);
+  const uint32_t mo_u = smem_u32(mo_base), ms_u = smem_u32(ms_base);
   const int part = split * C::kWarps + warp;
   cluster_wait();  // every CTA of the cluster has started
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int r = g + 8 * h;
+    const int r = TR ? 2 * t + h : g + 8 * h;
     if (r < a.R) {
       const uint32_t owner = static_cast<uint32_t>(r % S);
       const int slot = part * rpo + r / S;
       const uint32_t dst = dsmem_addr(mo_u + slot * C::kMoStride * 4, owner);
+      if constexpr (TR) {  // channels 16 mt + g and + 8 of row 2t + h
 #pragma unroll
-      for (int dn = 0; dn < kDN; ++dn)
-        st_dsmem_v2(dst + (8 * dn + 2 * t) * 4, o[dn][2 * h], o[dn][2 * h + 1]);
-      if (t == 0) st_dsmem_v4(dsmem_addr(ms_u + slot * 16, owner), m[h], l[h], lf[h], 0.0f);
+        for (int mt = 0; mt < kDN; ++mt) {
+          st_dsmem(dst + (16 * mt + g) * 4, o[mt][h]);
+          st_dsmem(dst + (16 * mt + g + 8) * 4, o[mt][2 + h]);
+        }
+        if (g == 0) st_dsmem_v4(dsmem_addr(ms_u + slot * 16, owner), m[h], l[h], lf[h], 0.0f);
+      } else {
+#pragma unroll
+        for (int dn = 0; dn < kDN; ++dn)
+          st_dsmem_v2(dst + (8 * dn + 2 * t) * 4, o[dn][2 * h], o[dn][2 * h + 1]);
+        if (t == 0) st_dsmem_v4(dsmem_addr(ms_u + slot * 16, owner), m[h], l[h], lf[h], 0.0f);
+      }
     }
   }
   cluster_sync();
@@ -496,8 +620,8 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
   // Owner: per owned row, one warp forms the maximum over the row's partials, their
   // weights 2^(m_p - M) (into shared memory) and the two denominators; then every
   // thread sums its channel over the partials.
-  const float* mo = reinterpret_cast<const float*>(smem + C::kMoOff);
-  const float4* ms = reinterpret_cast<const float4*>(smem + C::kMsOff);
+  const float* mo = reinterpret_cast<const float*>(mo_base);
+  const float4* ms = reinterpret_cast<const float4*>(ms_base);
   float* wt = reinterpret_cast<float*>(smem + C::kWtOff);      // [rpo][64] weights
   float* rs = reinterpret_cast<float*>(smem + C::kWtOff + 16 * 64 * 4);  // [rpo][4]: M, L, LF
   const int nown = split < a.R ? (a.R - split + S - 1) / S : 0;  // rows this CTA owns

@@ -65,8 +65,14 @@ struct FwdArgs {
   int tph;
   float scale_log2;  // scale * log2(e)
   float* lse;        // [units * R] natural-log lse or nullptr (non-split variant)
-  float* o_part;     // [splits, units, R, D] float32 (split variant)
-  float* lse_part;   // [2, splits, units, R] base-2 lse of the P.V weights, then of the
+  // Split variant: CTA b works on 128-row tile tile0 + b / splits (tiles numbered
+  // unit-major over the whole problem) and key split b % splits.  Its partial rows are
+  // the rows part_row0 .. part_row0 + part_rows - 1 of the problem (unit-major).
+  int tile0;
+  int part_row0;
+  int part_rows;
+  float* o_part;     // [splits, part_rows, D] float32 (split variant)
+  float* lse_part;   // [2, splits, part_rows] base-2 lse of the P.V weights, then of the
                      // float32 weights (split variant)
   const float* q_scale;  // quantised variant
   const float* k_scale;
@@ -352,7 +358,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>::kThre
     int lin = blockIdx.x;
     if constexpr (SPLIT) {
       split = lin % a.splits;
-      lin /= a.splits;
+      lin = lin / a.splits + a.tile0;
     }
     if (!SPLIT && a.causal && a.tph > 0) {
       const int per_band = a.units * a.G;  // row tiles of one position band
@@ -1136,7 +1142,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>::kThre
     const float lse2_w = (l > 0.0f) ? m_used + lg2(l) - C::kPScale : -INFINITY;
     const float lse2 = (lf > 0.0f) ? m_used + lg2(lf) - C::kPScale : -INFINITY;
     if constexpr (SPLIT) {
-      const size_t prow = ((size_t)split * a.units + u) * a.R + r;
+      const size_t prow = (size_t)split * a.part_rows + ((size_t)u * a.R + r - a.part_row0);
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -1169,7 +1175,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>::kThre
       }
       if (rvalid) {
         a.lse_part[prow] = lse2_w;
-        a.lse_part[(size_t)a.splits * a.units * a.R + prow] = lse2;
+        a.lse_part[(size_t)a.splits * a.part_rows + prow] = lse2;
       }
     } else {
       const uint32_t stage = C::kStageInQBuf ? sbase + C::kQOff + q * C::kQTile

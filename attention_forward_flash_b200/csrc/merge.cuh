@@ -20,7 +20,9 @@ namespace attn {
 constexpr int kMergeMaxSplits = 128;
 constexpr int kMergeWarps = 4;
 
-// grid: rows, 128 threads; one CTA per output row.  Every warp loads all
+// grid: rows, 128 threads; one CTA per output row.  The partials of split sp and
+// row r are at sp * stride + r (stride >= rows: a window of a larger partial
+// buffer).  Every warp loads all
 // splits' weight exponents (one per lane) together with the partial outputs of
 // its own splits w, w + 4, ..., so that both arrive in one memory round trip;
 // each warp then forms the maximum, its splits' weights and the denominator
@@ -28,7 +30,7 @@ constexpr int kMergeWarps = 4;
 template <int D, bool F16>
 __global__ void __launch_bounds__(32 * kMergeWarps) splitkv_merge_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
-    uint16_t* __restrict__ out, float* __restrict__ lse, int rows, int splits) {
+    uint16_t* __restrict__ out, float* __restrict__ lse, int stride, int splits) {
   constexpr int kPer = D / 32;                    // channels per lane
   constexpr int kMaxPerWarp = kMergeMaxSplits / kMergeWarps;
   __shared__ float red[kMergeWarps][D];
@@ -42,7 +44,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) splitkv_merge_kernel(
 #pragma unroll
   for (int k = 0; k < kMergeMaxSplits / 32; ++k) {
     const int sp = lane + 32 * k;
-    W[k] = sp < splits ? lse_part[(size_t)sp * rows + row] : -INFINITY;
+    W[k] = sp < splits ? lse_part[(size_t)sp * stride + row] : -INFINITY;
   }
   // this warp's partial outputs, all loads in flight
   float part[kMaxPerWarp / 4][kPer];  // splits warp + 4 i, in groups processed below
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) splitkv_merge_kernel(
 #pragma unroll
     for (int i = 0; i < kMaxPerWarp / 4; ++i) {
       const int sp = warp + 4 * (i0 + i);
-      const float* src = o_part + ((size_t)sp * rows + row) * D + lane * kPer;
+      const float* src = o_part + ((size_t)sp * stride + row) * D + lane * kPer;
       if (sp < splits) {
         if constexpr (kPer == 4) {
           const float4 v = *reinterpret_cast<const float4*>(src);
@@ -98,12 +100,12 @@ __global__ void __launch_bounds__(32 * kMergeWarps) splitkv_merge_kernel(
 #pragma unroll
   for (int e = 0; e < kPer; ++e) red[warp][lane * kPer + e] = acc[e];
   if (warp == 1 && lse != nullptr) {
-    const float* lf = lse_part + (size_t)splits * rows;
+    const float* lf = lse_part + (size_t)splits * stride;
     float ML = -INFINITY, F[kMergeMaxSplits / 32];
 #pragma unroll
     for (int k = 0; k < kMergeMaxSplits / 32; ++k) {
       const int sp = lane + 32 * k;
-      F[k] = sp < splits ? lf[(size_t)sp * rows + row] : -INFINITY;
+      F[k] = sp < splits ? lf[(size_t)sp * stride + row] : -INFINITY;
       ML = fmaxf(ML, F[k]);
     }
 #pragma unroll

@@ -186,7 +186,8 @@ def make_attention(w: Workload, precision):
 
 
 def launches_per_step(att, precision):
-    n = 1 + (1 if att.kernel_path == "split_merge" else 0)  # the merge kernel
+    path = att.kernel_path
+    n = {"split_merge": 2, "single_pass_tail": 3}.get(path, 1)  # + split kernel, merge
     if precision != "exact":
         n += 4  # Q and K block quantisers, V channel maxima, V quantiser
     elif att.params.rope_dim > 0 and not att.params.rope_keys_rotated:
@@ -406,7 +407,7 @@ def measure(w: Workload, precision, steps, warmup, device):
     ms_kernel = ms_step if precision == "exact" else time_steps(kernel_only, steps, 2, flush)
     att.check_error()
     return dict(ms_step=ms_step, ms_kernel=ms_kernel, att=att, q=q, k=k, v=v, out=out, qb=qb,
-                launches=launches_per_step(att, precision))
+                launches=launches_per_step(att, precision), flush=flush)
 
 
 def measure_e2e(w: Workload, precision, m, steps, warmup, chunks=0):
@@ -462,25 +463,40 @@ def run_native(args):
         step()
     torch.cuda.synchronize()
     barrier(world)
+    flush = m["flush"]  # inputs that fit in L2: flushed before every timed step
     with ClockSampler(local_rank) as clocks:
         torch.cuda.synchronize()
         barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
-            step()
-        e1.record()
-        torch.cuda.synchronize()
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                step()
+            e1.record()
+            torch.cuda.synchronize()
+            ms_local = e0.elapsed_time(e1) / args.steps
+        else:
+            total = 0.0
+            for _ in range(args.steps):
+                flush()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                step()
+                e1.record()
+                e1.synchronize()
+                total += e0.elapsed_time(e1)
+            torch.cuda.synchronize()
+            ms_local = total / args.steps
         barrier(world)
     att.check_error()
-    ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local, world)
     flops = work_flops(w)
     value = flops * world / (ms * 1e-3) / 1e12
 
     # ---- dominant kernel (the fused attention kernel) for the roofline
     if precision != "exact":
-        ms_kernel = time_steps(lambda: att.forward(q, k, v, qbufs=qb, out=out), args.steps, 2)
+        ms_kernel = time_steps(lambda: att.forward(q, k, v, qbufs=qb, out=out), args.steps, 2,
+                               flush)
     else:
         ms_kernel = ms_local
     peak_key = "bf16_tflops"
@@ -493,6 +509,16 @@ def run_native(args):
                 "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" +
                 (" x2 for INT8/FP8" if precision != "exact" else ""),
                 "kernel": "flash_fwd_kernel", "kernel_ms": ms_kernel}
+    if att.kernel_path == "decode":
+        # decode-shaped: bound by reading K and V once from HBM
+        kv_bytes = 2 * w.batch * w.n_kv_heads * w.kv_len * w.head_dim * 2
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        gbs = kv_bytes / (ms_kernel * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                    "frac": gbs / hbm, "traffic": None,
+                    "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json)",
+                    "kernel": "flash_decode_kernel", "kernel_ms": ms_kernel,
+                    "algorithmic_bytes": kv_bytes}
 
     # ---- the quantisers on their own (quantised mode): an HBM-bound pass whose
     # algorithmic bytes are Q and K read once, V read twice (channel maxima, then

@@ -342,6 +342,11 @@ int attn_num_splits(const attn_ctx *c);
  *   ATTN_PATH_SPLIT_MERGE  one 128-row query tile per CTA, the keys split across
  *                          CTAs, then a merge kernel (few rows per kv head, or too few
  *                          CTAs to fill the GPU);
+ *   ATTN_PATH_SINGLE_PASS_TAIL  the single-pass kernel, whose grid would end in a
+ *                          last wave at most half full: those last CTAs' rows run
+ *                          instead on the split kernel (keys split across CTAs) and a
+ *                          merge, so that every wave is full (non-causal, exact or
+ *                          INT8 mode, Hq/Hkv * q_len a multiple of 256, num_splits 0);
  *   ATTN_PATH_DECODE       exact mode with at most 16 stacked rows per unit
  *                          (Hq/Hkv * q_len <= 16, e.g. decode steps) and num_splits
  *                          0 or 2..16: one thread-block cluster of num_splits CTAs per
@@ -356,7 +361,8 @@ int attn_num_splits(const attn_ctx *c);
 typedef enum {
   ATTN_PATH_SINGLE_PASS = 1,
   ATTN_PATH_SPLIT_MERGE = 2,
-  ATTN_PATH_DECODE = 3
+  ATTN_PATH_DECODE = 3,
+  ATTN_PATH_SINGLE_PASS_TAIL = 4
 } attn_kernel_path_kind;
 int attn_kernel_path(const attn_ctx *c);
 

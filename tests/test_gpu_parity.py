@@ -410,3 +410,46 @@ def test_exact_rescale_forced(D, G, path):
     ro, rl = oracle_for(w, q, k, v)
     check_exact(o, ro, f"G={G}")
     check_lse(lse, rl, f"G={G}")
+
+
+# Short last wave of the single-pass grid: 40 units x 4 row tiles of 256 = 160 CTAs on
+# 148 SMs would leave a last wave of 12 CTAs; their rows run instead on the split kernel
+# (keys split across CTAs) and a merge.  Every row is checked against the oracle, lse
+# included, in both modes; and with unit ranges (the host-buffer pipeline) the rows come
+# out bit-identical to the whole-problem call.
+TAIL = [Workload("tail_d64", 1, 40, 40, 1024, 1000, 64, "bf16", seed=9401),
+        Workload("tail_gqa_d128", 2, 40, 10, 512, 777, 128, "fp16", window_lo=100, seed=9402)]
+
+
+@pytest.mark.parametrize("w", TAIL, ids=[t.name for t in TAIL])
+def test_short_last_wave_runs_on_the_split_kernel(w):
+    q, k, v = make_qkv(w)
+    o, lse, att = run_gpu(w, q, k, v)
+    assert att.kernel_path == "single_pass_tail"
+    ro, rl = oracle_for(w, q, k, v)
+    check_exact(o, ro, w.name)
+    check_lse(lse, rl, w.name)
+    oq, _, attq = run_gpu(w, q, k, v, precision="quant")
+    assert attq.kernel_path == "single_pass_tail"
+    assert rel_rmse(oq, ro) <= QUANT_RMSE
+    # the forced single-pass kernel agrees to rounding
+    o1, _, att1 = run_gpu(w, q, k, v, num_splits=1)
+    assert att1.kernel_path == "single_pass"
+    check_exact(o1, ro, w.name + " single pass")
+
+
+def test_tail_rows_bit_identical_across_unit_ranges():
+    w = TAIL[0]
+    q, k, v = make_qkv(w)
+    att = Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
+                    dtype=w.torch_dtype)
+    assert att.kernel_path == "single_pass_tail"
+    ref, rl = att.forward(q.cuda(), k.cuda(), v.cuda(), return_lse=True)
+    att.check_error()
+    for chunks in (3, 7):
+        o, lse = att.forward_host(q.pin_memory(), k.pin_memory(), v.pin_memory(),
+                                  return_lse=True, chunks=chunks)
+        torch.cuda.synchronize()
+        att.check_error()
+        assert torch.equal(o.view(torch.int16), ref.cpu().view(torch.int16)), chunks
+        assert torch.equal(lse, rl.cpu()), chunks
