@@ -14,13 +14,15 @@
 //    unit's visible key range into equal runs of 64-key (head_dim 64) or 32-key
 //    (head_dim 128) chunks, so each chunk of K and V is 16 KB;
 //  * each of a CTA's four warps is an independent flash-decoding worker: it
-//    streams its own chunks (every fourth) with TMA into its own two
-//    shared-memory slots (128-byte swizzle, no multicast), keeping two chunks in
-//    flight, and computes S = Q K^T and O += P V with warp-level mma.sync
-//    (m16n8k16, 16-bit operands, float32 accumulators; the unit's rows are the
-//    M = 16 side, keys and channels the N = 8 sides), an online softmax in base 2
-//    on the accumulator fragments, and P handed from the S fragments to the
-//    P V operand in registers;
+//    streams its own chunks (every fourth) with TMA into its own ring slots
+//    (128-byte swizzle, no multicast), the first ones issued before Q is staged,
+//    and computes the two products with warp-level mma.sync (m16n8k16, 16-bit
+//    operands, float32 accumulators) and an online softmax in base 2 on the
+//    accumulator fragments.  Up to 8 rows the products are transposed (S^T = K Q^T,
+//    O^T = V^T P^T: keys and channels on the M = 16 side, the rows on N = 8; P^T
+//    reaches the second product's operand by an in-register transpose); from 9 to
+//    16 rows the rows are the M side and P goes from the S fragments to the A
+//    operand in registers;
 //  * each warp's partial result (running maximum m, the sum of the 16-bit P
 //    values that entered P V, the float32 sum for the log-sum-exp, and O) is
 //    stored straight into the shared memory of the CTA that owns the row (row r:

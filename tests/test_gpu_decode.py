@@ -172,3 +172,31 @@ def test_graph_captured_calls_then_destroy_leave_no_error():
     o, lse = att.forward(q, k, v, return_lse=True)
     att.check_error()
     check_exact(o.double().cpu().numpy(), ro, "after destroy")
+
+
+@pytest.mark.parametrize("R_rope,inter,G,Sq", [(64, True, 2, 4), (128, False, 4, 3),
+                                               (96, False, 1, 1)],
+                         ids=["interleaved_partial_8rows", "half_12rows", "partial_1row"])
+def test_decode_kernel_with_rope(R_rope, inter, G, Sq):
+    """Q rotated in the decode kernel's staged rows (keys rotated once by the call):
+    against float64 attention on float64-rotated Q and K, both pair layouts, a partial
+    rotary width, the transposed (<= 8 rows) and the row-major (9..16 rows) products."""
+    from oracle import apply_rope, rope_frequencies
+    from oracle import rope_table as oracle_table
+    w = Workload("dr", 2, 4 * G, 4, Sq, 3000, 128, "bf16", causal=True, start_pos=3000 - Sq,
+                 seed=9330 + R_rope + G)
+    q, k, v = make_qkv(w)
+    theta = rope_frequencies(R_rope, scaling="ntk", factor=4.0)
+    table = oracle_table(3000, theta)
+    att = Attention(w.batch, w.n_q_heads, w.n_kv_heads, w.q_len, w.kv_len, w.head_dim,
+                    dtype=w.torch_dtype, causal=True, start_pos=w.start_pos, rope_dim=R_rope,
+                    rope_interleaved=inter, rope_table=torch.from_numpy(table))
+    assert att.kernel_path == "decode"
+    o = att.forward(q.cuda(), k.cuda(), v.cuda())
+    att.check_error()
+    layout = "interleaved" if inter else "half"
+    qr = apply_rope(q.double().numpy(), w.start_pos + np.arange(Sq), theta, layout=layout)
+    kr = apply_rope(k.double().numpy(), np.arange(3000), theta, layout=layout)
+    from oracle import attention_f64
+    ro, _ = attention_f64(qr, kr, v.double().numpy(), causal=True, start_pos=w.start_pos)
+    check_exact(o.double().cpu().numpy(), ro, f"rope R={R_rope}")
