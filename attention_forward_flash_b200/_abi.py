@@ -17,7 +17,7 @@ EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
             "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host",
             "attn_forward_paged", "attn_rope_table", "attn_set_rope_table", "attn_rope_apply",
-            "attn_qbufs_sf_sizes", "attn_kernel_path")
+            "attn_qbufs_sf_sizes", "attn_kernel_path", "attn_plan_for")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -89,6 +89,8 @@ def lib():
         L.attn_num_splits.restype = c_int
         L.attn_kernel_path.argtypes = [vp]
         L.attn_kernel_path.restype = c_int
+        L.attn_plan_for.argtypes = [ctypes.POINTER(AttnParams), c_int, ctypes.POINTER(AttnPlan)]
+        L.attn_plan_for.restype = c_int
         L.attn_debug_set.argtypes = [vp, ctypes.c_uint]
         L.attn_debug_set.restype = c_int
         L.attn_debug_exp2.argtypes = [vp, vp, ctypes.c_size_t, vp]
@@ -160,6 +162,19 @@ def attn_num_splits(ctx):
 
 def attn_kernel_path(ctx):
     return lib().attn_kernel_path(ctx)
+
+
+class AttnPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("path", "splits", "tiles_per_split", "ctas",
+                                            "tail_items", "tail_splits", "decode_chunk",
+                                            "decode_chunks")]
+
+
+def attn_plan_for(params, num_sms):
+    """The kernel choice for ``params`` (an AttnParams) on ``num_sms`` SMs, as a dict."""
+    out = AttnPlan()
+    _check(lib().attn_plan_for(ctypes.byref(params), num_sms, ctypes.byref(out)), "attn_plan_for")
+    return {n: getattr(out, n) for n, _ in AttnPlan._fields_}
 
 
 def attn_debug_set(ctx, flags):

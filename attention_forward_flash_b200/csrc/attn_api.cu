@@ -268,6 +268,89 @@ inline uint32_t decode_chunk(int head_dim) {
   return head_dim == 128 ? DecCfg<128>::kChunk : DecCfg<64>::kChunk;
 }
 
+// The kernel choice for a problem on a GPU with `sms` SMs (attn_create, attn_plan_for).
+// `max_clusters(S)`: how many decode clusters of S CTAs the device holds at once.
+struct Plan {
+  int path = ATTN_PATH_SINGLE_PASS;
+  int splits = 1;           // key splits (decode: CTAs per cluster)
+  int tiles_per_split = 1;  // split kernel: 128-key tiles per split
+  int row_tiles = 1;        // row tiles per unit (256 rows; 128 on the split kernel)
+  int tail_items = 0;       // single pass: last-wave CTAs moved to the split kernel
+  int tail_splits = 0;
+  int dec_chunk0 = 0;       // decode: first chunk of the rows' visible union
+  int dec_nchunks = 0;
+};
+
+template <typename MaxClusters>
+void plan_problem(const attn_params& p, int sms, Plan& pl, MaxClusters&& max_clusters) {
+  const int G = p.n_q_heads / p.n_kv_heads;
+  const int R = G * p.q_len;
+  const int units = p.batch * p.n_kv_heads;
+  const int kv_tiles = ceil_div(p.kv_len, 128);
+  const int big_ctas = units * ceil_div(R, 256);
+  bool split = false, decode = false;
+  int splits = 1;
+  if (p.precision == ATTN_MIXED_DIAG || p.precision == ATTN_MXFP4QK_FP8PV) {
+    // single-pass kernel only (the band and FP4 modes have no split-KV variant)
+  } else if (p.precision == ATTN_EXACT && R <= 16 && p.kv_len > 0 &&
+             (p.num_splits == 0 ||
+              (p.num_splits > 1 && p.num_splits <= DecCfg<128>::kMaxSplits))) {
+    // Decode-shaped (at most 16 stacked rows per unit): the cluster kernel.  The
+    // union of the rows' visible key ranges: row 0 has the lowest lower bound,
+    // the last position the highest upper bound.
+    decode = true;
+    const int chunk = static_cast<int>(decode_chunk(p.head_dim));
+    long long lo = std::max(p.window_lo, 0);
+    if (p.window_size > 0)
+      lo = std::max<long long>(lo, static_cast<long long>(p.start_pos) - p.window_size + 1);
+    long long hi = p.kv_len - 1;
+    if (p.causal) hi = std::min<long long>(hi, static_cast<long long>(p.start_pos) + p.q_len - 1);
+    pl.dec_chunk0 = lo <= hi ? static_cast<int>(lo / chunk) : 0;
+    pl.dec_nchunks = lo <= hi ? static_cast<int>(hi / chunk - lo / chunk + 1) : 0;
+    // about one CTA per SM over all units (at most 16 per cluster, at most one chunk
+    // each), then as large a cluster as lets every unit's cluster (or as many as
+    // the SMs hold) be resident at once
+    int S = p.num_splits > 1 ? p.num_splits
+                             : std::max(1, std::min(DecCfg<128>::kMaxSplits, sms / units));
+    S = std::max(1, std::min(S, std::max(pl.dec_nchunks, 1)));
+    while (S > 1 && max_clusters(S) < std::min(units, std::max(1, sms / S))) --S;
+    splits = S;
+  } else if (p.num_splits > 1) {
+    split = true;
+    splits = p.num_splits;
+  } else if (p.num_splits == 0) {
+    // Few rows per kv head or too few CTAs to fill the GPU: one 128-row query tile
+    // per CTA, keys split across CTAs, then a merge.
+    if (R <= 128 || (big_ctas * 2 < sms && kv_tiles >= 4)) {
+      split = true;
+      const int base = units * ceil_div(R, 128);
+      splits = std::max(1, std::min(kv_tiles, ceil_div(2 * sms, base)));  // two CTAs per SM
+    }
+  }
+  if (!decode) {
+    splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
+    splits = std::min(splits, kMergeMaxSplits);
+  }
+  pl.tiles_per_split = std::max(1, ceil_div(kv_tiles, splits));
+  pl.splits = split ? std::max(1, ceil_div(kv_tiles, pl.tiles_per_split)) : (decode ? splits : 1);
+  pl.row_tiles = ceil_div(R, split ? 128 : 256);
+  pl.path = decode ? ATTN_PATH_DECODE : (split ? ATTN_PATH_SPLIT_MERGE : ATTN_PATH_SINGLE_PASS);
+  // Tail of the single-pass grid (non-causal, whole 256-row tiles, library's split
+  // choice; the band and FP4 modes have no split variant): when the CTAs leave a
+  // last wave at most half full, its CTAs' keys are split instead.
+  if (!split && !decode && !p.causal && p.num_splits == 0 && R % 256 == 0 &&
+      (p.precision == ATTN_EXACT || p.precision == ATTN_INT8QK_FP8PV)) {
+    const int nctas = units * (R / 256);
+    const int T = nctas % sms;
+    if (nctas > sms && T > 0 && 2 * T <= sms && kv_tiles >= 2) {
+      // the split kernel holds two CTAs per SM: 2 T tiles x k splits <= 2 x #SM
+      pl.tail_items = T;
+      pl.tail_splits = std::max(2, std::min(std::min(sms / T, kv_tiles), kMergeMaxSplits));
+      pl.path = ATTN_PATH_SINGLE_PASS_TAIL;
+    }
+  }
+}
+
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
           bool DIAG = false, bool FP4 = false>
 attn_status launch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
@@ -957,45 +1040,24 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   c->scale = p->scale > 0.0f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
   const int kv_tiles = ceil_div(p->kv_len, 128);
 
-  // Few rows per kv head (decode-shaped) or too few CTAs to fill the GPU:
-  // one 128-row query tile per CTA, keys split across CTAs, then a merge.
-  const int big_ctas = c->units * ceil_div(c->R, 256);
-  bool split = false;
-  int splits = 1;
-  if (p->precision == ATTN_MIXED_DIAG || p->precision == ATTN_MXFP4QK_FP8PV) {
-    // single-pass kernel only (the band and FP4 modes have no split-KV variant)
-  } else if (p->precision == ATTN_EXACT && c->R <= 16 && p->kv_len > 0 &&
-             (p->num_splits == 0 ||
-              (p->num_splits > 1 && p->num_splits <= DecCfg<128>::kMaxSplits))) {
-    // Decode-shaped (at most 16 stacked rows per unit): the cluster kernel.  The
-    // union of the rows' visible key ranges: row 0 has the lowest lower bound,
-    // the last position the highest upper bound.
-    const int chunk = static_cast<int>(decode_chunk(p->head_dim));
-    long long lo = std::max(p->window_lo, 0);
-    if (p->window_size > 0)
-      lo = std::max<long long>(lo, static_cast<long long>(p->start_pos) - p->window_size + 1);
-    long long hi = p->kv_len - 1;
-    if (p->causal)
-      hi = std::min<long long>(hi, static_cast<long long>(p->start_pos) + p->q_len - 1);
-    c->decode = 1;
-    c->dec_chunk0 = lo <= hi ? static_cast<int>(lo / chunk) : 0;
-    c->dec_nchunks = lo <= hi ? static_cast<int>(hi / chunk - lo / chunk + 1) : 0;
-    // about one CTA per SM over all units (at most 16 per cluster, at most one chunk
-    // each), then as large a cluster as lets every unit's cluster (or as many as
-    // the SMs hold) be resident at once
-    int S = p->num_splits > 1 ? p->num_splits
-                              : std::max(1, std::min(DecCfg<128>::kMaxSplits, sms / c->units));
-    S = std::max(1, std::min(S, std::max(c->dec_nchunks, 1)));
-    while (S > 1) {
-      const int n = p->head_dim == 128 ? decode_max_clusters<128>(c->units, S)
-                                       : decode_max_clusters<64>(c->units, S);
-      if (n >= std::min(c->units, std::max(1, sms / S))) break;
-      --S;
-    }
-    splits = S;
+  Plan pl;
+  plan_problem(*p, sms, pl, [&](int S) {
+    return p->head_dim == 128 ? decode_max_clusters<128>(c->units, S)
+                              : decode_max_clusters<64>(c->units, S);
+  });
+  const bool split = pl.path == ATTN_PATH_SPLIT_MERGE;
+  c->decode = pl.path == ATTN_PATH_DECODE ? 1 : 0;
+  c->split_path = split ? 1 : 0;
+  c->splits = pl.splits;
+  c->tiles_per_split = pl.tiles_per_split;
+  c->row_tiles = pl.row_tiles;
+  c->dec_chunk0 = pl.dec_chunk0;
+  c->dec_nchunks = pl.dec_nchunks;
+  if (c->decode) {
     // the merge area for this S, and two ring slots per warp: the K/V stream is
     // bound by the bytes the whole GPU has in flight, and a third slot per warp
     // measured slower (decode workload: 9.3 against 8.2 us per call back to back)
+    const int S = pl.splits;
     const int rpo = (c->R + S - 1) / S;
     const bool d128 = p->head_dim == 128;
     c->dec_owner_slots = DecCfg<128>::kWarps * S * rpo;
@@ -1003,24 +1065,7 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
     c->dec_nsw = nsw;
     c->dec_smem = d128 ? DecCfg<128>::smem_bytes(nsw, c->dec_owner_slots)
                        : DecCfg<64>::smem_bytes(nsw, c->dec_owner_slots);
-  } else if (p->num_splits > 1) {
-    split = true;
-    splits = p->num_splits;
-  } else if (p->num_splits == 0) {
-    if (c->R <= 128 || (big_ctas * 2 < sms && kv_tiles >= 4)) {
-      split = true;
-      const int base = c->units * ceil_div(c->R, 128);
-      splits = std::max(1, std::min(kv_tiles, ceil_div(2 * sms, base)));  // two CTAs per SM
-    }
   }
-  if (!c->decode) {
-    splits = std::min(std::max(splits, 1), std::max(kv_tiles, 1));
-    splits = std::min(splits, kMergeMaxSplits);
-  }
-  c->split_path = split ? 1 : 0;
-  c->tiles_per_split = std::max(1, ceil_div(kv_tiles, splits));
-  c->splits = split ? std::max(1, ceil_div(kv_tiles, c->tiles_per_split)) : (c->decode ? splits : 1);
-  c->row_tiles = ceil_div(c->R, split ? 128 : 256);
 
   // workspace: error word | V channel maxima | split partials
   size_t off = 256;
@@ -1040,21 +1085,15 @@ attn_status attn_create(const attn_params* p, attn_ctx** out) {
   // choice; the band and FP4 modes have no split variant): when the CTAs leave a
   // last wave at most half full, its CTAs' keys are split instead.
   size_t topart_off = 0, tlse_off = 0;
-  if (!split && !c->decode && !p->causal && p->num_splits == 0 && c->R % 256 == 0 &&
-      (p->precision == ATTN_EXACT || p->precision == ATTN_INT8QK_FP8PV)) {
-    const int nctas = c->units * (c->R / 256);
-    const int T = nctas % sms;
-    if (nctas > sms && T > 0 && 2 * T <= sms && kv_tiles >= 2) {
-      // the split kernel holds two CTAs per SM: 2 T tiles x k splits <= 2 x #SM
-      const int k = std::max(2, std::min(std::min(sms / T, kv_tiles), kMergeMaxSplits));
-      c->tail_items = T;
-      c->tail_k = k;
-      const size_t rows = static_cast<size_t>(T) * 256;
-      topart_off = off;
-      off += (static_cast<size_t>(k) * rows * p->head_dim * 4 + 255) / 256 * 256;
-      tlse_off = off;
-      off += (2 * static_cast<size_t>(k) * rows * 4 + 255) / 256 * 256;
-    }
+  if (pl.path == ATTN_PATH_SINGLE_PASS_TAIL) {
+    const int T = pl.tail_items, k = pl.tail_splits;
+    c->tail_items = T;
+    c->tail_k = k;
+    const size_t rows = static_cast<size_t>(T) * 256;
+    topart_off = off;
+    off += (static_cast<size_t>(k) * rows * p->head_dim * 4 + 255) / 256 * 256;
+    tlse_off = off;
+    off += (2 * static_cast<size_t>(k) * rows * 4 + 255) / 256 * 256;
   }
   if (cudaEventCreateWithFlags(&c->done_ev, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
@@ -1123,6 +1162,27 @@ void attn_destroy(attn_ctx* c) {
 
 int attn_num_splits(const attn_ctx* c) {
   return c ? ((c->split_path || c->decode) ? c->splits : 1) : 0;
+}
+
+attn_status attn_plan_for(const attn_params* p, int num_sms, attn_plan* out) {
+  if (!out || num_sms < 1) return ATTN_ERR_INVALID_ARG;
+  const attn_status v = validate(p);
+  if (v != ATTN_OK) return v;
+  Plan pl;
+  plan_problem(*p, num_sms, pl, [](int) { return 1 << 30; });
+  const int units = p->batch * p->n_kv_heads;
+  out->path = pl.path;
+  out->splits = pl.splits;
+  out->tiles_per_split = pl.path == ATTN_PATH_SPLIT_MERGE ? pl.tiles_per_split : 0;
+  out->ctas = pl.path == ATTN_PATH_DECODE
+                  ? units * pl.splits
+                  : units * pl.row_tiles * (pl.path == ATTN_PATH_SPLIT_MERGE ? pl.splits : 1) -
+                        pl.tail_items;
+  out->tail_items = pl.tail_items;
+  out->tail_splits = pl.tail_splits;
+  out->decode_chunk = pl.path == ATTN_PATH_DECODE ? static_cast<int>(decode_chunk(p->head_dim)) : 0;
+  out->decode_chunks = pl.dec_nchunks;
+  return ATTN_OK;
 }
 
 int attn_kernel_path(const attn_ctx* c) {

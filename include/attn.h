@@ -366,6 +366,32 @@ typedef enum {
 } attn_kernel_path_kind;
 int attn_kernel_path(const attn_ctx *c);
 
+/* The kernel choice attn_create makes for `p` on a GPU with `num_sms` SMs, as plain
+ * host arithmetic (no device is touched).  attn_create makes the same choice, except
+ * that on the device it may lower a decode cluster's size (`splits`) until every
+ * (batch, kv head)'s cluster fits at once.
+ *   path             attn_kernel_path_kind
+ *   splits           key splits (1: none; ATTN_PATH_DECODE: CTAs per cluster)
+ *   tiles_per_split  ATTN_PATH_SPLIT_MERGE: 128-key tiles per split (else 0)
+ *   ctas             CTAs of the main launch
+ *   tail_items       ATTN_PATH_SINGLE_PASS_TAIL: 256-row CTAs moved to the split kernel
+ *   tail_splits      their key splits
+ *   decode_chunk     ATTN_PATH_DECODE: keys per chunk (32 at head_dim 128, 64 at 64)
+ *   decode_chunks    ATTN_PATH_DECODE: chunks covering the rows' visible keys
+ * Errors: those of attn_create's validation of `p`; ATTN_ERR_INVALID_ARG for a NULL
+ * `out` or num_sms < 1. */
+typedef struct {
+  int path;
+  int splits;
+  int tiles_per_split;
+  int ctas;
+  int tail_items;
+  int tail_splits;
+  int decode_chunk;
+  int decode_chunks;
+} attn_plan;
+attn_status attn_plan_for(const attn_params *p, int num_sms, attn_plan *out);
+
 /* TEST HOOK.  Bit 0 of `flags` makes the next attn_forward's loader skip the
  * second key tile of every CTA (ATTN_PATH_DECODE: the second key chunk of the
  * first warp of the first CTA), so that the waits on it run out: the kernel then

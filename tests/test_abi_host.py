@@ -133,6 +133,8 @@ int main(void) {
   attn_qbufs_sf_sizes(&p, sizes);
   attn_num_splits(c);
   if (attn_kernel_path(c) == ATTN_PATH_DECODE) return 2;
+  attn_plan plan;
+  if (attn_plan_for(&p, 148, &plan) != ATTN_OK || plan.path != ATTN_PATH_SINGLE_PASS) return 3;
   attn_debug_set(c, 0u);
   attn_debug_exp2(NULL, NULL, 0, NULL);
   attn_forward_splitkv_noalloc(&p, NULL, NULL, NULL, NULL, NULL, &err, NULL);
