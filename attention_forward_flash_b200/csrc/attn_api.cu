@@ -422,6 +422,15 @@ attn_status launch_merge_rows(const float* op, const float* lp, uint16_t* out, f
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // Few splits: one warp per row.  (The choice depends on the split count alone, so
+  // that a range of rows merges exactly as the whole problem does.)
+  if (splits <= 16) {
+    cfg.gridDim = dim3((rows + 3) / 4);
+    if (cudaLaunchKernelEx(&cfg, splitkv_merge_rows_kernel<D, F16>, op, lp, out, lse, rows,
+                           stride, splits) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
   if (cudaLaunchKernelEx(&cfg, splitkv_merge_kernel<D, F16>, op, lp, out, lse, stride, splits) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;

@@ -146,6 +146,76 @@ __global__ void __launch_bounds__(32 * kMergeWarps) splitkv_merge_kernel(
   }
 }
 
+// The same merge with one warp per row, for few splits (at most 32; the host takes
+// it up to 16, e.g. the short last wave of the single-pass grid): grid
+// ceil(rows / 4), 128 threads.
+// Lane s holds split s's two weight exponents; each lane owns D / 32 channels and
+// sums them over the splits, all partial loads of a split issued together.
+template <int D, bool F16>
+__global__ void __launch_bounds__(128) splitkv_merge_rows_kernel(
+    const float* __restrict__ o_part, const float* __restrict__ lse_part,
+    uint16_t* __restrict__ out, float* __restrict__ lse, int rows, int stride, int splits) {
+  constexpr int kPer = D / 32;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float W = lane < splits ? lse_part[(size_t)lane * stride + row] : -INFINITY;
+  const float F = lane < splits ? lse_part[(size_t)(splits + lane) * stride + row] : -INFINITY;
+  float M = W, ML = F;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    ML = fmaxf(ML, __shfl_xor_sync(0xffffffffu, ML, o));
+  }
+  const float w = (M == -INFINITY || W == -INFINITY) ? 0.0f : ex2(W - M);
+  const float f = (ML == -INFINITY || F == -INFINITY) ? 0.0f : ex2(F - ML);
+  float wsum = w, fsum = f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    fsum += __shfl_xor_sync(0xffffffffu, fsum, o);
+  }
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.0f;
+  for (int sp = 0; sp < splits; ++sp) {
+    const float ws = __shfl_sync(0xffffffffu, w, sp);
+    const float* src = o_part + ((size_t)sp * stride + row) * D + lane * kPer;
+    float v[kPer];
+    if constexpr (kPer == 4) {
+      const float4 t = *reinterpret_cast<const float4*>(src);
+      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+      const float2 t = *reinterpret_cast<const float2*>(src);
+      v[0] = t.x; v[1] = t.y;
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] += ws * v[e];
+  }
+  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+  uint16_t h[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const float val = acc[e] * inv;
+    if constexpr (F16) {
+      const __half b = __float2half_rn(val);
+      h[e] = *reinterpret_cast<const uint16_t*>(&b);
+    } else {
+      const __nv_bfloat16 b = __float2bfloat16_rn(val);
+      h[e] = *reinterpret_cast<const uint16_t*>(&b);
+    }
+  }
+  uint16_t* dst = out + (size_t)row * D + lane * kPer;
+  if constexpr (kPer == 4)
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+  else
+    *reinterpret_cast<uint32_t*>(dst) = h[0] | (uint32_t(h[1]) << 16);
+  if (lane == 0 && lse != nullptr)
+    lse[row] = fsum > 0.0f ? (ML + lg2(fsum)) * 0.69314718055994531f : -INFINITY;
+}
+
 // O = 0 and lse = -inf for every row (a problem whose rows see no key at all).
 __global__ void fill_lse_kernel(float* lse, size_t rows) {
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
