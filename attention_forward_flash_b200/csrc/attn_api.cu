@@ -353,7 +353,7 @@ void plan_problem(const attn_params& p, int sms, Plan& pl, MaxClusters&& max_clu
 
 template <int D, int NQT, bool QUANT, bool F16, bool SPLIT, bool LF, bool WIN, bool ROPE,
           bool DIAG = false, bool FP4 = false>
-attn_status launch_fwd(const attn_ctx* c, const FwdMaps& m, const FwdArgs& a, int grid,
+attn_status launch_fwd(const attn_ctx* /*context*/, const FwdMaps& m, const FwdArgs& a, int grid,
                        cudaStream_t st) {
   using Cfg = FwdCfg<D, NQT, QUANT, SPLIT, DIAG, FP4>;
   constexpr auto kern = flash_fwd_kernel<D, NQT, QUANT, F16, SPLIT, LF, WIN, ROPE, DIAG, FP4>;
