@@ -17,7 +17,7 @@ EXPORTED = ("attn_create", "attn_quantize_qk", "attn_forward", "attn_get_error",
             "attn_status_string", "attn_qbufs_sizes", "attn_num_splits", "attn_debug_set",
             "attn_debug_exp2", "attn_forward_splitkv_noalloc", "attn_forward_host",
             "attn_forward_paged", "attn_rope_table", "attn_set_rope_table", "attn_rope_apply",
-            "attn_qbufs_sf_sizes", "attn_kernel_path", "attn_plan_for")
+            "attn_qbufs_sf_sizes", "attn_kernel_path", "attn_plan_for", "attn_quantize_qk_paged")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -102,6 +102,9 @@ def lib():
         L.attn_forward_host.restype = c_int
         L.attn_forward_paged.argtypes = [vp, vp, vp, vp, vp, c_int, vp, vp, vp]
         L.attn_forward_paged.restype = c_int
+        L.attn_quantize_qk_paged.argtypes = [vp, vp, vp, vp, vp, c_int, ctypes.POINTER(AttnQBufs),
+                                             vp]
+        L.attn_quantize_qk_paged.restype = c_int
         L.attn_rope_table.argtypes = [c_int, c_int, ctypes.POINTER(AttnRopeFreq), vp]
         L.attn_rope_table.restype = c_int
         L.attn_set_rope_table.argtypes = [vp, vp, c_int]
@@ -129,6 +132,12 @@ def attn_create(params: AttnParams):
 
 def attn_quantize_qk(ctx, q, k, v, qbufs: AttnQBufs, stream):
     _check(lib().attn_quantize_qk(ctx, q, k, v, ctypes.byref(qbufs), stream), "attn_quantize_qk")
+
+
+def attn_quantize_qk_paged(ctx, q, k_pool, v_pool, block_table, num_blocks, qbufs: AttnQBufs,
+                           stream):
+    _check(lib().attn_quantize_qk_paged(ctx, q, k_pool, v_pool, block_table, num_blocks,
+                                        ctypes.byref(qbufs), stream), "attn_quantize_qk_paged")
 
 
 def attn_forward(ctx, q, k, v, qbufs, o, lse, stream):

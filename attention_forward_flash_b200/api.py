@@ -165,6 +165,34 @@ class Attention:
                               _stream_handle(stream))
         return qbufs
 
+    def _check_pools(self, k_pool, v_pool, block_table):
+        p = self.params
+        want = (p.n_kv_heads, 128, p.head_dim)
+        for name, t in (("k_pool", k_pool), ("v_pool", v_pool)):
+            if (t.dim() != 4 or tuple(t.shape[1:]) != want or t.dtype != self.dtype
+                    or not t.is_contiguous() or not t.is_cuda):
+                raise ValueError(f"{name}: expected contiguous CUDA {self.dtype} "
+                                 f"[blocks, {want[0]}, {want[1]}, {want[2]}]")
+        if v_pool.shape[0] != k_pool.shape[0]:
+            raise ValueError("k_pool and v_pool must hold the same number of blocks")
+        nbt = (p.kv_len + 127) // 128
+        if (block_table.dtype != torch.int32 or tuple(block_table.shape) != (p.batch, nbt)
+                or not block_table.is_contiguous() or not block_table.is_cuda):
+            raise ValueError(f"block_table: expected contiguous CUDA int32 [{p.batch}, {nbt}]")
+
+    def quantize_paged(self, q, k_pool, v_pool, block_table, qbufs=None, stream=None):
+        """INT8 mode: the quantisers with K and V read from a paged cache
+        (``attn_quantize_qk_paged``); returns the dense ``QuantBuffers`` that
+        ``forward(qbufs=...)`` takes."""
+        if self.precision != "quant":
+            raise ValueError("quantize_paged() needs precision='quant'")
+        self._check_pools(k_pool, v_pool, block_table)
+        qbufs = qbufs if qbufs is not None else QuantBuffers(self.params, q.device)
+        _abi.attn_quantize_qk_paged(self.ctx, q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                    block_table.data_ptr(), k_pool.shape[0], qbufs.struct(),
+                                    _stream_handle(stream))
+        return qbufs
+
     def forward(self, q=None, k=None, v=None, *, qbufs=None, out=None, lse=None, return_lse=False,
                 stream=None):
         p = self.params
@@ -203,19 +231,9 @@ class Attention:
         """
         p = self.params
         if self.precision != "exact":
-            raise ValueError("forward_paged() needs precision='exact'")
-        want = (p.n_kv_heads, 128, p.head_dim)
-        for name, t in (("k_pool", k_pool), ("v_pool", v_pool)):
-            if (t.dim() != 4 or tuple(t.shape[1:]) != want or t.dtype != self.dtype
-                    or not t.is_contiguous() or not t.is_cuda):
-                raise ValueError(f"{name}: expected contiguous CUDA {self.dtype} "
-                                 f"[blocks, {want[0]}, {want[1]}, {want[2]}]")
-        if v_pool.shape[0] != k_pool.shape[0]:
-            raise ValueError("k_pool and v_pool must hold the same number of blocks")
-        nbt = (p.kv_len + 127) // 128
-        if (block_table.dtype != torch.int32 or tuple(block_table.shape) != (p.batch, nbt)
-                or not block_table.is_contiguous() or not block_table.is_cuda):
-            raise ValueError(f"block_table: expected contiguous CUDA int32 [{p.batch}, {nbt}]")
+            raise ValueError("forward_paged() needs precision='exact' (the INT8 mode: "
+                             "quantize_paged(), then forward(qbufs=...))")
+        self._check_pools(k_pool, v_pool, block_table)
         if out is None:
             out = torch.empty((p.batch, p.n_q_heads, p.q_len, p.head_dim), dtype=self.dtype,
                               device=q.device)

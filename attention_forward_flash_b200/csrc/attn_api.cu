@@ -550,27 +550,27 @@ int causal_band_tiles(const attn_ctx* c) {
 template <int D, bool F16, bool ROPE>
 attn_status quant_qk_launch(const attn_ctx* c, const uint16_t* x, int8_t* codes, float* scales,
                             int S, int nblk, int tot, unsigned debug, const QuantRope& r,
-                            cudaStream_t st) {
+                            cudaStream_t st, const KvBlocks& src = KvBlocks{}) {
   using Cfg = QuantQkCfg<D, ROPE>;
   if (!set_smem<quant_qk_kernel<D, F16, ROPE>>(Cfg::kSmemBytes)) return ATTN_ERR_CUDA;
   const int ctas = std::min(tot, Cfg::kCtasPerSm * c->num_sms);
   quant_qk_kernel<D, F16, ROPE><<<ctas, 256, Cfg::kSmemBytes, st>>>(x, codes, scales, S, nblk,
-                                                                     tot, c->err, debug, r);
+                                                                     tot, c->err, debug, r, src);
   return ATTN_OK;
 }
 
 // V's channel maxima, then its transposed E4M3 codes (both quantised modes).
 template <int D, bool F16>
 attn_status v_launch(attn_ctx* c, const uint16_t* vx, unsigned* vamax, uint8_t* vt, float* vs,
-                     int nbk, unsigned BHk, cudaStream_t st) {
+                     int nbk, unsigned BHk, cudaStream_t st, const KvBlocks& src = KvBlocks{}) {
   const attn_params& p = c->p;
   const int tot = nbk * static_cast<int>(BHk);
   v_amax_kernel<D, F16><<<dim3(ceil_div(p.kv_len, kVTok), BHk), 256, 0, st>>>(vx, vamax,
-                                                                             p.kv_len);
+                                                                             p.kv_len, src);
   if (!set_smem<v_quant_kernel<D, F16>>(VQuantCfg<D>::kSmemBytes)) return ATTN_ERR_CUDA;
   const int vq_ctas = std::min(tot, VQuantCfg<D>::kCtasPerSm * c->num_sms);
   v_quant_kernel<D, F16><<<vq_ctas, 256, VQuantCfg<D>::kSmemBytes, st>>>(
-      vx, vamax, vt, vs, p.kv_len, nbk * 128, nbk, tot, c->err);
+      vx, vamax, vt, vs, p.kv_len, nbk * 128, nbk, tot, c->err, src);
   return ATTN_OK;
 }
 
@@ -581,7 +581,7 @@ attn_status quant_launch(attn_ctx* c, const uint16_t* qx, int8_t* qc, float* qs,
                          const uint16_t* kx, int8_t* kc, float* ks, const uint16_t* vx,
                          unsigned* vamax, uint8_t* vt, float* vs, int nbq, int nbk, unsigned BHq,
                          unsigned BHk, bool rope_q, bool rope_k, const QuantRope& rq,
-                         const QuantRope& rk, cudaStream_t st) {
+                         const QuantRope& rk, cudaStream_t st, const KvBlocks& kvsrc) {
   const attn_params& p = c->p;
   attn_status s = ATTN_OK;
   if (nbq > 0) {
@@ -593,10 +593,12 @@ attn_status quant_launch(attn_ctx* c, const uint16_t* qx, int8_t* qc, float* qs,
   }
   if (nbk > 0) {
     const int tot = nbk * static_cast<int>(BHk);
-    s = rope_k ? quant_qk_launch<D, F16, true>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st)
-               : quant_qk_launch<D, F16, false>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st);
+    s = rope_k ? quant_qk_launch<D, F16, true>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st,
+                                               kvsrc)
+               : quant_qk_launch<D, F16, false>(c, kx, kc, ks, p.kv_len, nbk, tot, 0u, rk, st,
+                                                kvsrc);
     if (s != ATTN_OK) return s;
-    return v_launch<D, F16>(c, vx, vamax, vt, vs, nbk, BHk, st);
+    return v_launch<D, F16>(c, vx, vamax, vt, vs, nbk, BHk, st, kvsrc);
   }
   return ATTN_OK;
 }
@@ -604,8 +606,11 @@ attn_status quant_launch(attn_ctx* c, const uint16_t* qx, int8_t* qc, float* qs,
 // Launches the quantisers on `st` for the units [u0, u0 + nu) (unit = one
 // (batch, kv head) pair with its query heads).  Pointers are those of the whole
 // problem, already validated.
+// With a paged key/value source (kvsrc.table set), k and v are the pools and the
+// range is the whole problem.
 attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const void* k,
-                           const void* v, const attn_qbufs* qb, cudaStream_t st) {
+                           const void* v, const attn_qbufs* qb, cudaStream_t st,
+                           const KvBlocks& kvsrc = KvBlocks{}) {
   const attn_params& p = c->p;
   const int D = p.head_dim;
   const bool f16 = p.dtype == ATTN_FP16;
@@ -617,8 +622,9 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
   const size_t qe = static_cast<size_t>(u0) * c->R * D;         // Q elements / codes before u0
   const size_t ke = static_cast<size_t>(u0) * p.kv_len * D;     // K, V elements before u0
   const uint16_t* qx = static_cast<const uint16_t*>(q) + (nbq > 0 ? qe : 0);
-  const uint16_t* kx = static_cast<const uint16_t*>(k) + (nbk > 0 ? ke : 0);
-  const uint16_t* vx = static_cast<const uint16_t*>(v) + (nbk > 0 ? ke : 0);
+  const size_t kvoff = (nbk > 0 && kvsrc.table == nullptr) ? ke : 0;
+  const uint16_t* kx = static_cast<const uint16_t*>(k) + kvoff;
+  const uint16_t* vx = static_cast<const uint16_t*>(v) + kvoff;
   int8_t* qc = nbq > 0 ? qb->q + qe : nullptr;
   float* qs = (nbq > 0 && qb->q_scale) ? qb->q_scale + static_cast<size_t>(u0) * c->G * nbq
                                        : nullptr;
@@ -661,14 +667,14 @@ attn_status quantize_units(attn_ctx* c, int u0, int nu, const void* q, const voi
   attn_status s = ATTN_OK;
   if (D == 128) {
     s = f16 ? quant_launch<128, true>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
-                                      BHq, BHk, rope, rope_k, rq, rk, st)
+                                      BHq, BHk, rope, rope_k, rq, rk, st, kvsrc)
             : quant_launch<128, false>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
-                                       BHq, BHk, rope, rope_k, rq, rk, st);
+                                       BHq, BHk, rope, rope_k, rq, rk, st, kvsrc);
   } else {
     s = f16 ? quant_launch<64, true>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
-                                     BHq, BHk, rope, rope_k, rq, rk, st)
+                                     BHq, BHk, rope, rope_k, rq, rk, st, kvsrc)
             : quant_launch<64, false>(c, qx, qc, qs, kx, kc, ks, vx, vamax, vt, vs, nbq, nbk,
-                                      BHq, BHk, rope, rope_k, rq, rk, st);
+                                      BHq, BHk, rope, rope_k, rq, rk, st, kvsrc);
   }
   if (s != ATTN_OK) return s;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -1223,7 +1229,8 @@ attn_status attn_get_error(attn_ctx* c, void* stream) {
   if (cudaMemcpy(&h, c->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
   if (h != 0) {
     if (cudaMemset(c->err, 0, 4) != cudaSuccess) return ATTN_ERR_CUDA;
-    return ATTN_ERR_TIMEOUT;
+    // a paged quantiser met a block-table entry outside the pool; else a wait ran out
+    return (h & kErrBadBlock) ? ATTN_ERR_INVALID_ARG : ATTN_ERR_TIMEOUT;
   }
   return ATTN_OK;
 }
@@ -1237,6 +1244,25 @@ attn_status attn_quantize_qk(attn_ctx* c, const void* q, const void* k, const vo
     return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return mark_done(c, quantize_units(c, 0, c->units, q, k, v, qb, st), st);
+}
+
+attn_status attn_quantize_qk_paged(attn_ctx* c, const void* q, const void* k_pool,
+                                   const void* v_pool, const int32_t* block_table,
+                                   int num_blocks, const attn_qbufs* qb, void* stream) {
+  if (!c || !qb) return ATTN_ERR_INVALID_ARG;
+  const attn_params& p = c->p;
+  if (p.precision != ATTN_INT8QK_FP8PV) return ATTN_ERR_UNSUPPORTED;
+  if (p.rope_dim > 0 && !p.rope_keys_rotated) return ATTN_ERR_UNSUPPORTED;  // pool keys rotated
+  if (!rope_ready(c)) return ATTN_ERR_INVALID_ARG;
+  const bool need_q = p.q_len > 0, need_kv = p.kv_len > 0;
+  if (bad_ptr(q, need_q) || bad_ptr(k_pool, need_kv) || bad_ptr(v_pool, need_kv) ||
+      bad_qbufs(p, qb) ||
+      (need_kv && (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u))) ||
+      (need_kv && num_blocks < 1))
+    return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const KvBlocks src{block_table, ceil_div(p.kv_len, 128), p.n_kv_heads, num_blocks, c->err};
+  return mark_done(c, quantize_units(c, 0, c->units, q, k_pool, v_pool, qb, st, src), st);
 }
 
 attn_status attn_forward(attn_ctx* c, const void* q, const void* k, const void* v,

@@ -90,6 +90,32 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 // its chunks (reading the partner chunk of the pairs from shared memory), keeps
 // the rotated floats in registers, and the maximum and the codes are those of
 // the rotated values.  The extra registers leave room for fewer CTAs per SM.
+// Where the 128-token blocks of a key or value tensor live: dense [units][S][D]
+// (table == nullptr), or a paged pool [num_blocks][n_kv_heads][128][D] in which block
+// table[b * bt_stride + t] holds tokens 128 t .. 128 t + 127 of batch entry b (unit
+// u = b * n_kv_heads + h).  A block is contiguous either way.  A table entry outside
+// [0, num_blocks) is read as block 0 and flagged (kErrBadBlock in *err): nothing is
+// read outside the pool.
+struct KvBlocks {
+  const int* table;
+  int bt_stride;
+  int n_kv_heads;
+  int num_blocks;
+  unsigned* err;
+  template <int D>
+  __device__ __forceinline__ const uint16_t* block(const uint16_t* base, size_t u, int t,
+                                                   int S) const {
+    if (table == nullptr) return base + (u * S + static_cast<size_t>(t) * 128) * D;
+    const int b = static_cast<int>(u / n_kv_heads), h = static_cast<int>(u % n_kv_heads);
+    int blk = __ldg(table + static_cast<size_t>(b) * bt_stride + t);
+    if (blk < 0 || blk >= num_blocks) {
+      atomicOr(err, (unsigned)kErrBadBlock);
+      blk = 0;
+    }
+    return base + (static_cast<size_t>(blk) * n_kv_heads + h) * 128 * D;
+  }
+};
+
 template <int D, bool ROPE = false>
 struct QuantQkCfg {
   static constexpr int kBlockBytes = 128 * D * 2;
@@ -108,7 +134,7 @@ struct QuantRope {
 template <int D, bool F16, bool ROPE = false>
 __global__ void __launch_bounds__(256, QuantQkCfg<D, ROPE>::kCtasPerSm) quant_qk_kernel(
     const uint16_t* __restrict__ x, int8_t* __restrict__ codes, float* __restrict__ scales, int S,
-    int nblk, int total, unsigned* err, unsigned debug, QuantRope rope) {
+    int nblk, int total, unsigned* err, unsigned debug, QuantRope rope, KvBlocks src) {
   using C = QuantQkCfg<D, ROPE>;
   constexpr int kChunks = 128 * D / 8;  // 16-byte chunks of a full block
   constexpr int kPer = kChunks / 256;
@@ -133,8 +159,7 @@ __global__ void __launch_bounds__(256, QuantQkCfg<D, ROPE>::kCtasPerSm) quant_qk
     const int t = b % nblk;
     const uint32_t bytes = block_bytes(b);
     mbar_arrive_expect_tx(bar0 + 8 * stage, bytes);
-    bulk_load(sbase + stage * C::kBlockBytes, x + (bh * S + (size_t)t * 128) * D, bytes,
-              bar0 + 8 * stage);
+    bulk_load(sbase + stage * C::kBlockBytes, src.block<D>(x, bh, t, S), bytes, bar0 + 8 * stage);
   };
   if (threadIdx.x == 0) {
     if (blockIdx.x < total) issue(blockIdx.x, 0);
@@ -330,7 +355,8 @@ constexpr int kVTok = 256;
 
 template <int D, bool F16>
 __global__ void __launch_bounds__(256) v_amax_kernel(const uint16_t* __restrict__ v,
-                                                     unsigned* __restrict__ amax_bits, int S) {
+                                                     unsigned* __restrict__ amax_bits, int S,
+                                                     KvBlocks src) {
   constexpr int kCC = D / 8;            // 16-byte chunks per token
   constexpr int kRows = 256 / kCC;      // tokens covered per pass
   __shared__ unsigned smax[D];
@@ -344,7 +370,7 @@ __global__ void __launch_bounds__(256) v_amax_kernel(const uint16_t* __restrict_
     const int tok = tok0 + tk;
     if (tok < S) {
       float f[8];
-      unpack8<F16>(ld_nc_v4(v + ((u * S + tok) * D + cc * 8)), f);
+      unpack8<F16>(ld_nc_v4(src.block<D>(v, u, tok / 128, S) + (tok % 128) * D + cc * 8), f);
 #pragma unroll
       for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
     }
@@ -379,7 +405,7 @@ template <int D, bool F16>
 __global__ void __launch_bounds__(256, VQuantCfg<D>::kCtasPerSm)
     v_quant_kernel(const uint16_t* __restrict__ v, const unsigned* __restrict__ amax_bits,
                    uint8_t* __restrict__ vt, float* __restrict__ v_scale, int S, int S_pad,
-                   int nbk, int total, unsigned* err) {
+                   int nbk, int total, unsigned* err, KvBlocks src) {
   using C = VQuantCfg<D>;
   extern __shared__ __align__(128) uint8_t vsm[];
   const uint32_t sbase = smem_u32(vsm);
@@ -397,7 +423,7 @@ __global__ void __launch_bounds__(256, VQuantCfg<D>::kCtasPerSm)
     const int t = b % nbk;
     const uint32_t bytes = (uint32_t)(min(128, S - t * 128) * D * 2);
     mbar_arrive_expect_tx(bar0 + 8 * stage, bytes);
-    bulk_load(sbase + stage * C::kTileBytes, v + (u * S + (size_t)t * 128) * D, bytes,
+    bulk_load(sbase + stage * C::kTileBytes, src.block<D>(v, u, t, S), bytes,
               bar0 + 8 * stage);
   };
   if (threadIdx.x == 0) {

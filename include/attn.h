@@ -188,6 +188,21 @@ attn_status attn_create(const attn_params *p, attn_ctx **out);
 attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const void *v,
                              const attn_qbufs *qb, void *stream);
 
+/* ATTN_INT8QK_FP8PV with a paged key/value cache: attn_quantize_qk with K and V read
+ * from the pools of attn_forward_paged ([num_blocks][n_kv_heads][128][head_dim], 16-bit;
+ * block_table [batch][ceil(kv_len / 128)] int32, device) and Q dense as usual.  The
+ * buffers *qb it writes are those of the dense layout, bit-identical to
+ * attn_quantize_qk's on the gathered keys and values (positions past kv_len in a
+ * block are not read); attn_forward(c, NULL, NULL, NULL, qb, o, lse, stream) then
+ * runs the quantised attention.  A table entry outside [0, num_blocks) is read as
+ * block 0 and makes the next attn_get_error return ATTN_ERR_INVALID_ARG.  With RoPE the pool's keys must be rotated already
+ * (rope_keys_rotated).  Errors: ATTN_ERR_INVALID_ARG (as attn_quantize_qk; NULL or
+ * misaligned block_table, num_blocks < 1), ATTN_ERR_UNSUPPORTED (another precision,
+ * or RoPE on unrotated keys). */
+attn_status attn_quantize_qk_paged(attn_ctx *c, const void *q, const void *k_pool,
+                                   const void *v_pool, const int32_t *block_table,
+                                   int num_blocks, const attn_qbufs *qb, void *stream);
+
 /* The attention forward.  Exact mode: q, k, v are read and qb must be NULL.
  * Quantised mode: q, k, v are ignored (may be NULL) and qb holds the output of
  * attn_quantize_qk.  Diagonal band mode: qb as in the quantised mode, and q and k
@@ -308,8 +323,9 @@ attn_status attn_rope_apply(attn_ctx *c, const void *x, void *y, int n_heads, in
                             void *stream);
 
 /* Synchronises `stream`, reads and clears the context's device error word.
- * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last call,
- * ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK. */
+ * Returns ATTN_ERR_INVALID_ARG if attn_quantize_qk_paged met a block-table entry
+ * outside the pool since the last call, ATTN_ERR_TIMEOUT if a kernel gave up on a
+ * wait, ATTN_ERR_CUDA if the stream reports an error, else ATTN_OK. */
 attn_status attn_get_error(attn_ctx *c, void *stream);
 
 /* Waits for the context's own work (its last call, recorded on that call's

@@ -79,6 +79,7 @@ def test_null_arguments():
     assert L.attn_debug_set(None, 0) == _abi.ATTN_ERR_INVALID_ARG
     assert L.attn_num_splits(None) == 0
     assert L.attn_kernel_path(None) == 0
+    assert L.attn_quantize_qk_paged(*([None] * 5), 0, None, None) == _abi.ATTN_ERR_INVALID_ARG
     L.attn_destroy(None)
 
 
@@ -133,6 +134,7 @@ int main(void) {
   attn_qbufs_sf_sizes(&p, sizes);
   attn_num_splits(c);
   if (attn_kernel_path(c) == ATTN_PATH_DECODE) return 2;
+  attn_quantize_qk_paged(c, NULL, NULL, NULL, table, 1, &qb, NULL);
   attn_plan plan;
   if (attn_plan_for(&p, 148, &plan) != ATTN_OK || plan.path != ATTN_PATH_SINGLE_PASS) return 3;
   attn_debug_set(c, 0u);

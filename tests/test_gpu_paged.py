@@ -110,3 +110,76 @@ def test_paged_argument_errors():
     assert L.attn_forward_paged(att.ctx, P(qd), P(kd), P(vd), P(td), kd.shape[0], P(o), None,
                                 s) == _abi.ATTN_OK
     att.check_error()
+
+
+QUANT_CASES = [
+    Workload("pq_gqa_causal", 2, 8, 2, 300, 1291, 128, "bf16", causal=True, start_pos=991,
+             seed=7201),
+    Workload("pq_d64", 1, 4, 4, 256, 1000, 64, "fp16", seed=7202),
+    Workload("pq_decode", 2, 16, 8, 4, 4133, 128, "fp16", causal=True, start_pos=4129,
+             seed=7203),
+]
+
+
+@pytest.mark.parametrize("w", QUANT_CASES, ids=[w.name for w in QUANT_CASES])
+def test_paged_quantised_mode(w):
+    """The INT8 mode on a paged cache: the quantisers read K and V through the block
+    table (``attn_quantize_qk_paged``) and write the same codes and scales as on the
+    gathered dense tensors, bit for bit (the pool's filler past kv_len is never read);
+    the attention on them is identical and within the quantised mode's tolerance of
+    the oracle."""
+    from parity_util import QUANT_RMSE, rel_rmse
+    q, k, v = make_qkv(w)
+    kp, vp, table = _paged(k, v, w.seed)
+    att = _att(w, precision="quant")
+    qd = q.cuda()
+    dense = att.quantize(qd, k.cuda(), v.cuda())
+    paged = att.quantize_paged(qd, kp.cuda(), vp.cuda(), table.cuda())
+    att.check_error()
+    for f in ("q", "k", "q_scale", "k_scale", "v_t", "v_scale"):
+        _same(getattr(paged, f).cpu(), getattr(dense, f).cpu(), f"{w.name}: {f}")
+    o_p = att.forward(qbufs=paged)
+    o_d = att.forward(qbufs=dense)
+    att.check_error()
+    _same(o_p.cpu(), o_d.cpu(), f"{w.name}: O")
+    ro, _ = oracle_for(w, q, k, v)
+    assert rel_rmse(o_p.double().cpu().numpy(), ro) <= QUANT_RMSE
+
+
+def test_paged_quantiser_argument_errors():
+    w = QUANT_CASES[1]
+    q, k, v = make_qkv(w)
+    kp, vp, table = _paged(k, v, 1)
+    L = _abi.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    qd, kd, vd, td = q.cuda(), kp.cuda(), vp.cuda(), table.cuda()
+    att = _att(w, precision="quant")
+    qb = att.quantize(qd, k.cuda(), v.cuda())
+    P = lambda t: t.data_ptr()  # noqa: E731
+    import ctypes
+    qbs = qb.struct()
+    st = ctypes.byref(qbs)
+    assert L.attn_quantize_qk_paged(att.ctx, P(qd), P(kd), P(vd), None, kd.shape[0], st,
+                                    s) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_quantize_qk_paged(att.ctx, P(qd), P(kd), P(vd), P(td), 0, st,
+                                    s) == _abi.ATTN_ERR_INVALID_ARG
+    exact = _att(w)
+    assert L.attn_quantize_qk_paged(exact.ctx, P(qd), P(kd), P(vd), P(td), kd.shape[0], st,
+                                    s) == _abi.ATTN_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        exact.quantize_paged(qd, kd, vd, td)
+    assert L.attn_quantize_qk_paged(att.ctx, P(qd), P(kd), P(vd), P(td), kd.shape[0], st,
+                                    s) == _abi.ATTN_OK
+    att.check_error()
+    # a table entry past the pool is read as block 0 and reported by attn_get_error
+    bad = td.clone()
+    bad[0, 0] = kd.shape[0]
+    assert L.attn_quantize_qk_paged(att.ctx, P(qd), P(kd), P(vd), P(bad), kd.shape[0], st,
+                                    s) == _abi.ATTN_OK
+    assert L.attn_get_error(att.ctx, s) == _abi.ATTN_ERR_INVALID_ARG
+    assert L.attn_get_error(att.ctx, s) == _abi.ATTN_OK
+    bad[0, 0] = -1
+    assert L.attn_quantize_qk_paged(att.ctx, P(qd), P(kd), P(vd), P(bad), kd.shape[0], st,
+                                    s) == _abi.ATTN_OK
+    assert L.attn_get_error(att.ctx, s) == _abi.ATTN_ERR_INVALID_ARG
+    att.check_error()
