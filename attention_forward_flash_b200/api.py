@@ -145,16 +145,29 @@ class Attention:
                 _abi.ATTN_PATH_SINGLE_PASS_TAIL: "single_pass_tail"}[
                     _abi.attn_kernel_path(self.ctx)]
 
+    def _check_tensor(self, name, t, shape, dtype, on_cuda=True):
+        where = "CUDA" if on_cuda else "host"
+        if (tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous()
+                or t.is_cuda != on_cuda):
+            raise ValueError(f"{name}: expected contiguous {where} {dtype} of shape "
+                             f"{shape}, got {t.dtype} {tuple(t.shape)} on {t.device}")
+
     def _check_inputs(self, q, k, v, on_cuda=True):
         p = self.params
         want_q = (p.batch, p.n_q_heads, p.q_len, p.head_dim)
         want_kv = (p.batch, p.n_kv_heads, p.kv_len, p.head_dim)
-        where = "CUDA" if on_cuda else "host"
         for name, t, shape in (("q", q, want_q), ("k", k, want_kv), ("v", v, want_kv)):
-            if (tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous()
-                    or t.is_cuda != on_cuda):
-                raise ValueError(f"{name}: expected contiguous {where} {self.dtype} of shape "
-                                 f"{shape}, got {t.dtype} {tuple(t.shape)} on {t.device}")
+            self._check_tensor(name, t, shape, self.dtype, on_cuda)
+
+    def _check_outputs(self, out, lse, on_cuda=True):
+        """A caller's O [B, Hq, Sq, D] (the context's dtype) and lse [B, Hq, Sq] (float32)."""
+        p = self.params
+        if out is not None:
+            self._check_tensor("out", out, (p.batch, p.n_q_heads, p.q_len, p.head_dim),
+                               self.dtype, on_cuda)
+        if lse is not None:
+            self._check_tensor("lse", lse, (p.batch, p.n_q_heads, p.q_len), torch.float32,
+                               on_cuda)
 
     def quantize(self, q, k, v, qbufs=None, stream=None):
         if self.precision == "exact":
@@ -165,8 +178,9 @@ class Attention:
                               _stream_handle(stream))
         return qbufs
 
-    def _check_pools(self, k_pool, v_pool, block_table):
+    def _check_pools(self, q, k_pool, v_pool, block_table):
         p = self.params
+        self._check_tensor("q", q, (p.batch, p.n_q_heads, p.q_len, p.head_dim), self.dtype)
         want = (p.n_kv_heads, 128, p.head_dim)
         for name, t in (("k_pool", k_pool), ("v_pool", v_pool)):
             if (t.dim() != 4 or tuple(t.shape[1:]) != want or t.dtype != self.dtype
@@ -186,7 +200,7 @@ class Attention:
         ``forward(qbufs=...)`` takes."""
         if self.precision != "quant":
             raise ValueError("quantize_paged() needs precision='quant'")
-        self._check_pools(k_pool, v_pool, block_table)
+        self._check_pools(q, k_pool, v_pool, block_table)
         qbufs = qbufs if qbufs is not None else QuantBuffers(self.params, q.device)
         _abi.attn_quantize_qk_paged(self.ctx, q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
                                     block_table.data_ptr(), k_pool.shape[0], qbufs.struct(),
@@ -197,6 +211,7 @@ class Attention:
                 stream=None):
         p = self.params
         device = (q if q is not None else qbufs.q).device
+        self._check_outputs(out, lse)
         if out is None:
             out = torch.empty((p.batch, p.n_q_heads, p.q_len, p.head_dim), dtype=self.dtype,
                               device=device)
@@ -233,7 +248,8 @@ class Attention:
         if self.precision != "exact":
             raise ValueError("forward_paged() needs precision='exact' (the INT8 mode: "
                              "quantize_paged(), then forward(qbufs=...))")
-        self._check_pools(k_pool, v_pool, block_table)
+        self._check_pools(q, k_pool, v_pool, block_table)
+        self._check_outputs(out, lse)
         if out is None:
             out = torch.empty((p.batch, p.n_q_heads, p.q_len, p.head_dim), dtype=self.dtype,
                               device=q.device)
@@ -259,6 +275,7 @@ class Attention:
         """
         p = self.params
         self._check_inputs(q, k, v, on_cuda=False)
+        self._check_outputs(out, lse, on_cuda=False)
         want_lse = return_lse or lse is not None
         if staging is None:
             cached = getattr(self, "_staging", None)

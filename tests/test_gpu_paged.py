@@ -168,6 +168,13 @@ def test_paged_quantiser_argument_errors():
                                     s) == _abi.ATTN_ERR_UNSUPPORTED
     with pytest.raises(ValueError):
         exact.quantize_paged(qd, kd, vd, td)
+    # the binding checks q and the caller's output buffers before any call
+    with pytest.raises(ValueError):
+        att.quantize_paged(qd[:, :1], kd, vd, td)
+    with pytest.raises(ValueError):
+        exact.forward_paged(qd, kd, vd, td, out=torch.empty_like(qd, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        att.forward(qbufs=qb, lse=torch.empty(1, device="cuda"))
     assert L.attn_quantize_qk_paged(att.ctx, P(qd), P(kd), P(vd), P(td), kd.shape[0], st,
                                     s) == _abi.ATTN_OK
     att.check_error()
