@@ -188,17 +188,21 @@ attn_status attn_create(const attn_params *p, attn_ctx **out);
 attn_status attn_quantize_qk(attn_ctx *c, const void *q, const void *k, const void *v,
                              const attn_qbufs *qb, void *stream);
 
-/* ATTN_INT8QK_FP8PV with a paged key/value cache: attn_quantize_qk with K and V read
- * from the pools of attn_forward_paged ([num_blocks][n_kv_heads][128][head_dim], 16-bit;
- * block_table [batch][ceil(kv_len / 128)] int32, device) and Q dense as usual.  The
- * buffers *qb it writes are those of the dense layout, bit-identical to
- * attn_quantize_qk's on the gathered keys and values (positions past kv_len in a
- * block are not read); attn_forward(c, NULL, NULL, NULL, qb, o, lse, stream) then
- * runs the quantised attention.  A table entry outside [0, num_blocks) is read as
- * block 0 and makes the next attn_get_error return ATTN_ERR_INVALID_ARG.  With RoPE the pool's keys must be rotated already
- * (rope_keys_rotated).  Errors: ATTN_ERR_INVALID_ARG (as attn_quantize_qk; NULL or
- * misaligned block_table, num_blocks < 1), ATTN_ERR_UNSUPPORTED (another precision,
- * or RoPE on unrotated keys). */
+/* ATTN_INT8QK_FP8PV with a paged key/value cache (the qsa2 audit's decode workload
+ * runs on a 32768-cell KV cache; the paging is as in attn_forward_paged below):
+ * attn_quantize_qk with K and V read from the pools of attn_forward_paged
+ * ([num_blocks][n_kv_heads][128][head_dim], 16-bit; block_table
+ * [batch][ceil(kv_len / 128)] int32, device) and Q dense as usual.  The buffers *qb
+ * it writes are those of the dense layout, bit-identical to attn_quantize_qk's on
+ * the gathered keys and values (positions past kv_len in a block are not read);
+ * attn_forward(c, NULL, NULL, NULL, qb, o, lse, stream) then runs the quantised
+ * attention.  V's scale is per channel over the whole sequence, so each call
+ * quantises the whole cache.  A table entry outside [0, num_blocks) is read as
+ * block 0 and makes the next attn_get_error return ATTN_ERR_INVALID_ARG.  With RoPE
+ * the pool's keys must be rotated already (rope_keys_rotated).
+ * Errors: ATTN_ERR_INVALID_ARG (as attn_quantize_qk; NULL or misaligned
+ * block_table, num_blocks < 1), ATTN_ERR_UNSUPPORTED (another precision, or RoPE on
+ * unrotated keys), ATTN_ERR_CUDA (launch failure). */
 attn_status attn_quantize_qk_paged(attn_ctx *c, const void *q, const void *k_pool,
                                    const void *v_pool, const int32_t *block_table,
                                    int num_blocks, const attn_qbufs *qb, void *stream);
@@ -277,7 +281,8 @@ attn_status attn_forward_host(attn_ctx *c, const void *q_host, const void *k_hos
  * memory outside the pool.  The positions past kv_len in a batch entry's last
  * block must hold finite values.
  * Errors: ATTN_ERR_INVALID_ARG (NULL or misaligned pointer, num_blocks < 1),
- * ATTN_ERR_UNSUPPORTED (quantised mode), ATTN_ERR_CUDA (tensor-map encode or
+ * ATTN_ERR_UNSUPPORTED (a quantised mode: the INT8 mode reads a paged cache through
+ * attn_quantize_qk_paged, then attn_forward), ATTN_ERR_CUDA (tensor-map encode or
  * launch failure). */
 attn_status attn_forward_paged(attn_ctx *c, const void *q, const void *k_pool,
                                const void *v_pool, const int32_t *block_table, int num_blocks,
