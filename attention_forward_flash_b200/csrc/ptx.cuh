@@ -14,7 +14,6 @@ namespace attn {
 
 constexpr uint64_t kWaitTimeoutNs = 1500ull * 1000ull * 1000ull;  // 1.5 s
 constexpr int kErrTimeout = 1;  // error word bit: a bounded wait ran out
-constexpr int kErrBadBlock = 2;  // error word bit: a block-table entry outside the pool
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

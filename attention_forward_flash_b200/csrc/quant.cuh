@@ -96,6 +96,7 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 // u = b * n_kv_heads + h).  A block is contiguous either way.  A table entry outside
 // [0, num_blocks) is read as block 0 and flagged (kErrBadBlock in *err): nothing is
 // read outside the pool.
+constexpr int kErrBadBlock = 2;  // error word bit (beside kErrTimeout)
 struct KvBlocks {
   const int* table;
   int bt_stride;
