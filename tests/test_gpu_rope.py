@@ -11,7 +11,8 @@
   float64 attention on the float64-rotated inputs at the usual tolerances (the
   oracle's table as input; one case with the library's own table); keys rotated
   once into a cache (rope_keys_rotated) and a paged cache give the same bits as
-  rotating inside the forward; the host-buffer pipeline is bit-identical.
+  rotating inside the forward; the INT8 mode on such a cache rotates only Q, dense
+  and paged alike; the host-buffer pipeline is bit-identical.
 """
 
 import numpy as np
@@ -198,6 +199,52 @@ def test_keys_rotated_once_into_a_cache_and_paged():
     o_p = cached.forward_paged(q, pool_k, pool_v, table_b)
     cached.check_error()
     assert torch.equal(o_p, o_ref)
+
+
+def test_quantised_mode_on_keys_rotated_once_dense_and_paged():
+    """INT8 mode on a cache of keys rotated once (rope_keys_rotated): the quantiser
+    rotates Q only and takes the cached keys as they are.  Q's codes and scales are
+    those of the mode that rotates both; K's are the oracle quantiser's on the cached
+    keys; the paged quantiser's buffers equal the dense ones bit for bit; the attention
+    is within the quantised tolerance of the float64 definition."""
+    w = Workload("cacheq", 2, 16, 8, 4, 2000, 128, "bf16", causal=True, start_pos=1996,
+                 seed=8401)
+    q, k, v = make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    table = rope_table(128, 2000, scaling="yarn", factor=4.0, original_len=1024)
+    both = _att(w, precision="quant", table=table)
+    qb_both = both.quantize(qd, kd, vd)
+    both.check_error()
+    cached = _att(w, precision="quant", keys_rotated=True, table=table)
+    k_rot = cached.rope_apply(kd, pos0=0)
+    dense = cached.quantize(qd, k_rot, vd)
+    cached.check_error()
+    assert torch.equal(dense.q, qb_both.q) and torch.equal(dense.q_scale, qb_both.q_scale)
+    rk, rks = quantize_qk_int8(k_rot.float().cpu().numpy())
+    assert np.array_equal(dense.k.cpu().numpy(), rk)
+    assert np.array_equal(dense.k_scale.cpu().numpy().view(np.uint32), rks.view(np.uint32))
+    # the same cache as a paged pool (blocks of 128 positions, shuffled)
+    nblk = (2000 + 127) // 128
+    perm = torch.randperm(w.batch * nblk, generator=torch.Generator().manual_seed(6))
+    pool_k = torch.zeros((w.batch * nblk + 3, 8, 128, 128), dtype=k.dtype, device="cuda")
+    pool_v = torch.zeros_like(pool_k)
+    table_b = perm.view(w.batch, nblk).int().cuda()
+    for b in range(w.batch):
+        for t in range(nblk):
+            n = min(128, 2000 - 128 * t)
+            pool_k[table_b[b, t], :, :n] = k_rot[b, :, 128 * t:128 * t + n]
+            pool_v[table_b[b, t], :, :n] = vd[b, :, 128 * t:128 * t + n]
+    paged = cached.quantize_paged(qd, pool_k, pool_v, table_b)
+    cached.check_error()
+    for f in ("q", "k", "q_scale", "k_scale", "v_t", "v_scale"):
+        assert torch.equal(getattr(paged, f), getattr(dense, f)), f
+    o = cached.forward(qbufs=paged)
+    cached.check_error()
+    assert torch.equal(o, cached.forward(qbufs=dense))
+    theta, m = _theta_m(128, "yarn", original_len=1024)
+    ro, _ = _oracle_rope_attention(w, q, k, v, theta, m, False)
+    e = rel_rmse(o.double().cpu().numpy(), ro)
+    assert e <= QUANT_RMSE, f"{e:.3e}"
 
 
 @pytest.mark.parametrize("precision", ["exact", "quant"])
