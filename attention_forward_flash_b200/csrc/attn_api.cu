@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -474,6 +476,17 @@ attn_status validate(const attn_params* p) {
   const long long rows = static_cast<long long>(p->n_q_heads / p->n_kv_heads) * p->q_len;
   if (rows > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->start_pos) + p->q_len > (1ll << 30)) return ATTN_ERR_UNSUPPORTED;
+  // Grid and block counts are 32-bit: the (batch, kv head) units times their row tiles
+  // and splits, and the quantisers' 128-token blocks of all heads.
+  const long long units = static_cast<long long>(p->batch) * p->n_kv_heads;
+  const long long row_tiles = std::max(1ll, (rows + 127) / 128);
+  if (units * row_tiles * std::max(1, p->num_splits) > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+  const long long nbq = (p->q_len + 127ll) / 128, nbk = (p->kv_len + 127ll) / 128;
+  if (static_cast<long long>(p->batch) * p->n_q_heads * nbq > INT_MAX ||
+      units * nbk > INT_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  // the quantisers run the units along gridDim.y (at most 65535)
+  if (p->precision != ATTN_EXACT && units > 65535) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 

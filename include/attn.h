@@ -168,7 +168,11 @@ typedef struct attn_ctx attn_ctx;
  * with RoPE on unrotated keys a buffer of K's size for the rotated keys).  On
  * success *out owns that workspace until attn_destroy().  Launches nothing.
  * Errors: ATTN_ERR_INVALID_ARG (bad field or NULL), ATTN_ERR_UNSUPPORTED
- * (head_dim not 64/128), ATTN_ERR_CUDA (no device), ATTN_ERR_OOM. */
+ * (head_dim not 64/128; the FP4 mode at head_dim 128 or with RoPE; the diagonal
+ * band mode with RoPE; more than 2^30 stacked rows per kv head or positions past
+ * 2^30; batch * n_kv_heads above 65535 in a quantised mode; a problem whose CTA or
+ * 128-token block count passes 2^31 - 1; a device other than sm_100),
+ * ATTN_ERR_CUDA (no device), ATTN_ERR_OOM. */
 attn_status attn_create(const attn_params *p, attn_ctx **out);
 
 /* Quantised, diagonal band and FP4 modes, step 1 (the quantisers): reads q, k, v (dtype of

@@ -57,6 +57,16 @@ def _params(**kw):
     (dict(precision=3, num_splits=2), _abi.ATTN_ERR_INVALID_ARG),    # single-pass modes
     (dict(precision=2, num_splits=2), _abi.ATTN_ERR_INVALID_ARG),
     (dict(precision=2, rope_dim=64), _abi.ATTN_ERR_UNSUPPORTED),
+    # size limits: stacked rows and positions below 2^30, 32-bit grid and block counts,
+    # and the quantisers' units on gridDim.y
+    (dict(n_q_heads=64, n_kv_heads=1, q_len=1 << 25), _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(start_pos=(1 << 30) - 100, q_len=101), _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(batch=1 << 20, n_q_heads=1 << 11, n_kv_heads=1 << 11, q_len=1),
+     _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(batch=1 << 16, n_q_heads=1 << 8, n_kv_heads=1 << 8, q_len=1, kv_len=1 << 16),
+     _abi.ATTN_ERR_UNSUPPORTED),
+    (dict(precision=1, batch=65536, n_q_heads=1, n_kv_heads=1, q_len=16, kv_len=16),
+     _abi.ATTN_ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_params_before_any_device_call(kw, status):
     L = afb.lib()
